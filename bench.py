@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the token-choice MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config mixtral|switch|deepseekmoe|deepseek_v3|tiny]
+
+One step = one forward of the whole layer (route, capacity, dispatch, expert
+FFNs, combine, losses) over one batch of T synthetic tokens.  The default
+workload is the Mixtral-shaped layer (T=8192, d=4096, E=8 SwiGLU experts with
+d_ff=14336, top-2, cf=1.25): it is the layer the headline targets name.  With
+N > 1 (torchrun, one process per GPU) every rank runs an independent replica
+on its own batch: the layer needs no exchange between GPUs, so the scaling is
+weak and no collective touches the data path; the per-step time is the max
+over ranks.
+
+Rank 0 prints one JSON line.  `value` is device-timed (CUDA events, inputs
+resident in HBM); `e2e` repeats the measurement with the step's input copied
+from pinned host memory and the result read back inside the timed region;
+`roofline` covers the dominant stage (the expert FFN: two grouped tcgen05
+GEMMs) from its own CUDA events in the same timed region; `cpu_baseline` times
+the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+from moe_inputs import CONFIGS, generate, seed_for  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s on 1 B200; grouped-GEMM % BF16 peak; dispatch % HBM BW"
+UNIT = "tokens/s"
+KERNELS_PER_STEP = 9   # route 1, capacity 3, dispatch 1, expert FFN 2, combine 1, losses 1
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Slowest rank's time (every rank calls this the same number of times)."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        time.sleep(0.1)
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [s.strip() for s in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, flag in zip(names, f[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ work accounting
+
+def layer_work(shape, counts, kept_total, dropped_tokens):
+    """Algorithmic FLOPs and bytes of one step (no padding rows, no dense E-way
+    work), per stage."""
+    T, d, E, k, F = shape.T, shape.d, shape.E, shape.k, shape.d_ff
+    b = 2 if shape.dtype == 1 else 4
+    m = 3 if shape.act == 1 else 2
+    S, Fs = shape.n_shared, shape.d_ff_shared
+    N = kept_total
+    ffn_flops = 2.0 * m * N * d * F + 2.0 * m * S * T * d * Fs
+    w_bytes = (E * m * d * F + S * m * d * Fs) * b
+    ffn_bytes = w_bytes + (N + (T if S else 0)) * d * b * 2 + (N + S * T) * F * b * 2
+    routed_tokens = T - dropped_tokens
+    return {
+        "route": {"bytes": T * d * b + d * E * 4 + T * k * 8 + math.ceil(T / 32) * (E + 1) * 4,
+                  "flops": 2.0 * T * d * E},
+        "dispatch": {"bytes": routed_tokens * d * b + N * d * b + T * k * 9},
+        "expert_ffn": {"flops": ffn_flops, "bytes": ffn_bytes},
+        "combine": {"bytes": N * d * b + (T * d * b if S else 0) + T * d * b + T * k * 9},
+        "capacity": {"bytes": T * k * 4 * 3 + T * k + T},
+        "losses": {"bytes": math.ceil(T / 32) * (E + 1) * 4 + E * 4},
+    }
+
+
+# ------------------------------------------------------------ oracle timing
+
+def oracle_inputs(inp):
+    import numpy as np
+
+    def host(t):
+        if t is None:
+            return None
+        t = t.detach().contiguous().cpu()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16)
+        return t.numpy()
+    return {k: host(getattr(inp, k)) for k in
+            ("x", "W_r", "logit_bias", "select_bias", "W1", "W3", "W2", "Ws1", "Ws3", "Ws2")}
+
+
+def time_oracle(shape, h, n_tokens):
+    """Oracle routing, capacity and losses over all T tokens plus the expert
+    FFNs of the first n_tokens tokens; returns (t_route_s, t_ffn_s)."""
+    import numpy as np
+    import oracle
+    t0 = time.perf_counter()
+    r = oracle.route(h["x"], h["W_r"], shape.k, shape.score, shape.renorm, h["logit_bias"],
+                     h["select_bias"])
+    cap = oracle.capacity_walk(r.topk, shape.E, shape.cf, shape.priority)
+    oracle.losses(r.scores, cap.counts, r.lse, shape.k, shape.score)
+    t1 = time.perf_counter()
+    tokens = np.arange(n_tokens, dtype=np.int32)
+    oracle.ffn_tokens(h["x"], r.topk, r.gates, cap.keep, h["W1"], h["W3"], h["W2"], shape.act,
+                      h["Ws1"], h["Ws3"], h["Ws2"], tokens)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1
+
+
+def size_oracle_sample(shape, h, seconds):
+    """Tokens whose FFNs take about `seconds` on the host cores."""
+    _, t4 = time_oracle(shape, h, 4)
+    per = max(t4 / 4, 1e-6)
+    return int(max(4, min(shape.T, seconds / per)))
+
+
+def cpu_baseline(shape, inp, seconds):
+    import oracle
+    h = oracle_inputs(inp)
+    n = size_oracle_sample(shape, h, seconds)
+    t_route, t_ffn = time_oracle(shape, h, n)
+    per_token = t_route / shape.T + t_ffn / n
+    return {"value": 1.0 / per_token, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"routing, capacity and losses over all {shape.T} tokens "
+                       f"({t_route:.2f} s) plus expert FFNs of {n} tokens ({t_ffn:.2f} s), "
+                       f"per-token cost extrapolated to the full batch")}
+
+
+def workload_name(shape):
+    act = "SwiGLU" if shape.act == 1 else "GELU"
+    sh = f" + {shape.n_shared} shared (d_ff={shape.d_ff_shared})" if shape.n_shared else ""
+    sc = "sigmoid+selection bias" if shape.score == 1 else "softmax"
+    cf = "no capacity" if math.isinf(shape.cf) else f"cf={shape.cf}"
+    return (f"{shape.name} MoE layer fwd: T={shape.T} d={shape.d} E={shape.E} {act} experts "
+            f"d_ff={shape.d_ff}{sh}, top-{shape.k} {sc}, {cf}")
+
+
+# ------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    shape = CONFIGS[args.config]
+    inp = generate(shape, device="cpu")
+    h = oracle_inputs(inp)
+    n = size_oracle_sample(shape, h, 1.0)
+    for _ in range(args.warmup):
+        time_oracle(shape, h, n)
+    tr = tf = 0.0
+    for _ in range(args.steps):
+        a, b = time_oracle(shape, h, n)
+        tr += a
+        tf += b
+    per_token = (tr / args.steps) / shape.T + (tf / args.steps) / n
+    value = 1.0 / per_token
+    sample = (f"each step: oracle routing, capacity and losses over all {shape.T} tokens plus "
+              f"expert FFNs of {n} tokens, per-token cost extrapolated to the full batch")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * shape.T / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_name(shape), "global_batch": shape.T,
+                       "parallelism": "none (host cores)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import mixture_experts_layer_54_b200 as moe
+
+    world, rank, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    shape = CONFIGS[args.config]
+    inp = generate(shape, device=dev, seed=seed_for(shape) + 1000 * rank)
+    cfg = moe.moe_config(shape)
+    staged = moe.StagedForward(cfg, dev)
+    wargs = (inp.x, inp.W_r, inp.W1, inp.W2, inp.W3, inp.logit_bias, inp.select_bias, inp.Ws1,
+             inp.Ws3, inp.Ws2)
+    nst = len(moe.StagedForward.STAGES)
+
+    for _ in range(max(args.warmup, 3)):
+        staged(*wargs)
+    torch.cuda.synchronize()
+    kept_total = int(staged.kept.sum().item())
+    dropped_tokens = int(staged.dropped.sum().item())
+    status = moe.moe_device_status(staged.ws)
+
+    # ---- device-timed region: K steps, events between the stages ----
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+              for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            staged(*wargs, events=events[i])
+        torch.cuda.synchronize()
+    barrier(dev)
+    total_ms = events[0][0].elapsed_time(events[-1][-1])
+    stage_ms = [sum(ev[s].elapsed_time(ev[s + 1]) for ev in events) / args.steps
+                for s in range(nst)]
+    ms_per_step = max_over_ranks(total_ms / args.steps, dev)
+
+    # ---- end to end: pinned host input in, result out, inside the timed region ----
+    fwd = moe.MoEForward(cfg, dev, keep_routing=False)
+    w = moe.weights_struct(inp.W_r, inp.W1, inp.W2, inp.W3, inp.logit_bias, inp.select_bias,
+                           inp.Ws1, inp.Ws3, inp.Ws2)
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty(fwd.y.shape, dtype=fwd.y.dtype).pin_memory()
+    loss_host = torch.empty((2,), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    for _ in range(max(args.warmup, 3)):
+        x_dev.copy_(x_host, non_blocking=True)
+        fwd(x_dev, w)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        fwd(x_dev, w)
+        y_host.copy_(fwd.y, non_blocking=True)
+        loss_host[0:1].copy_(fwd.aux, non_blocking=True)
+        loss_host[1:2].copy_(fwd.zloss, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    work = layer_work(shape, None, kept_total, dropped_tokens)
+    tokens = shape.T * world
+    value = tokens / (ms_per_step / 1e3)
+    st = dict(zip(moe.StagedForward.STAGES, stage_ms))
+    stages = {}
+    for name, ms in st.items():
+        entry = {"us": round(ms * 1e3, 2)}
+        if "bytes" in work[name]:
+            entry["GB/s"] = round(work[name]["bytes"] / (ms / 1e3) / 1e9, 1)
+            entry["hbm_frac"] = round(entry["GB/s"] / peaks["hbm_gbs"], 3)
+        if "flops" in work[name]:
+            entry["TFLOP/s"] = round(work[name]["flops"] / (ms / 1e3) / 1e12, 1)
+        stages[name] = entry
+    ffn = work["expert_ffn"]
+    ach = ffn["flops"] / (st["expert_ffn"] / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
+                "traffic": None,
+                "kernel": "moe_expert_ffn: grouped tcgen05 GEMM1 (act fused) + GEMM2",
+                "flops_per_launch": ffn["flops"],
+                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
+                "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4)}
+    t_flop = ffn["flops"] / (peaks["bf16_tflops"] * 1e12)
+    all_bytes = sum(v.get("bytes", 0) for v in work.values())
+    t_byte = all_bytes / (peaks["hbm_gbs"] * 1e9)
+    layer_roof = {"t_flop_us": round(t_flop * 1e6, 1), "t_byte_us": round(t_byte * 1e6, 1),
+                  "bound": "tensor" if t_flop >= t_byte else "hbm",
+                  "frac": round(max(t_flop, t_byte) / (ms_per_step / 1e3), 4)}
+    b = 2 if shape.dtype == 1 else 4
+    h2d = shape.T * shape.d * b
+    d2h = shape.T * shape.d * b + 8
+    clocks = clk.summary()
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if shape.dtype == 1 else "f32", "data": "synthetic",
+            "config": {"workload": workload_name(shape), "global_batch": tokens,
+                       "tokens_per_gpu": shape.T, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (expert weights "
+                             f"{(shape.E * (3 if shape.act == 1 else 2) * shape.d * shape.d_ff * b) / 1e9:.2f} GB)",
+                       "kept_assignments": kept_total, "dropped_tokens": dropped_tokens},
+            "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "roofline": roofline, "layer_roofline": layer_roof, "stages": stages,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
+            "device_status": status}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(shape, inp, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,286 @@
+/*
+ * moe_b200.h - C ABI of the token-choice Mixture-of-Experts forward pass on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (page "Lab 18 - Mixture of experts", section 1):
+ *     z = x W_r,  p = softmax(z),  y = sum over top-k(p) of g_i FFN_i(x)
+ * plus the capacity limit of section 3, the balancing losses of section 2 and
+ * shared experts that run on every token.  Each stage is one call; moe_forward
+ * runs them all.
+ *
+ * Conventions for every call:
+ *   - Pointers named x, W*, y, ... are DEVICE pointers unless marked "host".
+ *     The caller allocates every buffer (including the workspace); the library
+ *     never allocates, frees or synchronises.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous to the host.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns a status and launches nothing.  A failed launch
+ *     returns MOE_ERR_CUDA.
+ *   - Row-major layouts throughout.  "dtype" is the activation / expert-weight
+ *     storage type chosen by moe_config.dtype: fp32, or bf16 (2-byte).  The
+ *     router weights, biases, gates and losses are always fp32.
+ *   - T = tokens, d = model dim, E = routed experts, k = experts per token,
+ *     F = expert hidden dim (d_ff), S = shared experts, Fs = their hidden dim.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_NULL = 1,            /* a required pointer is NULL */
+    MOE_ERR_SHAPE = 2,           /* T < 0, d < 1, k < 1, k > E, E > 256, k > 8, ... */
+    MOE_ERR_CAPACITY_FACTOR = 3, /* capacity_factor < 1.0 or NaN ("Lab 01" traps) */
+    MOE_ERR_ALIGN = 4,           /* a pointer or row pitch breaks the 16-byte rule */
+    MOE_ERR_WORKSPACE = 5,       /* workspace smaller than the size query says */
+    MOE_ERR_DTYPE = 6,           /* unknown dtype / activation / score code */
+    MOE_ERR_CUDA = 7,            /* a CUDA launch or attribute call failed */
+    MOE_ERR_DEVICE_TIMEOUT = 8   /* a kernel's bounded wait ran out (see moe_device_status) */
+} moe_status;
+
+enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 };
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+enum { MOE_PRIORITY_TOKEN = 0, MOE_PRIORITY_RANK = 1 };
+
+/* Every expert's segment of the permuted row buffers starts on a multiple of
+ * this many rows (the expert GEMM's M tile). */
+#define MOE_ROW_ALIGN 128
+
+/*
+ * One layer's shape and options.
+ *   act      MOE_ACT_GELU: two-matrix expert W2 gelu(W1 x), exact erf GELU;
+ *            MOE_ACT_SWIGLU: three-matrix W2 (silu(W1 x) * (W3 x))
+ *            ("Lab 18" section 1, expert description).
+ *   score    MOE_SCORE_SOFTMAX, or MOE_SCORE_SIGMOID (DeepSeek-V3 note of
+ *            "Lab 18" section 1; selection may add a per-expert bias).
+ *   renorm   -1: renormalize the gates over the selected experts exactly when
+ *            k > 1 (raw p for k = 1, "Lab 18" section 1 gate values); 0: raw;
+ *            1: renormalized.
+ *   dtype    MOE_DTYPE_F32 or MOE_DTYPE_BF16 for x, y and all expert weights.
+ *   priority order in which assignments claim expert slots: token order, first
+ *            come first served ("Lab 01", where to start step 4), or rank-major
+ *            (every first choice before any second, "Lab 18" section 3).
+ *   capacity_factor  C = ceil(capacity_factor * T * k / E) slots per expert
+ *            ("Lab 18" section 3); +infinity = no limit.  Must be >= 1.0.
+ * Limits: 1 <= k <= min(E, 8), E <= 256.  bf16 needs d, d_ff, d_ff_shared
+ * multiples of 64.
+ */
+typedef struct moe_config {
+    int32_t T, d, E, k, d_ff, n_shared, d_ff_shared;
+    int32_t act, score, renorm, dtype, priority;
+    double capacity_factor;
+} moe_config;
+
+/* Weights of one layer (device pointers, dtype unless noted).
+ *   W_r [d, E] fp32 router ("Lab 18" section 1: z = x W_r; routers stay fp32,
+ *       cs336 lecture 4, "Stability, fine-tuning, and upcycling").
+ *   logit_bias [E] fp32, nullable: added to every token's logits.
+ *   select_bias [E] fp32, nullable, sigmoid scores only: added to the scores
+ *       used to pick the top k, never to the gates ("Lab 18" section 2,
+ *       auxiliary-loss-free balancing).
+ *   W1, W3 [E, F, d] (W3 only for SwiGLU), W2 [E, d, F]: hidden = W1 x, output
+ *       = W2 hidden (row f of W1[e] holds hidden unit f's input weights).
+ *   Ws1, Ws3 [S, Fs, d], Ws2 [S, d, Fs]: shared experts, NULL when S = 0. */
+typedef struct moe_weights {
+    const float *W_r;
+    const float *logit_bias;
+    const float *select_bias;
+    const void *W1, *W3, *W2;
+    const void *Ws1, *Ws3, *Ws2;
+} moe_weights;
+
+/* Outputs of moe_forward (device pointers).  y, aux and zloss are required;
+ * every other field may be NULL, in which case the value lives only in the
+ * workspace.
+ *   y [T, d] dtype          the layer output; the residual x + y is the
+ *                           caller's ("Lab 18", GPU scale-up listing)
+ *   topk_idx [T, k] int32   experts of each token, best first
+ *   gates [T, k] fp32
+ *   keep [T, k] uint8       1 = the assignment got a slot
+ *   dropped [T] uint8       1 = every assignment of the token was dropped
+ *   counts [E] int32        assignments per expert before capacity
+ *   n_dropped [1] int32     dropped assignments
+ *   aux, zloss [1] fp32     unweighted L_aux and L_z ("Lab 18" section 2) */
+typedef struct moe_outputs {
+    void *y;
+    int32_t *topk_idx;
+    float *gates;
+    uint8_t *keep;
+    uint8_t *dropped;
+    int32_t *counts;
+    int32_t *n_dropped;
+    float *aux;
+    float *zloss;
+} moe_outputs;
+
+/* Human-readable text of a status code (static storage). */
+const char *moe_status_string(moe_status s);
+
+/* Validate a configuration (shape limits, codes, capacity factor). */
+moe_status moe_validate(const moe_config *cfg);
+
+/* C = ceil(capacity_factor * T * k / E), computed in double on the host in
+ * exactly that order of operations; T when the factor is +infinity
+ * ("Lab 18" section 3).  Writes *C (host). */
+moe_status moe_capacity_value(const moe_config *cfg, int64_t *C);
+
+/* Rows the caller must allocate for the permuted buffers x_perm and Y_perm:
+ * min(T*k, E*C) kept assignments plus per-expert padding to MOE_ROW_ALIGN.
+ * Returns -1 for an invalid configuration. */
+int64_t moe_perm_rows(const moe_config *cfg);
+
+/* Number of fp32 values moe_route writes to loss_partials. */
+int64_t moe_loss_partials_count(const moe_config *cfg);
+
+/* Scratch bytes the stage calls need (moe_capacity, moe_expert_ffn). */
+size_t moe_stage_workspace_size(const moe_config *cfg);
+
+/* Workspace bytes moe_forward needs (includes the stage scratch).  0 for an
+ * invalid configuration. */
+size_t moe_workspace_size(const moe_config *cfg);
+
+/*
+ * moe_route - router, scores, top-k and gates ("Lab 18" section 1 and the
+ * route() row of "What to implement"; router listing of "Mixture of Experts -
+ * parameters without the FLOPs", section 2).
+ *   x [T, d] dtype; W_r [d, E] fp32; logit_bias / select_bias as in moe_weights.
+ *   topk_idx [T, k] int32 out: the k experts with the largest selection key,
+ *     best first, equal keys to the lower index ("Lab 01" traps).  The key is
+ *     the logit for softmax scores (the same order as p) and s + select_bias
+ *     for sigmoid scores.
+ *   gates [T, k] fp32 out: p or s of the selected experts, renormalized over
+ *     them when cfg->renorm says so.
+ *   loss_partials [moe_loss_partials_count] fp32 out: per token block, the sum
+ *     of each expert's probability (sigmoid: s / sum s) and of lse^2, summed
+ *     by moe_losses in a fixed order.
+ *   logits_out [T, E] fp32, nullable: the router logits z.
+ *   scores_out [T, E] fp32, nullable: p (softmax) or s (sigmoid).
+ * Logits are computed in fp32 from the exact fp32 widening of x.
+ */
+moe_status moe_route(const moe_config *cfg, const void *x, const float *W_r,
+                     const float *logit_bias, const float *select_bias,
+                     int32_t *topk_idx, float *gates, float *loss_partials,
+                     float *logits_out, float *scores_out, moe_stream_t stream);
+
+/*
+ * moe_capacity - slot assignment under the capacity limit ("Lab 18" section 3;
+ * "Lab 01", where to start step 4).  Bit-exact with a sequential walk over the
+ * assignments in priority order that gives each one position = (number of
+ * earlier assignments to the same expert) and keeps it while position < C.
+ *   topk_idx [T, k] int32 in.
+ *   counts [E] int32 out: assignments per expert before capacity.
+ *   pos [T, k] int32 out: queue position of each assignment in its expert.
+ *   keep [T, k] uint8 out: pos < C.
+ *   kept [E] int32 out: min(counts, C).
+ *   offsets [E + 1] int32 out: first row of each expert's segment in the
+ *     permuted buffers; offsets[e + 1] - offsets[e] = kept[e] rounded up to
+ *     MOE_ROW_ALIGN; offsets[E] = rows used.
+ *   dropped [T] uint8 out: 1 when every slot of the token was dropped.
+ *   n_dropped [1] int32 out: number of dropped assignments.
+ *   ws: scratch of at least moe_stage_workspace_size bytes, 256-byte aligned.
+ * Returns MOE_ERR_CAPACITY_FACTOR for capacity_factor < 1 ("Lab 01" traps).
+ */
+moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx,
+                        int32_t *counts, int32_t *pos, uint8_t *keep,
+                        int32_t *kept, int32_t *offsets, uint8_t *dropped,
+                        int32_t *n_dropped, void *ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
+/*
+ * moe_dispatch - permute token rows into expert-grouped order ("Lab 18" tips:
+ * gather each expert's tokens and run the expert once on them).
+ *   x [T, d] dtype in; topk_idx, pos, keep, offsets from moe_capacity.
+ *   x_perm [moe_perm_rows, d] dtype out: row offsets[e] + pos[t, j] = x[t] for
+ *     every kept (t, j).  Padding rows are left untouched.
+ */
+moe_status moe_dispatch(const moe_config *cfg, const void *x,
+                        const int32_t *topk_idx, const int32_t *pos,
+                        const uint8_t *keep, const int32_t *offsets,
+                        void *x_perm, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn - the expert FFNs over the expert segments, and the shared
+ * experts over all tokens ("Lab 18" section 1 expert definitions, tips: one
+ * grouped matrix multiply over all experts).
+ *   x_perm [moe_perm_rows, d] dtype in; offsets [E + 1] from moe_capacity.
+ *   W1, W3, W2 routed weights; x [T, d] and Ws1, Ws3, Ws2 for the shared
+ *     experts (all NULL when S = 0).
+ *   Y_perm [moe_perm_rows, d] dtype out: FFN_e of each row of segment e.
+ *   Y_shared [T, d] dtype out (NULL when S = 0): sum over s of FFN_s(x_t).
+ *   ws: scratch (hidden activations), moe_stage_workspace_size bytes.
+ * bf16 runs on the tensor cores (tcgen05, fp32 accumulation, hidden
+ * activations rounded to bf16); fp32 runs on the CUDA cores in fp32.
+ */
+moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm,
+                          const int32_t *offsets, const void *W1,
+                          const void *W3, const void *W2, const void *x,
+                          const void *Ws1, const void *Ws3, const void *Ws2,
+                          void *Y_perm, void *Y_shared, void *ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_combine - gate-weighted sum plus shared experts ("Lab 18" section 1,
+ * y = sum g_i FFN_i(x); section 3, a dropped slot contributes nothing):
+ *   y[t] = sum_{j = 0..k-1, keep[t, j]} gates[t, j] * Y_perm[offsets[e] + pos[t, j]]
+ *          + Y_shared[t] (+ residual[t])
+ * summed in fp32 in that order and stored as dtype.  A token with every slot
+ * dropped gets Y_shared[t] (or 0), plus the residual when given.
+ *   Y_shared, residual [T, d] dtype: nullable.
+ */
+moe_status moe_combine(const moe_config *cfg, const void *Y_perm,
+                       const void *Y_shared, const float *gates,
+                       const int32_t *topk_idx, const int32_t *pos,
+                       const uint8_t *keep, const int32_t *offsets,
+                       const void *residual, void *y, moe_stream_t stream);
+
+/*
+ * moe_losses - Switch load-balance loss and router z-loss ("Lab 18" section 2;
+ * "Lab 01" step 3: f divides by the T k slots):
+ *   aux = E * sum_i (counts_i / (T k)) * P_i,  P_i = (1/T) sum_t p_{t,i}
+ *   zloss = (1/T) sum_t lse_t^2
+ * from counts (moe_capacity) and loss_partials (moe_route), reduced in a fixed
+ * order (deterministic).  aux, zloss: device fp32 scalars, unweighted.
+ */
+moe_status moe_losses(const moe_config *cfg, const int32_t *counts,
+                      const float *loss_partials, float *aux, float *zloss,
+                      moe_stream_t stream);
+
+/*
+ * moe_forward - the whole layer: route, capacity, dispatch, expert FFNs,
+ * combine, losses ("Lab 18", MoE.forward row of "What to implement").
+ *   x [T, d] dtype; weights; outputs as described at moe_outputs.
+ *   ws: at least moe_workspace_size(cfg) bytes, 256-byte aligned.
+ * Six kernel stages, no host synchronisation, safe to capture in a CUDA graph.
+ */
+moe_status moe_forward(const moe_config *cfg, const moe_weights *w,
+                       const void *x, const moe_outputs *out, void *ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_device_status - read the device status word that the expert GEMM's
+ * bounded waits set when they give up (MOE_OK or MOE_ERR_DEVICE_TIMEOUT).
+ * ws is the workspace passed to moe_expert_ffn / moe_forward; *status is host
+ * memory.  Synchronises `stream` (a cudaMemcpyAsync followed by a stream
+ * synchronise) - the only call in this library that does.
+ */
+moe_status moe_device_status(const void *ws, int32_t *status,
+                             moe_stream_t stream);
+
+/* Clear the device status word (asynchronous, on `stream`). */
+moe_status moe_clear_device_status(void *ws, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,672 @@
+// Expert FFNs in bf16 on the 5th-generation tensor cores: a persistent,
+// warp-specialised grouped GEMM (TMA -> shared memory -> tcgen05.mma -> TMEM
+// -> epilogue -> TMA store) over the variable-length expert segments.
+//
+// Page "Lab 18 - Mixture of experts": section 1 (experts are W2 gelu(W1 x) or
+// W2 (silu(W1 x) * (W3 x))), tips ("production kernels do the same thing as one
+// grouped matrix multiply over all experts"); shared experts run on every token
+// ("Lab 18" section 1, DeepSeekMoE row).
+//
+// Two launches: GEMM1 (hidden = act(A W1^T), SwiGLU fuses W3) and GEMM2
+// (out = hidden W2^T).  Each launch covers two tile sets:
+//   set 0, routed: for expert e the rows [offsets[e], offsets[e+1]) of the
+//          permuted buffer, read from device memory (no host sync); segments
+//          start on multiples of 128 rows, so a 128-row tile has one expert;
+//   set 1, shared: all T token rows.  GEMM1 spreads the S shared experts over
+//          the N tiles (each writes its own column block of the hidden
+//          buffer); GEMM2 runs K over all S experts so their outputs add up in
+//          the TMEM accumulator.
+// Tile = 128 rows x 256 accumulator columns, K step 64 (one 128-byte swizzle
+// atom of bf16), 4-stage TMA ring, double-buffered TMEM accumulator (2 x 256
+// of the 512 columns) so the epilogue of one tile overlaps the MMAs of the
+// next.  SwiGLU tiles load 128 rows of W1 and the same 128 rows of W3 into one
+// 256-row B tile: accumulator columns [0,128) hold x W1^T, [128,256) x W3^T.
+//
+// Warps: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..5 = epilogue
+// (warp w reads TMEM lanes 32 (w mod 4) .. +31).  Every wait on an mbarrier is
+// bounded by a wall-clock limit; on expiry the CTA records
+// MOE_ERR_DEVICE_TIMEOUT in the status word, every role leaves its loop, the
+// CTA drains what it issued (bounded as well), frees TMEM and returns.
+#include "internal.cuh"
+
+#include <cuda.h>
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
+constexpr int EPI_WARPS = 4;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;         // 192
+constexpr int CHUNK = 32;                            // epilogue columns per step
+constexpr int STG_BYTES = 32 * CHUNK * 2;            // 32 rows x 32 bf16 = 2 KB
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_BAR = OFF_STG + EPI_WARPS * 2 * STG_BYTES;
+constexpr int OFF_TILES = OFF_BAR + 256;
+constexpr int SMEM_BYTES = OFF_TILES + 2 * 4 * (kMaxE + 1) + 1024;   // + alignment slack
+
+enum Epi { EPI_NONE = 0, EPI_GELU = 1, EPI_SWIGLU = 2 };
+
+struct SetDesc {
+    int routed;     // 1: rows and B group from the segment table
+    int rows;       // dense row count (shared set)
+    int n_tiles;    // N tiles per N group
+    int n_groups;   // groups the N tiles run over (shared GEMM1: S), else 1
+    int k_blocks;   // K blocks per tile
+    int kbg;        // > 0: K runs over groups, kbg blocks each (shared GEMM2)
+    int c_cols;     // columns of the output tensor (chunks at or past it are skipped)
+};
+
+struct __align__(64) Params {
+    CUtensorMap tmA[2], tmB[2], tmB3[2], tmC[2];
+    SetDesc set[2];
+    int nsets;
+    int E;
+    const int32_t *offsets;
+    int32_t *status;
+    unsigned long long timeout_ns;
+};
+
+// ------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+struct Ctl {
+    volatile int *abort;
+    int32_t *status;
+    uint64_t timeout_ns;
+};
+
+// Wait for the phase of `bar` with the given parity to complete.  Gives up
+// (returns false) when the time limit passed or, if honor_abort, when another
+// role already gave up.  Drain waits pass honor_abort = false: they must see
+// their own copies land even after an abort, but stay bounded.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &c,
+                                      bool honor_abort = true)
+{
+    if (mbar_try(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try(bar, parity))
+            return true;
+        if ((i & 31u) == 0) {
+            if (honor_abort && *c.abort)
+                return false;
+            if (global_ns() - t0 > c.timeout_ns) {
+                *c.abort = 1;
+                atomicExch(c.status, (int32_t)MOE_ERR_DEVICE_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
+                                             int c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::
+                     "l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// K-major operand tile in shared memory, 128-byte swizzle: rows of 128 bytes,
+// 8-row groups 1024 bytes apart (stride byte offset 64 x 16 B), leading byte
+// offset unused for this layout (1), descriptor version 1, layout code 2.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)64 << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                     "r"(bar)
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns: thread i gets lane (base + i)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------ tile schedule
+
+struct Tile {
+    int set;
+    int m0;       // first row of A and C
+    int b_group;  // group of the B tensor (K not split)
+    int b_row;    // first B row inside the group
+    int c_col;    // first C column
+    int c_group;  // group of the C tensor
+};
+
+__device__ __forceinline__ Tile decode(const Params &p, const int *tstart, const int *mtiles,
+                                       int routed_total, int tile, int bn_b, int bn_out)
+{
+    Tile t;
+    if (tile < routed_total) {
+        int lo = 0, hi = p.E;   // last e with tstart[e] <= tile
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (tstart[mid] <= tile)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int e = lo, i = tile - tstart[e], mt = mtiles[e];
+        const int n = i / mt, m = i % mt;
+        t.set = 0;
+        t.m0 = p.offsets[e] + m * BM;
+        t.b_group = e;
+        t.b_row = n * bn_b;
+        t.c_col = n * bn_out;
+        t.c_group = 0;
+    } else {
+        const SetDesc &s = p.set[1];
+        const int i = tile - routed_total;
+        const int mt = (s.rows + BM - 1) / BM;
+        const int n = i / mt, m = i % mt;
+        const int g = n / s.n_tiles, nn = n % s.n_tiles;
+        t.set = 1;
+        t.m0 = m * BM;
+        t.b_group = g;
+        t.b_row = nn * bn_b;
+        t.c_col = nn * bn_out;
+        t.c_group = g;
+    }
+    return t;
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const float *g, const float *u, uint32_t *packed)
+{
+#pragma unroll
+    for (int i = 0; i < CHUNK; i += 2) {
+        float a, b;
+        if (EPI == EPI_SWIGLU) {
+            a = g[i] / (1.f + __expf(-g[i])) * u[i];
+            b = g[i + 1] / (1.f + __expf(-g[i + 1])) * u[i + 1];
+        } else if (EPI == EPI_GELU) {
+            a = 0.5f * g[i] * (1.f + erff(g[i] * 0.70710678118654752f));
+            b = 0.5f * g[i + 1] * (1.f + erff(g[i + 1] * 0.70710678118654752f));
+        } else {
+            a = g[i];
+            b = g[i + 1];
+        }
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        packed[i / 2] = *reinterpret_cast<uint32_t *>(&h);
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p)
+{
+    constexpr int BN_B = EPI == EPI_SWIGLU ? BN / 2 : BN;     // B rows per tensor per tile
+    constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;   // output columns per tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sA = smem_u32(smem + OFF_A);
+    const uint32_t sB = smem_u32(smem + OFF_B);
+    const uint32_t sStg = smem_u32(smem + OFF_STG);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    // full[0..S), empty[S..2S), tfull[2S, 2S+2), tempty[2S+2, 2S+4), drain 2S+4
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8 * (2 * STAGES + 5));
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *tstart = reinterpret_cast<int *>(smem + OFF_TILES);    // [E + 1]
+    int *mtiles = tstart + (kMaxE + 1);                         // [E]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Ctl ctl{abort_flag, p.status, p.timeout_ns};
+
+    // ---- set-up: barriers, TMEM, tile table ----
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), EPI_WARPS);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    int routed_total = 0;
+    if (p.set[0].routed && p.nsets > 0) {
+        for (int e = threadIdx.x; e < p.E; e += THREADS)
+            mtiles[e] = (p.offsets[e + 1] - p.offsets[e]) / BM;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int acc = 0;
+            for (int e = 0; e < p.E; ++e) {
+                tstart[e] = acc;
+                acc += mtiles[e] * p.set[0].n_tiles;
+            }
+            tstart[p.E] = acc;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (p.set[0].routed && p.nsets > 0)
+        routed_total = tstart[p.E];
+    int shared_total = 0;
+    if (p.nsets > 1) {
+        const SetDesc &s = p.set[1];
+        shared_total = (s.rows + BM - 1) / BM * s.n_tiles * s.n_groups;
+    }
+    const int total = routed_total + shared_total;
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[STAGES];
+            uint32_t last_phase[STAGES];
+            for (int s = 0; s < STAGES; ++s)
+                issued[s] = 0, last_phase[s] = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+                const SetDesc &sd = p.set[t.set];
+                for (int kb = 0; kb < sd.k_blocks; ++kb) {
+                    if (!wait_bar(empty_bar(stage), phase ^ 1u, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    int kcol = kb * BK, ga = 0, gb = t.b_group;
+                    if (sd.kbg > 0) {
+                        ga = gb = kb / sd.kbg;
+                        kcol = (kb % sd.kbg) * BK;
+                    }
+                    const uint32_t fb = full_bar(stage);
+                    mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                    tma_load_3d(sA + stage * A_BYTES, &p.tmA[t.set], fb, kcol, t.m0, ga);
+                    if (EPI == EPI_SWIGLU) {
+                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                        tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &p.tmB3[t.set], fb, kcol,
+                                    t.b_row, gb);
+                    } else {
+                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                    }
+                    issued[stage] = 1;
+                    last_phase[stage] = phase;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // drain: every load this thread issued has landed before the CTA exits
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s])
+                    wait_bar(full_bar(s), last_phase[s], ctl, false);
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, any = false;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+                const SetDesc &sd = p.set[t.set];
+                if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < sd.k_blocks; ++kb) {
+                    if (!wait_bar(full_bar(stage), phase, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = sA + stage * A_BYTES, b_base = sB + stage * B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        mma_bf16(tmem_d, sdesc_sw128(a_base + kk * 32), sdesc_sw128(b_base + kk * 32),
+                                 (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(empty_bar(stage));
+                    any = true;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                mma_commit(tfull_bar(acc));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (any) {   // all MMAs issued by this thread complete before TMEM is freed
+                mma_commit(drain_bar);
+                wait_bar(drain_bar, 0, ctl, false);
+            }
+        }
+    } else {
+        // ================= epilogue (warps 2..5) =================
+        const int q = warp & 3;                      // TMEM lane quarter
+        const int ew = warp - 2;                     // staging buffer owner
+        const uint32_t stg0 = sStg + ew * 2 * STG_BYTES;
+        uint8_t *stg_ptr0 = smem + OFF_STG + ew * 2 * STG_BYTES;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int buf = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+            if (!wait_bar(tfull_bar(acc), acc_phase, ctl))
+                break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            const int c_end = min(BN_OUT, p.set[t.set].c_cols - t.c_col);
+#pragma unroll 1
+            for (int c = 0; c < c_end; c += CHUNK) {
+                float g[CHUNK], u[CHUNK];
+                uint32_t packed[CHUNK / 2];
+                tmem_ld32(tbase + c, g);
+                if (EPI == EPI_SWIGLU) {
+                    tmem_ld32(tbase + BN / 2 + c, u);
+                    epilogue_chunk<EPI>(g, u, packed);
+                } else {
+                    epilogue_chunk<EPI>(g, g, packed);
+                }
+                // staging tile: 32 rows x 64 bytes, 64-byte swizzle (16-byte
+                // chunk index XOR bits 1-2 of the row), as the store map expects
+                if (lane == 0)
+                    bulk_wait_read1();
+                __syncwarp();
+                uint8_t *row = stg_ptr0 + buf * STG_BYTES + lane * 64;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int phys = ch ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4 *>(row + phys * 16) =
+                        make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2],
+                                   packed[4 * ch + 3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&p.tmC[t.set], stg0 + buf * STG_BYTES, t.c_col + c, t.m0 + q * 32,
+                                 t.c_group);
+                    bulk_commit();
+                }
+                buf ^= 1;
+            }
+            // this warp's reads of the accumulator are done
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(tempty_bar(acc));
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0)
+            bulk_wait_all();
+        __syncwarp();
+    }
+
+    // ---- tear-down ----
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder()
+{
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(ptr);
+    }
+    return fn;
+}
+
+// 3-D bf16 tensor: dim0 (contiguous) x dim1 x dim2 with byte strides s1, s2.
+bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw)
+{
+    EncodeTiled enc = encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[3] = {d0, d1, d2 > 0 ? d2 : 1};
+    cuuint64_t strides[2] = {s1, s2 > 0 ? s2 : s1 * (d1 > 0 ? d1 : 1)};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count()
+{
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+template <int EPI>
+cudaError_t launch(const Params &p, cudaStream_t s)
+{
+    auto kern = grouped_gemm_kernel<EPI>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (err != cudaSuccess)
+        return err;
+    kern<<<sm_count(), THREADS, SMEM_BYTES, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const int32_t *offsets,
+                               const void *W1, const void *W3, const void *W2, const void *x,
+                               const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
+                               void *Y_sh, void *H, void *H_sh, int32_t *status, cudaStream_t s)
+{
+    using namespace tc;
+    const uint64_t R = (uint64_t)perm_rows(c), d = c.d, F = c.d_ff, E = c.E;
+    const uint64_t T = c.T, S = c.n_shared, Fs = c.d_ff_shared;
+    const bool swiglu = c.act == MOE_ACT_SWIGLU;
+    const int bn_b = swiglu ? BN / 2 : BN;
+    const int bn_out = swiglu ? BN / 2 : BN;
+    const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B, SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
+    const bool shared = S > 0 && T > 0;
+
+    // ---- GEMM1: H = act(x_perm W1^T [, x_perm W3^T]); H_sh likewise from x ----
+    Params p1;
+    memset(&p1, 0, sizeof p1);
+    p1.E = c.E;
+    p1.offsets = offsets;
+    p1.status = status;
+    p1.timeout_ns = 2000000000ull;
+    p1.nsets = shared ? 2 : 1;
+    bool ok = true;
+    ok &= make_map(&p1.tmA[0], x_perm, d, R, 1, d * 2, 0, BK, BM, SW128);
+    ok &= make_map(&p1.tmB[0], W1, d, F, E, d * 2, F * d * 2, BK, bn_b, SW128);
+    if (swiglu)
+        ok &= make_map(&p1.tmB3[0], W3, d, F, E, d * 2, F * d * 2, BK, bn_b, SW128);
+    ok &= make_map(&p1.tmC[0], H, F, R, 1, F * 2, 0, CHUNK, 32, SW64);
+    p1.set[0] = SetDesc{1, 0, (int)ceil_div(F, bn_out), 1, (int)ceil_div(d, BK), 0, (int)F};
+    if (shared) {
+        ok &= make_map(&p1.tmA[1], x, d, T, 1, d * 2, 0, BK, BM, SW128);
+        ok &= make_map(&p1.tmB[1], Ws1, d, Fs, S, d * 2, Fs * d * 2, BK, bn_b, SW128);
+        if (swiglu)
+            ok &= make_map(&p1.tmB3[1], Ws3, d, Fs, S, d * 2, Fs * d * 2, BK, bn_b, SW128);
+        // H_sh [S][T][Fs]: shared expert s owns one [T][Fs] slab
+        ok &= make_map(&p1.tmC[1], H_sh, Fs, T, S, Fs * 2, T * Fs * 2, CHUNK, 32, SW64);
+        p1.set[1] = SetDesc{0, (int)T, (int)ceil_div(Fs, bn_out), (int)S, (int)ceil_div(d, BK), 0,
+                            (int)Fs};
+    }
+    if (!ok)
+        return cudaErrorInvalidValue;
+    cudaError_t err = swiglu ? launch<EPI_SWIGLU>(p1, s) : launch<EPI_GELU>(p1, s);
+    if (err != cudaSuccess)
+        return err;
+
+    // ---- GEMM2: Y_perm = H W2^T; Y_sh = sum_s H_sh[:, s] Ws2[s]^T ----
+    Params p2;
+    memset(&p2, 0, sizeof p2);
+    p2.E = c.E;
+    p2.offsets = offsets;
+    p2.status = status;
+    p2.timeout_ns = 2000000000ull;
+    p2.nsets = shared ? 2 : 1;
+    ok = true;
+    ok &= make_map(&p2.tmA[0], H, F, R, 1, F * 2, 0, BK, BM, SW128);
+    ok &= make_map(&p2.tmB[0], W2, F, d, E, F * 2, d * F * 2, BK, BN, SW128);
+    ok &= make_map(&p2.tmC[0], Y_perm, d, R, 1, d * 2, 0, CHUNK, 32, SW64);
+    p2.set[0] = SetDesc{1, 0, (int)ceil_div(d, BN), 1, (int)ceil_div(F, BK), 0, (int)d};
+    if (shared) {
+        ok &= make_map(&p2.tmA[1], H_sh, Fs, T, S, Fs * 2, T * Fs * 2, BK, BM, SW128);
+        ok &= make_map(&p2.tmB[1], Ws2, Fs, d, S, Fs * 2, d * Fs * 2, BK, BN, SW128);
+        ok &= make_map(&p2.tmC[1], Y_sh, d, T, 1, d * 2, 0, CHUNK, 32, SW64);
+        const int kbg = (int)ceil_div(Fs, BK);
+        p2.set[1] = SetDesc{0, (int)T, (int)ceil_div(d, BN), 1, kbg * (int)S, kbg, (int)d};
+    }
+    if (!ok)
+        return cudaErrorInvalidValue;
+    return launch<EPI_NONE>(p2, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,81 @@
+// Library-private declarations shared by the CUDA translation units of
+// libmoe_b200.so.  Nothing here is visible through the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 8;
+constexpr int kRouteTokens = 32;   // tokens per route block
+constexpr int kCapTokens = 256;    // tokens per capacity block
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline int dtype_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+// Shape limits and codes; also the capacity factor rule.
+moe_status validate(const moe_config &c);
+int64_t capacity_of(const moe_config &c);          // valid config only
+int64_t perm_rows(const moe_config &c);            // valid config only
+int route_blocks(const moe_config &c);
+int cap_blocks(const moe_config &c);
+
+// Scratch carving of the stage workspace.
+struct StageScratch {
+    int32_t *status;      // device status word (timeouts)
+    int32_t *hist;        // [cap_blocks][k][E]
+    int32_t *base;        // [cap_blocks][k][E]
+    void *H;              // [perm_rows][F] dtype
+    void *H_sh;           // [T][S * Fs] dtype
+};
+size_t stage_scratch_bytes(const moe_config &c);
+StageScratch carve_stage(const moe_config &c, void *ws);
+
+// ---- launches (return the first CUDA error, cudaSuccess otherwise) ----
+cudaError_t launch_route(const moe_config &c, const void *x, const float *W_r,
+                         const float *logit_bias, const float *select_bias,
+                         int32_t *topk, float *gates, float *partials,
+                         float *logits_out, float *scores_out, cudaStream_t s);
+
+cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
+                            int32_t *counts, int32_t *pos, uint8_t *keep,
+                            int32_t *kept, int32_t *offsets, uint8_t *dropped,
+                            int32_t *n_dropped, int32_t *hist, int32_t *base,
+                            cudaStream_t s);
+
+cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *topk,
+                            const int32_t *pos, const uint8_t *keep,
+                            const int32_t *offsets, void *x_perm, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config &c, const void *Y_perm, const void *Y_sh,
+                           const float *gates, const int32_t *topk, const int32_t *pos,
+                           const uint8_t *keep, const int32_t *offsets,
+                           const void *residual, void *y, cudaStream_t s);
+
+cudaError_t launch_losses(const moe_config &c, const int32_t *counts,
+                          const float *partials, float *aux, float *zloss,
+                          cudaStream_t s);
+
+// fp32 expert FFNs on the CUDA cores
+cudaError_t launch_ffn_simt(const moe_config &c, const void *x_perm, const int32_t *offsets,
+                            const void *W1, const void *W3, const void *W2,
+                            const void *x, const void *Ws1, const void *Ws3,
+                            const void *Ws2, void *Y_perm, void *Y_sh, void *H,
+                            void *H_sh, cudaStream_t s);
+
+// bf16 expert FFNs on the tensor cores (tcgen05 + TMEM + TMA)
+cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm,
+                               const int32_t *offsets, const void *W1, const void *W3,
+                               const void *W2, const void *x, const void *Ws1,
+                               const void *Ws3, const void *Ws2, void *Y_perm,
+                               void *Y_sh, void *H, void *H_sh, int32_t *status,
+                               cudaStream_t s);
+
+}  // namespace moe

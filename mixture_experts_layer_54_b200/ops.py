@@ -1,0 +1,301 @@
+"""Thin torch-facing binding of the C ABI: same names as the C calls, argument
+marshalling only (device pointers, sizes, the current CUDA stream).  Every
+step of the layer runs in the library's kernels; output tensors are allocated
+here with torch, which is the library's memory manager.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _abi
+from ._abi import MoeConfig, MoeOutputs, MoeWeights, check, lib
+
+DTYPE_F32, DTYPE_BF16 = 0, 1
+
+
+def moe_config(shape=None, **kw) -> MoeConfig:
+    """Build the C config from any object with the layer's attributes
+    (T, d, E, k, d_ff, act, dtype, cf, and optionally n_shared, d_ff_shared,
+    score, renorm, priority) and/or keyword overrides."""
+    def get(name, default=None):
+        if name in kw:
+            return kw[name]
+        if shape is not None and hasattr(shape, name):
+            return getattr(shape, name)
+        return default
+    cf = get("cf", get("capacity_factor", 1.0))
+    return MoeConfig(T=get("T"), d=get("d"), E=get("E"), k=get("k"), d_ff=get("d_ff"),
+                     n_shared=get("n_shared", 0), d_ff_shared=get("d_ff_shared", 0),
+                     act=get("act", 0), score=get("score", 0), renorm=get("renorm", -1),
+                     dtype=get("dtype", DTYPE_BF16), priority=get("priority", 0),
+                     capacity_factor=float(cf))
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("moe ops take CUDA tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _tdtype(cfg: MoeConfig):
+    return torch.bfloat16 if cfg.dtype == DTYPE_BF16 else torch.float32
+
+
+def _dev(t):
+    return t.device
+
+
+def moe_validate(cfg: MoeConfig):
+    check(lib().moe_validate(ctypes.byref(cfg)), "moe_validate")
+
+
+def moe_capacity_value(cfg: MoeConfig) -> int:
+    C = ctypes.c_int64()
+    check(lib().moe_capacity_value(ctypes.byref(cfg), ctypes.byref(C)), "moe_capacity_value")
+    return int(C.value)
+
+
+def moe_perm_rows(cfg: MoeConfig) -> int:
+    moe_validate(cfg)
+    return int(lib().moe_perm_rows(ctypes.byref(cfg)))
+
+
+def moe_loss_partials_count(cfg: MoeConfig) -> int:
+    moe_validate(cfg)
+    return int(lib().moe_loss_partials_count(ctypes.byref(cfg)))
+
+
+def moe_stage_workspace_size(cfg: MoeConfig) -> int:
+    moe_validate(cfg)
+    return int(lib().moe_stage_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_workspace_size(cfg: MoeConfig) -> int:
+    moe_validate(cfg)
+    return int(lib().moe_workspace_size(ctypes.byref(cfg)))
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned uint8 device buffer (torch's allocator aligns to 512)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def moe_route(cfg: MoeConfig, x, W_r, logit_bias=None, select_bias=None, want_logits=False,
+              want_scores=False):
+    dev = _dev(x)
+    T, k, E = cfg.T, cfg.k, cfg.E
+    topk = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    partials = torch.empty((max(moe_loss_partials_count(cfg), 1),), dtype=torch.float32,
+                           device=dev)
+    logits = torch.empty((T, E), dtype=torch.float32, device=dev) if want_logits else None
+    scores = torch.empty((T, E), dtype=torch.float32, device=dev) if want_scores else None
+    check(lib().moe_route(ctypes.byref(cfg), _p(x), _p(W_r), _p(logit_bias), _p(select_bias),
+                          _p(topk), _p(gates), _p(partials), _p(logits), _p(scores), _stream()),
+          "moe_route")
+    return topk, gates, partials, logits, scores
+
+
+@dataclass
+class CapacityOut:
+    counts: torch.Tensor
+    pos: torch.Tensor
+    keep: torch.Tensor
+    kept: torch.Tensor
+    offsets: torch.Tensor
+    dropped: torch.Tensor
+    n_dropped: torch.Tensor
+
+
+def moe_capacity(cfg: MoeConfig, topk, ws=None) -> CapacityOut:
+    dev = _dev(topk)
+    T, k, E = cfg.T, cfg.k, cfg.E
+    out = CapacityOut(
+        counts=torch.empty((E,), dtype=torch.int32, device=dev),
+        pos=torch.empty((T, k), dtype=torch.int32, device=dev),
+        keep=torch.empty((T, k), dtype=torch.uint8, device=dev),
+        kept=torch.empty((E,), dtype=torch.int32, device=dev),
+        offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+        dropped=torch.empty((T,), dtype=torch.uint8, device=dev),
+        n_dropped=torch.empty((1,), dtype=torch.int32, device=dev))
+    if ws is None:
+        ws = workspace(moe_stage_workspace_size(cfg), dev)
+    check(lib().moe_capacity(ctypes.byref(cfg), _p(topk), _p(out.counts), _p(out.pos),
+                             _p(out.keep), _p(out.kept), _p(out.offsets), _p(out.dropped),
+                             _p(out.n_dropped), _p(ws), ws.numel(), _stream()), "moe_capacity")
+    return out
+
+
+def moe_dispatch(cfg: MoeConfig, x, topk, pos, keep, offsets, x_perm=None):
+    if x_perm is None:
+        x_perm = torch.empty((moe_perm_rows(cfg), cfg.d), dtype=_tdtype(cfg), device=_dev(x))
+    check(lib().moe_dispatch(ctypes.byref(cfg), _p(x), _p(topk), _p(pos), _p(keep), _p(offsets),
+                             _p(x_perm), _stream()), "moe_dispatch")
+    return x_perm
+
+
+def moe_expert_ffn(cfg: MoeConfig, x_perm, offsets, W1, W3, W2, x=None, Ws1=None, Ws3=None,
+                   Ws2=None, ws=None, Y_perm=None, Y_shared=None):
+    dev = _dev(x_perm)
+    if Y_perm is None:
+        Y_perm = torch.empty((moe_perm_rows(cfg), cfg.d), dtype=_tdtype(cfg), device=dev)
+    if cfg.n_shared > 0 and Y_shared is None:
+        Y_shared = torch.empty((cfg.T, cfg.d), dtype=_tdtype(cfg), device=dev)
+    if ws is None:
+        ws = workspace(moe_stage_workspace_size(cfg), dev)
+    check(lib().moe_expert_ffn(ctypes.byref(cfg), _p(x_perm), _p(offsets), _p(W1), _p(W3),
+                               _p(W2), _p(x), _p(Ws1), _p(Ws3), _p(Ws2), _p(Y_perm),
+                               _p(Y_shared), _p(ws), ws.numel(), _stream()), "moe_expert_ffn")
+    return Y_perm, Y_shared, ws
+
+
+def moe_combine(cfg: MoeConfig, Y_perm, Y_shared, gates, topk, pos, keep, offsets,
+                residual=None, y=None):
+    if y is None:
+        y = torch.empty((cfg.T, cfg.d), dtype=_tdtype(cfg), device=_dev(Y_perm))
+    check(lib().moe_combine(ctypes.byref(cfg), _p(Y_perm), _p(Y_shared), _p(gates), _p(topk),
+                            _p(pos), _p(keep), _p(offsets), _p(residual), _p(y), _stream()),
+          "moe_combine")
+    return y
+
+
+def moe_losses(cfg: MoeConfig, counts, partials):
+    dev = _dev(counts)
+    aux = torch.empty((1,), dtype=torch.float32, device=dev)
+    zl = torch.empty((1,), dtype=torch.float32, device=dev)
+    check(lib().moe_losses(ctypes.byref(cfg), _p(counts), _p(partials), _p(aux), _p(zl),
+                           _stream()), "moe_losses")
+    return aux, zl
+
+
+def moe_device_status(ws) -> int:
+    st = ctypes.c_int32()
+    check(lib().moe_device_status(_p(ws), ctypes.byref(st), _stream()), "moe_device_status")
+    return int(st.value)
+
+
+def weights_struct(W_r, W1, W2, W3=None, logit_bias=None, select_bias=None, Ws1=None, Ws3=None,
+                   Ws2=None) -> MoeWeights:
+    def v(t):
+        return None if t is None else _p(t).value
+    return MoeWeights(W_r=v(W_r), logit_bias=v(logit_bias), select_bias=v(select_bias),
+                      W1=v(W1), W3=v(W3), W2=v(W2), Ws1=v(Ws1), Ws3=v(Ws3), Ws2=v(Ws2))
+
+
+class MoEForward:
+    """Reusable forward of one layer: owns the workspace and the outputs, so
+    repeated calls allocate nothing (the benchmark and CUDA-graph friendly
+    form of moe_forward)."""
+
+    def __init__(self, cfg: MoeConfig, device, keep_routing: bool = True):
+        self.cfg = cfg
+        moe_validate(cfg)
+        dev = torch.device(device)
+        T, k, E = cfg.T, cfg.k, cfg.E
+        self.ws = workspace(moe_workspace_size(cfg), dev)
+        self.y = torch.empty((T, cfg.d), dtype=_tdtype(cfg), device=dev)
+        self.aux = torch.empty((1,), dtype=torch.float32, device=dev)
+        self.zloss = torch.empty((1,), dtype=torch.float32, device=dev)
+        self.topk = self.gates = self.keep = self.dropped = self.counts = self.n_dropped = None
+        if keep_routing:
+            self.topk = torch.empty((T, k), dtype=torch.int32, device=dev)
+            self.gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+            self.keep = torch.empty((T, k), dtype=torch.uint8, device=dev)
+            self.dropped = torch.empty((T,), dtype=torch.uint8, device=dev)
+            self.counts = torch.empty((E,), dtype=torch.int32, device=dev)
+            self.n_dropped = torch.empty((1,), dtype=torch.int32, device=dev)
+
+        def v(t):
+            return None if t is None else t.data_ptr()
+        self._out = MoeOutputs(y=v(self.y), topk_idx=v(self.topk), gates=v(self.gates),
+                               keep=v(self.keep), dropped=v(self.dropped),
+                               counts=v(self.counts), n_dropped=v(self.n_dropped),
+                               aux=v(self.aux), zloss=v(self.zloss))
+
+    def __call__(self, x, weights: MoeWeights):
+        check(lib().moe_forward(ctypes.byref(self.cfg), ctypes.byref(weights), _p(x),
+                                ctypes.byref(self._out), _p(self.ws), self.ws.numel(), _stream()),
+              "moe_forward")
+        return self.y
+
+
+def moe_forward(cfg: MoeConfig, x, W_r, W1, W2, W3=None, logit_bias=None, select_bias=None,
+                Ws1=None, Ws3=None, Ws2=None):
+    """One-shot forward: returns (y, aux, zloss, MoEForward state with routing)."""
+    fwd = MoEForward(cfg, x.device)
+    w = weights_struct(W_r, W1, W2, W3, logit_bias, select_bias, Ws1, Ws3, Ws2)
+    fwd(x, w)
+    return fwd.y, fwd.aux, fwd.zloss, fwd
+
+
+__all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
+           "moe_loss_partials_count", "moe_stage_workspace_size", "moe_workspace_size",
+           "workspace", "moe_route", "moe_capacity", "moe_dispatch", "moe_expert_ffn",
+           "moe_combine", "moe_losses", "moe_device_status", "weights_struct", "MoEForward",
+           "moe_forward", "CapacityOut", "StagedForward"]
+
+
+class StagedForward:
+    """The forward as its six stage calls on preallocated buffers.  Runs the
+    same kernels as moe_forward; `events`, when given, are seven CUDA events
+    recorded before, between and after the stages so each stage's device time
+    can be read (route, capacity, dispatch, expert_ffn, combine, losses)."""
+
+    STAGES = ("route", "capacity", "dispatch", "expert_ffn", "combine", "losses")
+
+    def __init__(self, cfg: MoeConfig, device):
+        moe_validate(cfg)
+        self.cfg = cfg
+        dev = torch.device(device)
+        T, k, E, d = cfg.T, cfg.k, cfg.E, cfg.d
+        dt = _tdtype(cfg)
+        R = moe_perm_rows(cfg)
+        e = lambda shape, t: torch.empty(shape, dtype=t, device=dev)
+        self.topk, self.gates = e((T, k), torch.int32), e((T, k), torch.float32)
+        self.partials = e((max(moe_loss_partials_count(cfg), 1),), torch.float32)
+        self.counts, self.kept = e((E,), torch.int32), e((E,), torch.int32)
+        self.offsets, self.n_dropped = e((E + 1,), torch.int32), e((1,), torch.int32)
+        self.pos, self.keep = e((T, k), torch.int32), e((T, k), torch.uint8)
+        self.dropped = e((T,), torch.uint8)
+        self.x_perm, self.Y_perm = e((R, d), dt), e((R, d), dt)
+        self.Y_sh = e((T, d), dt) if cfg.n_shared > 0 else None
+        self.y = e((T, d), dt)
+        self.aux, self.zloss = e((1,), torch.float32), e((1,), torch.float32)
+        self.ws = workspace(moe_stage_workspace_size(cfg), dev)
+
+    def __call__(self, x, W_r, W1, W2, W3=None, logit_bias=None, select_bias=None, Ws1=None,
+                 Ws3=None, Ws2=None, events=None):
+        L, c, s = lib(), ctypes.byref(self.cfg), _stream()
+        rec = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        rec(0)
+        check(L.moe_route(c, _p(x), _p(W_r), _p(logit_bias), _p(select_bias), _p(self.topk),
+                          _p(self.gates), _p(self.partials), None, None, s), "moe_route")
+        rec(1)
+        check(L.moe_capacity(c, _p(self.topk), _p(self.counts), _p(self.pos), _p(self.keep),
+                             _p(self.kept), _p(self.offsets), _p(self.dropped),
+                             _p(self.n_dropped), _p(self.ws), self.ws.numel(), s), "moe_capacity")
+        rec(2)
+        check(L.moe_dispatch(c, _p(x), _p(self.topk), _p(self.pos), _p(self.keep),
+                             _p(self.offsets), _p(self.x_perm), s), "moe_dispatch")
+        rec(3)
+        check(L.moe_expert_ffn(c, _p(self.x_perm), _p(self.offsets), _p(W1), _p(W3), _p(W2),
+                               _p(x), _p(Ws1), _p(Ws3), _p(Ws2), _p(self.Y_perm), _p(self.Y_sh),
+                               _p(self.ws), self.ws.numel(), s), "moe_expert_ffn")
+        rec(4)
+        check(L.moe_combine(c, _p(self.Y_perm), _p(self.Y_sh), _p(self.gates), _p(self.topk),
+                            _p(self.pos), _p(self.keep), _p(self.offsets), None, _p(self.y), s),
+              "moe_combine")
+        rec(5)
+        check(L.moe_losses(c, _p(self.counts), _p(self.partials), _p(self.aux), _p(self.zloss),
+                           s), "moe_losses")
+        rec(6)
+        return self.y

@@ -72,10 +72,14 @@ int oracle_route(int T, int d, int E, int k, int score, int renorm,
     if (T < 0 || d < 1 || E < 1 || k < 1 || k > E)
         return OR_ERR_SHAPE;
     int do_renorm = renorm < 0 ? (k > 1) : renorm;
+    /* tokens are independent: the loop runs on OpenMP threads when available */
+#pragma omp parallel
+    {
     double *z = malloc(sizeof(double) * E);
     double *v = malloc(sizeof(double) * E);
     double *key = malloc(sizeof(double) * E);
     int *order = malloc(sizeof(int) * E);
+#pragma omp for schedule(static)
     for (int t = 0; t < T; ++t) {
         for (int e = 0; e < E; ++e) {
             double acc = 0.0;
@@ -130,6 +134,7 @@ int oracle_route(int T, int d, int E, int k, int score, int renorm,
     free(v);
     free(key);
     free(order);
+    }
     return OR_OK;
 }
 

@@ -1,0 +1,221 @@
+"""Stage-level GPU tests through the C ABI: each kernel against a plain
+float64 PyTorch (or pure integer) reference of the same operation on the same
+inputs.  End-to-end parity with the oracle is in test_gpu_parity.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as Fn
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mixture_experts_layer_54_b200 as moe
+
+DEV = "cuda"
+BF16_REL_FROB = 1e-2
+BF16_MAX_ABS = 2e-2
+
+
+def _ffn_ref(x, W1, W3, W2, act):
+    x, W1, W2 = x.double(), W1.double(), W2.double()
+    h = x @ W1.T
+    h = Fn.gelu(h) if act == 0 else Fn.silu(h) * (x @ W3.double().T)
+    return h @ W2.T
+
+
+def _close_bf16(got, ref):
+    got = got.double().cpu()
+    ref = ref.double().cpu()
+    err = (got - ref)
+    frob = err.norm() / max(ref.norm().item(), 1e-30)
+    mx = err.abs().max().item()
+    scale = ref.abs().max().item()
+    assert frob <= BF16_REL_FROB, f"relative Frobenius error {frob:.3e}"
+    assert mx <= BF16_MAX_ABS * scale, f"max abs error {mx:.3e} vs max|y| {scale:.3e}"
+
+
+def _segments(kept, align=128):
+    offsets = [0]
+    for c in kept:
+        offsets.append(offsets[-1] + (c + align - 1) // align * align)
+    return offsets
+
+
+@pytest.mark.parametrize("act", [0, 1])
+@pytest.mark.parametrize("dims", [(256, 384), (512, 128), (192, 256)])
+def test_expert_ffn_grouped_gemm_against_torch(act, dims):
+    """Ragged segments (empty, 1 row, 127, 128, 129, several tiles) through the
+    tcgen05 grouped GEMM; every kept row compared with its expert's FFN."""
+    d, F = dims
+    kept = [0, 1, 127, 128, 129, 300, 5, 260]
+    E = len(kept)
+    T = 400
+    cfg = moe.moe_config(T=T, d=d, E=E, k=2, d_ff=F, act=act, dtype=1, cf=math.inf)
+    R = moe.moe_perm_rows(cfg)
+    offsets = _segments(kept)
+    assert offsets[-1] <= R
+    g = torch.Generator(device=DEV).manual_seed(7)
+    x_perm = torch.randn((R, d), generator=g, device=DEV).to(torch.bfloat16)
+    W1 = (torch.randn((E, F, d), generator=g, device=DEV) / math.sqrt(d)).to(torch.bfloat16)
+    W3 = (torch.randn((E, F, d), generator=g, device=DEV) / math.sqrt(d)).to(torch.bfloat16) \
+        if act == 1 else None
+    W2 = (torch.randn((E, d, F), generator=g, device=DEV) / math.sqrt(F)).to(torch.bfloat16)
+    off_t = torch.tensor(offsets, dtype=torch.int32, device=DEV)
+    Y, _, ws = moe.moe_expert_ffn(cfg, x_perm, off_t, W1, W3, W2)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status(ws) == 0
+    for e in range(E):
+        if kept[e] == 0:
+            continue
+        rows = slice(offsets[e], offsets[e] + kept[e])
+        ref = _ffn_ref(x_perm[rows], W1[e], None if W3 is None else W3[e], W2[e], act)
+        _close_bf16(Y[rows], ref)
+
+
+@pytest.mark.parametrize("act,S", [(1, 2), (0, 1), (1, 1)])
+def test_shared_experts_against_torch(act, S):
+    d, F, Fs, T, E = 256, 128, 192, 333, 4
+    cfg = moe.moe_config(T=T, d=d, E=E, k=1, d_ff=F, act=act, dtype=1, cf=math.inf,
+                         n_shared=S, d_ff_shared=Fs)
+    R = moe.moe_perm_rows(cfg)
+    g = torch.Generator(device=DEV).manual_seed(11)
+    rnd = lambda *s, sc=1.0: (torch.randn(s, generator=g, device=DEV) * sc).to(torch.bfloat16)
+    x = rnd(T, d)
+    x_perm = rnd(R, d)
+    W1, W2 = rnd(E, F, d, sc=d ** -0.5), rnd(E, d, F, sc=F ** -0.5)
+    W3 = rnd(E, F, d, sc=d ** -0.5) if act else None
+    Ws1, Ws2 = rnd(S, Fs, d, sc=d ** -0.5), rnd(S, d, Fs, sc=Fs ** -0.5)
+    Ws3 = rnd(S, Fs, d, sc=d ** -0.5) if act else None
+    off_t = torch.tensor(_segments([T // 4] * E), dtype=torch.int32, device=DEV)
+    Y, Ysh, ws = moe.moe_expert_ffn(cfg, x_perm, off_t, W1, W3, W2, x, Ws1, Ws3, Ws2)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status(ws) == 0
+    ref = sum(_ffn_ref(x, Ws1[s], None if Ws3 is None else Ws3[s], Ws2[s], act) for s in range(S))
+    _close_bf16(Ysh, ref)
+
+
+def test_expert_ffn_fp32_simt_against_torch():
+    d, F, E, T = 32, 64, 4, 64
+    kept = [40, 0, 13, 75]
+    cfg = moe.moe_config(T=T, d=d, E=E, k=2, d_ff=F, act=0, dtype=0, cf=math.inf, n_shared=1,
+                         d_ff_shared=48)
+    R = moe.moe_perm_rows(cfg)
+    offsets = _segments(kept)
+    g = torch.Generator(device=DEV).manual_seed(3)
+    x_perm = torch.randn((R, d), generator=g, device=DEV)
+    x = torch.randn((T, d), generator=g, device=DEV)
+    W1 = torch.randn((E, F, d), generator=g, device=DEV) / math.sqrt(d)
+    W2 = torch.randn((E, d, F), generator=g, device=DEV) / math.sqrt(F)
+    Ws1 = torch.randn((1, 48, d), generator=g, device=DEV) / math.sqrt(d)
+    Ws2 = torch.randn((1, d, 48), generator=g, device=DEV) / math.sqrt(48)
+    Y, Ysh, _ = moe.moe_expert_ffn(cfg, x_perm, torch.tensor(offsets, dtype=torch.int32,
+                                                             device=DEV), W1, None, W2, x, Ws1,
+                                   None, Ws2)
+    torch.cuda.synchronize()
+    for e in range(E):
+        rows = slice(offsets[e], offsets[e] + kept[e])
+        if kept[e]:
+            ref = _ffn_ref(x_perm[rows], W1[e], None, W2[e], 0)
+            err = (Y[rows].double() - ref).abs().max().item()
+            assert err <= 1e-4 * ref.abs().max().item()
+    ref = _ffn_ref(x, Ws1[0], None, Ws2[0], 0)
+    assert (Ysh.double() - ref).abs().max().item() <= 1e-4 * ref.abs().max().item()
+
+
+@pytest.mark.parametrize("priority", [0, 1])
+@pytest.mark.parametrize("T,E,k,cf", [(1000, 8, 2, 1.0), (777, 64, 6, 1.25), (300, 256, 8, 1.0),
+                                      (5, 4, 4, 1.0), (1, 3, 1, 1.0)])
+def test_capacity_bit_exact_with_sequential_walk(priority, T, E, k, cf):
+    """Skewed random top-k lists (distinct experts per token) against the pages'
+    one-hot cumulative-sum formulation, in integers."""
+    rng = np.random.default_rng(T + E + priority)
+    w = 1.0 / np.arange(1, E + 1) ** 1.1
+    topk = np.stack([rng.choice(E, size=k, replace=False, p=w / w.sum()) for _ in range(T)])
+    topk = topk.astype(np.int32)
+    cfg = moe.moe_config(T=T, d=64, E=E, k=k, d_ff=64, dtype=1, cf=cf, priority=priority)
+    C = moe.moe_capacity_value(cfg)
+    out = moe.moe_capacity(cfg, torch.tensor(topk, device=DEV))
+    flat = topk.reshape(-1) if priority == 0 else topk.T.reshape(-1)
+    onehot = np.eye(E, dtype=np.int64)[flat]
+    pf = np.take_along_axis(np.cumsum(onehot, axis=0), flat[:, None], axis=1)[:, 0] - 1
+    pos = pf.reshape(T, k) if priority == 0 else pf.reshape(k, T).T
+    counts = np.bincount(flat, minlength=E)
+    kept = np.minimum(counts, C)
+    keep = (pos < C).astype(np.uint8)
+    np.testing.assert_array_equal(out.pos.cpu().numpy(), pos)
+    np.testing.assert_array_equal(out.keep.cpu().numpy(), keep)
+    np.testing.assert_array_equal(out.counts.cpu().numpy(), counts)
+    np.testing.assert_array_equal(out.kept.cpu().numpy(), kept)
+    np.testing.assert_array_equal(out.dropped.cpu().numpy(), (keep.sum(axis=1) == 0).astype(np.uint8))
+    padded = (kept + 127) // 128 * 128
+    np.testing.assert_array_equal(out.offsets.cpu().numpy(), np.concatenate([[0], np.cumsum(padded)]))
+    assert int(out.n_dropped.item()) == int((counts - kept).sum())
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_dispatch_and_combine_move_rows_exactly(dtype):
+    T, d, E, k = 300, 128, 8, 2
+    tdt = torch.bfloat16 if dtype else torch.float32
+    rng = np.random.default_rng(5)
+    topk = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    cfg = moe.moe_config(T=T, d=d, E=E, k=k, d_ff=64, dtype=dtype, cf=1.0)
+    cap = moe.moe_capacity(cfg, torch.tensor(topk, device=DEV))
+    x = torch.randn((T, d), device=DEV).to(tdt)
+    xp = moe.moe_dispatch(cfg, x, torch.tensor(topk, device=DEV), cap.pos, cap.keep, cap.offsets)
+    pos, keep, off = cap.pos.cpu().numpy(), cap.keep.cpu().numpy(), cap.offsets.cpu().numpy()
+    xp_c, x_c = xp.cpu(), x.cpu()
+    for t in range(T):
+        for j in range(k):
+            if keep[t, j]:
+                assert torch.equal(xp_c[off[topk[t, j]] + pos[t, j]], x_c[t])
+    # combine: y = sum_j keep g Y_perm[row] + Y_sh + residual, fp32 accumulation in slot order
+    Y_perm = torch.randn_like(xp)
+    Y_sh = torch.randn((T, d), device=DEV).to(tdt)
+    res = torch.randn((T, d), device=DEV).to(tdt)
+    gates = torch.rand((T, k), device=DEV)
+    y = moe.moe_combine(cfg, Y_perm, Y_sh, gates, torch.tensor(topk, device=DEV), cap.pos,
+                        cap.keep, cap.offsets, residual=res)
+    ref = torch.zeros((T, d), dtype=torch.float32)
+    Yp, g = Y_perm.cpu().float(), gates.cpu()
+    for t in range(T):
+        for j in range(k):
+            if keep[t, j]:
+                ref[t] = ref[t] + g[t, j] * Yp[off[topk[t, j]] + pos[t, j]]
+    ref = ref + Y_sh.cpu().float() + res.cpu().float()
+    tol = 1e-6 if dtype == 0 else 8e-3
+    assert (y.cpu().float() - ref).abs().max().item() <= tol * max(ref.abs().max().item(), 1.0)
+
+
+def test_route_logits_and_selection_against_torch():
+    T, d, E, k = 1000, 512, 64, 6
+    g = torch.Generator(device=DEV).manual_seed(9)
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    W_r = torch.randn((d, E), generator=g, device=DEV) * 0.05
+    cfg = moe.moe_config(T=T, d=d, E=E, k=k, d_ff=64, dtype=1, cf=1.0)
+    topk, gates, part, logits, scores = moe.moe_route(cfg, x, W_r, want_logits=True,
+                                                      want_scores=True)
+    z = x.double() @ W_r.double()
+    # recursive fp32 summation bound: |dz| <= d * 2^-24 * sum |x_c W_c|
+    bound = d * 2.0 ** -24 * (x.double().abs() @ W_r.double().abs())
+    assert torch.all((logits.double() - z).abs() <= bound + 1e-7)
+    p = torch.softmax(z, dim=1)
+    assert (scores.double() - p).abs().max().item() < 1e-6
+    # top-k of the GPU's own logits, lower index on ties
+    lz = logits.double().cpu().numpy()
+    ref = np.argsort(-lz, axis=1, kind="stable")[:, :k]
+    np.testing.assert_array_equal(topk.cpu().numpy(), ref)
+    sel = torch.gather(z, 1, topk.long())
+    assert (gates.double() - torch.softmax(sel, dim=1)).abs().max().item() < 1e-5
+
+
+def test_status_word_is_clear_after_a_normal_call():
+    cfg = moe.moe_config(T=128, d=128, E=2, k=1, d_ff=128, act=1, dtype=1, cf=math.inf)
+    R = moe.moe_perm_rows(cfg)
+    x_perm = torch.zeros((R, 128), dtype=torch.bfloat16, device=DEV)
+    W = torch.zeros((2, 128, 128), dtype=torch.bfloat16, device=DEV)
+    off = torch.tensor([0, 128, 128], dtype=torch.int32, device=DEV)
+    Y, _, ws = moe.moe_expert_ffn(cfg, x_perm, off, W, W, W)
+    assert moe.moe_device_status(ws) == 0
+    assert torch.count_nonzero(Y[:128]).item() == 0
