@@ -235,7 +235,8 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm,
  *          + Y_shared[t] (+ residual[t])
  * summed in fp32 in that order and stored as dtype.  A token with every slot
  * dropped gets Y_shared[t] (or 0), plus the residual when given.
- *   Y_shared, residual [T, d] dtype: nullable.
+ *   Y_shared [T, d] dtype: required when S > 0, added whenever given.
+ *   residual [T, d] dtype: nullable.
  */
 moe_status moe_combine(const moe_config *cfg, const void *Y_perm,
                        const void *Y_shared, const float *gates,

@@ -310,8 +310,8 @@ moe_status moe_combine(const moe_config *cfg, const void *Y_perm, const void *Y_
     for (const void *p : ptrs)
         if (p && !aligned16(p))
             return MOE_ERR_ALIGN;
-    return cuda_status(launch_combine(*cfg, Y_perm, cfg->n_shared > 0 ? Y_shared : nullptr,
-                                      gates, topk_idx, pos, keep, offsets, residual, y,
+    return cuda_status(launch_combine(*cfg, Y_perm, Y_shared, gates, topk_idx, pos, keep,
+                                      offsets, residual, y,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
