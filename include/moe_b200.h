@@ -197,6 +197,32 @@ moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx,
                         moe_stream_t stream);
 
 /*
+ * moe_capacity_noalloc - moe_capacity with its scratch inside the library.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory where they run the capacity step (memory
+ * planned once at start-up that may not grow, or device memory owned by
+ * another allocator that must not be bypassed).  The caller still allocates
+ * and passes every input and output; the arguments mean what they mean for
+ * moe_capacity, and the results are identical to it.
+ *   - The scratch is a file-scope device array of 512 KiB (two tables of
+ *     65536 int32), held by every GPU that loads the library until the process
+ *     exits.  Shapes that need more, ceil(T / 256) * k * E > 65536, return
+ *     MOE_ERR_WORKSPACE and launch nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - No cudaMalloc, cudaFree or other allocating call is made.
+ *   - All calls share the one array: calls whose work overlaps on the GPU
+ *     (other streams, other threads) race and give wrong results.  Each call
+ *     writes every scratch entry it reads, so nothing needs clearing between
+ *     calls.
+ */
+moe_status moe_capacity_noalloc(const moe_config *cfg, const int32_t *topk_idx,
+                                int32_t *counts, int32_t *pos, uint8_t *keep,
+                                int32_t *kept, int32_t *offsets, uint8_t *dropped,
+                                int32_t *n_dropped, moe_stream_t stream);
+
+/*
  * moe_dispatch - permute token rows into expert-grouped order ("Lab 18" tips:
  * gather each expert's tokens and run the expert once on them).
  *   x [T, d] dtype in; topk_idx, pos, keep, offsets from moe_capacity.

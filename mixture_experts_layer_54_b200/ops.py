@@ -135,6 +135,26 @@ def moe_capacity(cfg: MoeConfig, topk, ws=None) -> CapacityOut:
     return out
 
 
+def moe_capacity_noalloc(cfg: MoeConfig, topk) -> CapacityOut:
+    """moe_capacity with the library's own static scratch instead of a
+    workspace (for callers that cannot allocate device memory)."""
+    dev = _dev(topk)
+    T, k, E = cfg.T, cfg.k, cfg.E
+    out = CapacityOut(
+        counts=torch.empty((E,), dtype=torch.int32, device=dev),
+        pos=torch.empty((T, k), dtype=torch.int32, device=dev),
+        keep=torch.empty((T, k), dtype=torch.uint8, device=dev),
+        kept=torch.empty((E,), dtype=torch.int32, device=dev),
+        offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+        dropped=torch.empty((T,), dtype=torch.uint8, device=dev),
+        n_dropped=torch.empty((1,), dtype=torch.int32, device=dev))
+    check(lib().moe_capacity_noalloc(ctypes.byref(cfg), _p(topk), _p(out.counts), _p(out.pos),
+                                     _p(out.keep), _p(out.kept), _p(out.offsets),
+                                     _p(out.dropped), _p(out.n_dropped), _stream()),
+          "moe_capacity_noalloc")
+    return out
+
+
 def moe_dispatch(cfg: MoeConfig, x, topk, pos, keep, offsets, x_perm=None):
     if x_perm is None:
         x_perm = torch.empty((moe_perm_rows(cfg), cfg.d), dtype=_tdtype(cfg), device=_dev(x))
@@ -238,6 +258,7 @@ def moe_forward(cfg: MoeConfig, x, W_r, W1, W2, W3=None, logit_bias=None, select
 
 
 __all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
+           "moe_capacity_noalloc",
            "moe_loss_partials_count", "moe_stage_workspace_size", "moe_workspace_size",
            "workspace", "moe_route", "moe_capacity", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_losses", "moe_device_status", "weights_struct", "MoEForward",
