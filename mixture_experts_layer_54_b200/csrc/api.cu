@@ -52,6 +52,7 @@ int64_t perm_rows(const moe_config &c)
 }
 
 int route_blocks(const moe_config &c) { return (int)ceil_div(c.T, kRouteTokens); }
+int partial_rows(const moe_config &c) { return (int)ceil_div(c.T, kPartialTokens); }
 int cap_blocks(const moe_config &c) { return (int)ceil_div(c.T, kCapTokens); }
 
 namespace {
@@ -95,7 +96,7 @@ void carve_forward_into(const moe_config &c, Carver &cv, ForwardBufs &f)
     const size_t A = (size_t)c.T * c.k;
     f.topk = static_cast<int32_t *>(cv.take(A * 4));
     f.gates = static_cast<float *>(cv.take(A * 4));
-    f.partials = static_cast<float *>(cv.take((size_t)route_blocks(c) * (c.E + 1) * 4));
+    f.partials = static_cast<float *>(cv.take((size_t)partial_rows(c) * (c.E + 1) * 4));
     f.counts = static_cast<int32_t *>(cv.take((size_t)c.E * 4));
     f.kept = static_cast<int32_t *>(cv.take((size_t)c.E * 4));
     f.offsets = static_cast<int32_t *>(cv.take((size_t)(c.E + 1) * 4));
@@ -183,7 +184,7 @@ int64_t moe_perm_rows(const moe_config *cfg)
 
 int64_t moe_loss_partials_count(const moe_config *cfg)
 {
-    return check_cfg(cfg) == MOE_OK ? (int64_t)route_blocks(*cfg) * (cfg->E + 1) : -1;
+    return check_cfg(cfg) == MOE_OK ? (int64_t)partial_rows(*cfg) * (cfg->E + 1) : -1;
 }
 
 size_t moe_stage_workspace_size(const moe_config *cfg)

@@ -539,6 +539,386 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     }
 }
 
+// ===================================================================== 2-SM
+// The same grouped GEMM on SM pairs (cta_group::2): a 2-CTA cluster owns a
+// 256-row x 256-column accumulator tile, each CTA holding 128 rows of it in
+// its own TMEM.  Each CTA loads its 128 rows of A and its half of the B tile
+// (SwiGLU: CTA 0 the W1 rows, CTA 1 the same W3 rows), so a K step moves 32 KB
+// into each SM instead of 48 KB, and six stages fit.  The leader CTA's MMA
+// thread issues the M = 256 MMAs for both; its commits are multicast to the
+// empty / accumulator-full barriers of both CTAs; both CTAs' TMA loads report
+// to the leader's full barriers; both CTAs' epilogues report to the leader's
+// accumulator-empty barriers.  A 256-row pair tile lies inside one expert's
+// segment; when the segment ends after the first 128 rows, CTA 1 computes
+// rows it does not store.
+
+constexpr int STAGES2 = 6;
+constexpr int HALF_BYTES = 128 * BK * 2;             // 16 KB: 128 rows x 64 bf16
+constexpr int OFF2_A = 0;
+constexpr int OFF2_B = OFF2_A + STAGES2 * HALF_BYTES;
+constexpr int OFF2_STG = OFF2_B + STAGES2 * HALF_BYTES;
+constexpr int OFF2_BAR = OFF2_STG + EPI_WARPS * 2 * STG_BYTES;
+constexpr int OFF2_TILES = OFF2_BAR + 256;
+constexpr int SMEM2_BYTES = OFF2_TILES + 2 * 4 * (kMaxE + 1) + 1024;
+
+// kind::f16, fp32 accumulator, bf16 A and B, K-major, N = 256, M = 256
+constexpr uint32_t IDESC2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the same shared variable in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank)
+{
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+    return out;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                     "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t bar_leader, int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar_leader)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(IDESC2), "r"(accumulate)
+        : "memory");
+}
+
+// arrive on the barrier at this shared offset in both CTAs of the pair
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar)
+{
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n\t}" ::"r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_local2(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                     "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+struct Tile2 {
+    int set;
+    int m0;        // first row of the pair tile
+    int b_group;   // B group when K is not split
+    int n_idx;     // N tile index inside the group
+    int c_group;
+    bool second;   // rows m0 + 128 .. belong to the tile's segment
+};
+
+__device__ __forceinline__ Tile2 decode2(const Params &p, const int *tstart, const int *mpairs,
+                                         int routed_total, int tile)
+{
+    Tile2 t;
+    if (tile < routed_total) {
+        int lo = 0, hi = p.E;
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (tstart[mid] <= tile)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int e = lo, i = tile - tstart[e], mp = mpairs[e];
+        t.set = 0;
+        t.m0 = p.offsets[e] + (i % mp) * 256;
+        t.second = t.m0 + 128 < p.offsets[e + 1];
+        t.b_group = e;
+        t.n_idx = i / mp;
+        t.c_group = 0;
+    } else {
+        const SetDesc &sd = p.set[1];
+        const int i = tile - routed_total;
+        const int mp = (sd.rows + 255) / 256;
+        const int n = i / mp;
+        t.set = 1;
+        t.m0 = (i % mp) * 256;
+        t.second = t.m0 + 128 < sd.rows;
+        t.b_group = n / sd.n_tiles;
+        t.n_idx = n % sd.n_tiles;
+        t.c_group = t.b_group;
+    }
+    return t;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __grid_constant__ Params p)
+{
+    constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;   // output columns per tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sA = smem_u32(smem + OFF2_A);
+    const uint32_t sB = smem_u32(smem + OFF2_B);
+    const uint32_t sStg = smem_u32(smem + OFF2_STG);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF2_BAR);
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES2 + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES2 + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES2 + 2 + a); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES2 + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF2_BAR + 8 * (2 * STAGES2 + 5));
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *tstart = reinterpret_cast<int *>(smem + OFF2_TILES);   // [E + 1]
+    int *mpairs = tstart + (kMaxE + 1);                        // [E]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const Ctl ctl{abort_flag, p.status, p.timeout_ns};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES2; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 2 * EPI_WARPS);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    int routed_total = 0;
+    if (p.set[0].routed && p.nsets > 0) {
+        for (int e = threadIdx.x; e < p.E; e += THREADS) {
+            const int mt = (p.offsets[e + 1] - p.offsets[e]) / BM;
+            mpairs[e] = (mt + 1) / 2;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int acc = 0;
+            for (int e = 0; e < p.E; ++e) {
+                tstart[e] = acc;
+                acc += mpairs[e] * p.set[0].n_tiles;
+            }
+            tstart[p.E] = acc;
+        }
+    }
+    tc_fence_before();
+    cluster_sync();   // barriers of both CTAs initialised, TMEM allocated, tables ready
+    tc_fence_after();
+    if (p.set[0].routed && p.nsets > 0)
+        routed_total = tstart[p.E];
+    int shared_total = 0;
+    if (p.nsets > 1) {
+        const SetDesc &sd = p.set[1];
+        shared_total = (sd.rows + 255) / 256 * sd.n_tiles * sd.n_groups;
+    }
+    const int total = routed_total + shared_total;
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ================= TMA producer (both CTAs) =================
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[STAGES2];
+            uint32_t last_phase[STAGES2];
+            for (int s = 0; s < STAGES2; ++s)
+                issued[s] = 0, last_phase[s] = 0;
+            bool ok = true;
+            for (int tile = cluster_id; ok && tile < total; tile += nclusters) {
+                const Tile2 t = decode2(p, tstart, mpairs, routed_total, tile);
+                const SetDesc &sd = p.set[t.set];
+                const int brow = EPI == EPI_SWIGLU ? t.n_idx * (BN / 2)
+                                                   : t.n_idx * BN + (int)rank * (BN / 2);
+                const CUtensorMap *bmap =
+                    (EPI == EPI_SWIGLU && rank == 1) ? &p.tmB3[t.set] : &p.tmB[t.set];
+                for (int kb = 0; kb < sd.k_blocks; ++kb) {
+                    if (!wait_bar(empty_bar(stage), phase ^ 1u, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    int kcol = kb * BK, ga = 0, gb = t.b_group;
+                    if (sd.kbg > 0) {
+                        ga = gb = kb / sd.kbg;
+                        kcol = (kb % sd.kbg) * BK;
+                    }
+                    if (leader)
+                        mbar_expect_tx(full_bar(stage), 4 * HALF_BYTES);
+                    const uint32_t fb = map_to_rank(full_bar(stage), 0);
+                    tma_load_3d_pair(sA + stage * HALF_BYTES, &p.tmA[t.set], fb, kcol,
+                                     t.m0 + (int)rank * 128, ga);
+                    tma_load_3d_pair(sB + stage * HALF_BYTES, bmap, fb, kcol, brow, gb);
+                    issued[stage] = 1;
+                    last_phase[stage] = phase;
+                    if (++stage == STAGES2) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // the leader's full barriers count both CTAs' bytes: drain there
+            if (leader)
+                for (int s = 0; s < STAGES2; ++s)
+                    if (issued[s])
+                        wait_bar(full_bar(s), last_phase[s], ctl, false);
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer (leader CTA only) =================
+        if (lane == 0 && leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, any = false;
+            for (int tile = cluster_id; ok && tile < total; tile += nclusters) {
+                const Tile2 t = decode2(p, tstart, mpairs, routed_total, tile);
+                const SetDesc &sd = p.set[t.set];
+                if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < sd.k_blocks; ++kb) {
+                    if (!wait_bar(full_bar(stage), phase, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = sA + stage * HALF_BYTES, b_base = sB + stage * HALF_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16_pair(tmem_d, sdesc_sw128(a_base + kk * 32),
+                                      sdesc_sw128(b_base + kk * 32), (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit_pair(empty_bar(stage));
+                    any = true;
+                    if (++stage == STAGES2) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                mma_commit_pair(tfull_bar(acc));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (any) {
+                mma_commit_local2(drain_bar);
+                wait_bar(drain_bar, 0, ctl, false);
+            }
+        }
+    } else {
+        // ================= epilogue (warps 2..5, both CTAs) =================
+        const int q = warp & 3;
+        const int ew = warp - 2;
+        const uint32_t stg0 = sStg + ew * 2 * STG_BYTES;
+        uint8_t *stg_ptr0 = smem + OFF2_STG + ew * 2 * STG_BYTES;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int buf = 0;
+        for (int tile = cluster_id; tile < total; tile += nclusters) {
+            const Tile2 t = decode2(p, tstart, mpairs, routed_total, tile);
+            if (!wait_bar(tfull_bar(acc), acc_phase, ctl))
+                break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            const int c_col = t.n_idx * BN_OUT;
+            const int c_end = (rank == 0 || t.second) ? min(BN_OUT, p.set[t.set].c_cols - c_col) : 0;
+            const int row = t.m0 + (int)rank * 128 + q * 32;
+#pragma unroll 1
+            for (int c = 0; c < c_end; c += CHUNK) {
+                float g[CHUNK], u[CHUNK];
+                uint32_t packed[CHUNK / 2];
+                tmem_ld32(tbase + c, g);
+                if (EPI == EPI_SWIGLU) {
+                    tmem_ld32(tbase + BN / 2 + c, u);
+                    epilogue_chunk<EPI>(g, u, packed);
+                } else {
+                    epilogue_chunk<EPI>(g, g, packed);
+                }
+                if (lane == 0)
+                    bulk_wait_read1();
+                __syncwarp();
+                uint8_t *rowp = stg_ptr0 + buf * STG_BYTES + lane * 64;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int phys = ch ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4 *>(rowp + phys * 16) =
+                        make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2],
+                                   packed[4 * ch + 3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&p.tmC[t.set], stg0 + buf * STG_BYTES, c_col + c, row, t.c_group);
+                    bulk_commit();
+                }
+                buf ^= 1;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_remote(map_to_rank(tempty_bar(acc), 0));
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0)
+            bulk_wait_all();
+        __syncwarp();
+    }
+
+    // ---- tear-down: both CTAs done with the pair's TMEM before it is freed ----
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
 // ------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -586,6 +966,39 @@ int sm_count()
 }
 
 template <int EPI>
+cudaError_t launch_2sm(const Params &p, cudaStream_t s)
+{
+    auto kern = grouped_gemm_2sm_kernel<EPI>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+    if (err != cudaSuccess)
+        return err;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    int clusters = 0;
+    err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    if (err != cudaSuccess)
+        return err;
+    if (clusters < 1)
+        return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    err = cudaLaunchKernelEx(&cfg, kern, p);
+    if (err != cudaSuccess)
+        return err;
+    return cudaGetLastError();
+}
+
+template <int EPI>
 cudaError_t launch(const Params &p, cudaStream_t s)
 {
     auto kern = grouped_gemm_kernel<EPI>;
@@ -608,7 +1021,16 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     const uint64_t R = (uint64_t)perm_rows(c), d = c.d, F = c.d_ff, E = c.E;
     const uint64_t T = c.T, S = c.n_shared, Fs = c.d_ff_shared;
     const bool swiglu = c.act == MOE_ACT_SWIGLU;
-    const int bn_b = swiglu ? BN / 2 : BN;
+    // SM-pair tiles (256 rows) when experts average at least 512 rows; single-SM
+    // tiles (128 rows) for small segments, where a 256-row tile would mostly
+    // compute padding.
+    const bool pair = (int64_t)c.T * c.k >= (int64_t)512 * c.E;
+    // B rows one TMA box brings into one CTA: half the 256-column accumulator
+    // for SwiGLU (W1 and W3 halves) and for every SM-pair tile (one half per
+    // CTA), the whole 256 otherwise.  The box must match what the kernel
+    // expects, or the stage's byte count is wrong.
+    const int bn_b = (swiglu || pair) ? BN / 2 : BN;
+    const int bn2_b = pair ? BN / 2 : BN;
     const int bn_out = swiglu ? BN / 2 : BN;
     const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B, SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
     const bool shared = S > 0 && T > 0;
@@ -640,7 +1062,8 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     }
     if (!ok)
         return cudaErrorInvalidValue;
-    cudaError_t err = swiglu ? launch<EPI_SWIGLU>(p1, s) : launch<EPI_GELU>(p1, s);
+    cudaError_t err = pair ? (swiglu ? launch_2sm<EPI_SWIGLU>(p1, s) : launch_2sm<EPI_GELU>(p1, s))
+                           : (swiglu ? launch<EPI_SWIGLU>(p1, s) : launch<EPI_GELU>(p1, s));
     if (err != cudaSuccess)
         return err;
 
@@ -654,19 +1077,19 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     p2.nsets = shared ? 2 : 1;
     ok = true;
     ok &= make_map(&p2.tmA[0], H, F, R, 1, F * 2, 0, BK, BM, SW128);
-    ok &= make_map(&p2.tmB[0], W2, F, d, E, F * 2, d * F * 2, BK, BN, SW128);
+    ok &= make_map(&p2.tmB[0], W2, F, d, E, F * 2, d * F * 2, BK, bn2_b, SW128);
     ok &= make_map(&p2.tmC[0], Y_perm, d, R, 1, d * 2, 0, CHUNK, 32, SW64);
     p2.set[0] = SetDesc{1, 0, (int)ceil_div(d, BN), 1, (int)ceil_div(F, BK), 0, (int)d};
     if (shared) {
         ok &= make_map(&p2.tmA[1], H_sh, Fs, T, S, Fs * 2, T * Fs * 2, BK, BM, SW128);
-        ok &= make_map(&p2.tmB[1], Ws2, Fs, d, S, Fs * 2, d * Fs * 2, BK, BN, SW128);
+        ok &= make_map(&p2.tmB[1], Ws2, Fs, d, S, Fs * 2, d * Fs * 2, BK, bn2_b, SW128);
         ok &= make_map(&p2.tmC[1], Y_sh, d, T, 1, d * 2, 0, CHUNK, 32, SW64);
         const int kbg = (int)ceil_div(Fs, BK);
         p2.set[1] = SetDesc{0, (int)T, (int)ceil_div(d, BN), 1, kbg * (int)S, kbg, (int)d};
     }
     if (!ok)
         return cudaErrorInvalidValue;
-    return launch<EPI_NONE>(p2, s);
+    return pair ? launch_2sm<EPI_NONE>(p2, s) : launch<EPI_NONE>(p2, s);
 }
 
 }  // namespace moe

@@ -10,34 +10,44 @@
 namespace moe {
 namespace {
 
-constexpr int THREADS = 256;
+constexpr int THREADS = 1024;
 
+// Column c of the partials (expert c < E, or the lse^2 column c = E) is
+// summed by ny threads, each over rows y, y + ny, ... in order, then the ny
+// partial sums in order: a fixed reduction tree, so the result does not depend
+// on timing.
 __global__ void __launch_bounds__(THREADS)
-losses_kernel(const int32_t *counts, const float *partials, int nblk, int T, int k, int E,
+losses_kernel(const int32_t *counts, const float *partials, int rows, int T, int k, int E,
               float *aux, float *zloss)
 {
-    __shared__ double term[THREADS];
-    double acc = 0.0;
-    // expert i: P_i summed over blocks in block order, times f_i
-    for (int i = threadIdx.x; i < E; i += THREADS) {
-        double P = 0.0;
-        for (int b = 0; b < nblk; ++b)
-            P += (double)partials[(int64_t)b * (E + 1) + i];
-        acc += ((double)counts[i] / ((double)T * (double)k)) * (P / (double)T);
+    extern __shared__ double part[];   // [ny][C]
+    __shared__ double term[kMaxE + 1];
+    const int C = E + 1;
+    const int ny = THREADS / C;
+    const int tx = threadIdx.x % C, ty = threadIdx.x / C;
+    if (ty < ny) {
+        double s = 0.0;
+        for (int r = ty; r < rows; r += ny)
+            s += (double)partials[(int64_t)r * C + tx];
+        part[ty * C + tx] = s;
     }
-    term[threadIdx.x] = acc;
     __syncthreads();
-    for (int s = THREADS / 2; s > 0; s >>= 1) {
-        if (threadIdx.x < s)
-            term[threadIdx.x] += term[threadIdx.x + s];
-        __syncthreads();
+    if (threadIdx.x < C) {
+        double s = 0.0;
+        for (int y = 0; y < ny; ++y)
+            s += part[y * C + threadIdx.x];
+        term[threadIdx.x] = threadIdx.x < E
+                                ? ((double)counts[threadIdx.x] / ((double)T * (double)k)) *
+                                      (s / (double)T)
+                                : s / (double)T;
     }
+    __syncthreads();
     if (threadIdx.x == 0) {
-        double z = 0.0;
-        for (int b = 0; b < nblk; ++b)
-            z += (double)partials[(int64_t)b * (E + 1) + E];
-        *aux = (float)((double)E * term[0]);
-        *zloss = (float)(z / (double)T);
+        double a = 0.0;
+        for (int i = 0; i < E; ++i)
+            a += term[i];
+        *aux = (float)((double)E * a);
+        *zloss = (float)term[E];
     }
 }
 
@@ -46,8 +56,10 @@ losses_kernel(const int32_t *counts, const float *partials, int nblk, int T, int
 cudaError_t launch_losses(const moe_config &c, const int32_t *counts, const float *partials,
                           float *aux, float *zloss, cudaStream_t s)
 {
-    losses_kernel<<<1, THREADS, 0, s>>>(counts, partials, route_blocks(c), c.T > 0 ? c.T : 1,
-                                        c.k, c.E, aux, zloss);
+    const int C = c.E + 1;
+    const size_t smem = sizeof(double) * (THREADS / C) * C;
+    losses_kernel<<<1, THREADS, smem, s>>>(counts, partials, partial_rows(c),
+                                           c.T > 0 ? c.T : 1, c.k, c.E, aux, zloss);
     return cudaGetLastError();
 }
 

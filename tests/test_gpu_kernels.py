@@ -43,15 +43,17 @@ def _segments(kept, align=128):
     return offsets
 
 
+@pytest.mark.parametrize("pair", [False, True], ids=["1sm", "2sm"])
 @pytest.mark.parametrize("act", [0, 1])
 @pytest.mark.parametrize("dims", [(256, 384), (512, 128), (192, 256)])
-def test_expert_ffn_grouped_gemm_against_torch(act, dims):
+def test_expert_ffn_grouped_gemm_against_torch(act, dims, pair):
     """Ragged segments (empty, 1 row, 127, 128, 129, several tiles) through the
-    tcgen05 grouped GEMM; every kept row compared with its expert's FFN."""
+    tcgen05 grouped GEMM; every kept row compared with its expert's FFN.  T*k
+    >= 512*E selects SM-pair (256-row) tiles, smaller T single-SM tiles."""
     d, F = dims
     kept = [0, 1, 127, 128, 129, 300, 5, 260]
     E = len(kept)
-    T = 400
+    T = 2048 if pair else 400
     cfg = moe.moe_config(T=T, d=d, E=E, k=2, d_ff=F, act=act, dtype=1, cf=math.inf)
     R = moe.moe_perm_rows(cfg)
     offsets = _segments(kept)
@@ -74,9 +76,10 @@ def test_expert_ffn_grouped_gemm_against_torch(act, dims):
         _close_bf16(Y[rows], ref)
 
 
-@pytest.mark.parametrize("act,S", [(1, 2), (0, 1), (1, 1)])
-def test_shared_experts_against_torch(act, S):
-    d, F, Fs, T, E = 256, 128, 192, 333, 4
+@pytest.mark.parametrize("act,S,T", [(1, 2, 333), (0, 1, 333), (1, 1, 333), (1, 2, 2100),
+                                     (0, 1, 2100)])
+def test_shared_experts_against_torch(act, S, T):
+    d, F, Fs, E = 256, 128, 192, 4
     cfg = moe.moe_config(T=T, d=d, E=E, k=1, d_ff=F, act=act, dtype=1, cf=math.inf,
                          n_shared=S, d_ff_shared=Fs)
     R = moe.moe_perm_rows(cfg)
