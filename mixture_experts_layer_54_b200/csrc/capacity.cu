@@ -45,9 +45,10 @@ __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int 
 }
 
 __global__ void __launch_bounds__(1024)
-cap_scan_kernel(const int32_t *hist, int nblk, int k, int E, int priority, long long C,
-                int32_t *base, int32_t *counts, int32_t *kept, int32_t *offsets,
-                int32_t *n_dropped)
+cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int priority,
+                long long C, int32_t *__restrict__ base, int32_t *__restrict__ counts,
+                int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
+                int32_t *__restrict__ n_dropped)
 {
     __shared__ int32_t total[kMaxK * kMaxE];   // per (j, e), all blocks
     __shared__ int32_t cnt[kMaxE];
@@ -55,6 +56,7 @@ cap_scan_kernel(const int32_t *hist, int nblk, int k, int E, int priority, long 
     // exclusive scan over blocks of each (j, e) column
     for (int col = threadIdx.x; col < cols; col += blockDim.x) {
         int run = 0;
+#pragma unroll 8
         for (int b = 0; b < nblk; ++b) {
             int v = hist[(int64_t)b * cols + col];
             base[(int64_t)b * cols + col] = run;
