@@ -1,0 +1,80 @@
+"""Host-side logic of the benchmark on CPU: two gloo ranks agree on the slowest
+rank's time, and the workload accounting is what the design doc states."""
+import math
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from moe_inputs import CONFIGS
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dev = torch.device("cpu")
+        bench.barrier(dev)
+        t = bench.max_over_ranks(1.5 + rank, dev)
+        again = bench.max_over_ranks(10.0 - rank, dev)
+        out[rank] = (t, again, bench.dist_env())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    for rank in range(world):
+        t, again, env = res[rank]
+        assert t == 2.5 and again == 10.0
+        assert env == (world, rank, rank)
+
+
+def test_single_process_needs_no_process_group():
+    assert bench.max_over_ranks(3.25, torch.device("cpu")) == 3.25
+
+
+def test_layer_work_counts_only_algorithmic_flops():
+    s = CONFIGS["mixtral"]
+    w = bench.layer_work(s, None, kept_total=2 * s.T, dropped_tokens=0)
+    # three matrices of d x d_ff per kept assignment, 2 FLOP per multiply-add
+    assert w["expert_ffn"]["flops"] == 2.0 * 3 * (2 * s.T) * s.d * s.d_ff
+    assert w["dispatch"]["bytes"] == s.T * s.d * 2 + 2 * s.T * s.d * 2 + s.T * s.k * 9
+    ds = CONFIGS["deepseekmoe"]
+    wd = bench.layer_work(ds, None, kept_total=ds.T * ds.k, dropped_tokens=0)
+    shared = 2.0 * 3 * ds.n_shared * ds.T * ds.d * ds.d_ff_shared
+    assert wd["expert_ffn"]["flops"] == 2.0 * 3 * ds.T * ds.k * ds.d * ds.d_ff + shared
+    assert wd["route"]["bytes"] == ds.T * ds.d * 2 + ds.d * ds.E * 4 + ds.T * ds.k * 8 + \
+        math.ceil(ds.T / 4) * (ds.E + 1) * 4
+
+
+def test_clock_summary_flags_throttle_reasons():
+    c = bench.ClockSampler(0)
+    c.lines = ["0, 1900, 1965, 900.0, 0x1, Not Active, Not Active, Not Active, Active",
+               "0, 1800, 1965, 990.0, 0x1, Not Active, Active, Not Active, Active",
+               "garbage"]
+    s = c.summary()
+    assert s["sm_mhz"] == 1850.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"] and s["samples"] == 2
+
+
+def test_peaks_fall_back_when_the_file_is_missing(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert src == "fallback" and peaks["hbm_gbs"] == 6650.0
