@@ -43,8 +43,31 @@ from moe_inputs import CONFIGS, generate, seed_for  # noqa: E402
 
 METRIC = "MoE layer fwd tokens/s on 1 B200; grouped-GEMM % BF16 peak; dispatch % HBM BW"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 9   # route 1, capacity 3, dispatch 1, expert FFN 2, combine 1, losses 1
+def kernels_per_step(shape) -> int:
+    """Kernels of ours one forward launches: route (bf16: weight split, logits,
+    select; fp32: one), capacity 3, dispatch 1, expert FFN (bf16: the two
+    grouped GEMMs; fp32: two, plus two for shared experts), combine 1, losses 1."""
+    route = 3 if shape.dtype == 1 else 1
+    ffn = 2 if shape.dtype == 1 else (4 if shape.n_shared else 2)
+    return route + 3 + 1 + ffn + 1 + 1
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes (read + write) of the expert-FFN stage (GEMM1 + GEMM2) per launch, from one ncu
+# capture (profiles/gemm_2sm_mixtral.md), valid only for the GEMM source it was taken on.
+GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_54_b200", "csrc", "ffn_tcgen05.cu")
+MEASURED_TRAFFIC = {
+    ("mixtral", "2552d78e7c3833aa21e3be7d002760efa36ebea2f049ef2fced01ea7231f723c"): 5.752e9,
+}
+
+
+def measured_traffic(config: str):
+    import hashlib
+    try:
+        with open(GEMM_SOURCE, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return MEASURED_TRAFFIC.get((config, sha))
 
 
 def parse(argv=None):
@@ -302,19 +325,28 @@ def run_ours(args):
         raise SystemExit(f"device status {status} after warm-up: the expert GEMM gave up "
                          "waiting; not timing a failing kernel")
 
-    # ---- device-timed region: K steps, events between the stages ----
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+    # ---- device-timed region: the K steps, captured once in a CUDA graph with
+    # timing events between the stages, replayed once between barriers ----
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nst + 1)]
               for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        for i in range(args.steps):
+            staged(*wargs, events=events[i])
+    torch.cuda.synchronize()
     barrier(dev)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            staged(*wargs, events=events[i])
+        graph.replay()
         torch.cuda.synchronize()
     barrier(dev)
+    status = moe.moe_device_status(staged.ws)
+    if status != 0:
+        raise SystemExit(f"device status {status} in the timed region")
     total_ms = events[0][0].elapsed_time(events[-1][-1])
     stage_ms = [sum(ev[s].elapsed_time(ev[s + 1]) for ev in events) / args.steps
                 for s in range(nst)]
+    del graph
     ms_per_step = max_over_ranks(total_ms / args.steps, dev)
 
     # ---- end to end: pinned host input in, result out, inside the timed region ----
@@ -367,7 +399,9 @@ def run_ours(args):
     ach = ffn["flops"] / (st["expert_ffn"] / 1e3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
-                "traffic": None,
+                "traffic": measured_traffic(args.config),
+                "traffic_unit": "bytes per launch (ncu dram read + write, GEMM1 + GEMM2)",
+                "algorithmic_bytes": ffn["bytes"],
                 "kernel": "moe_expert_ffn: grouped tcgen05 GEMM1 (act fused) + GEMM2",
                 "flops_per_launch": ffn["flops"],
                 "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
@@ -393,7 +427,8 @@ def run_ours(args):
                        "kept_assignments": kept_total, "dropped_tokens": dropped_tokens},
             "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": kernels_per_step(shape) * args.steps,
+            "timing": "device: one CUDA graph of the K steps; e2e: direct moe_forward calls",
             "roofline": roofline, "layer_roofline": layer_roof, "stages": stages,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},

@@ -142,7 +142,8 @@ int64_t moe_perm_rows(const moe_config *cfg);
 /* Number of fp32 values moe_route writes to loss_partials. */
 int64_t moe_loss_partials_count(const moe_config *cfg);
 
-/* Scratch bytes the stage calls need (moe_capacity, moe_expert_ffn). */
+/* Scratch bytes the stage calls need (moe_route, moe_capacity,
+ * moe_expert_ffn).  One workspace serves all of them, one call at a time. */
 size_t moe_stage_workspace_size(const moe_config *cfg);
 
 /* Workspace bytes moe_forward needs (includes the stage scratch).  0 for an
@@ -165,12 +166,19 @@ size_t moe_workspace_size(const moe_config *cfg);
  *     by moe_losses in a fixed order.
  *   logits_out [T, E] fp32, nullable: the router logits z.
  *   scores_out [T, E] fp32, nullable: p (softmax) or s (sigmoid).
- * Logits are computed in fp32 from the exact fp32 widening of x.
+ *   ws: scratch of at least moe_stage_workspace_size bytes, 256-byte aligned;
+ *     its first word is the device status word (cleared by this call).
+ * Logits are fp32: for bf16 x the tensor cores compute x W_hi + x W_mid +
+ * x W_lo, where hi + mid + lo is an exact three-term bf16 split of each fp32
+ * weight, so every product is exact and the sum accumulates in fp32; fp32 x
+ * uses fp32 FMAs.  A wait that times out sets MOE_ERR_DEVICE_TIMEOUT in the
+ * status word (see moe_device_status); the routing is then not valid.
  */
 moe_status moe_route(const moe_config *cfg, const void *x, const float *W_r,
                      const float *logit_bias, const float *select_bias,
                      int32_t *topk_idx, float *gates, float *loss_partials,
-                     float *logits_out, float *scores_out, moe_stream_t stream);
+                     float *logits_out, float *scores_out, void *ws, size_t ws_bytes,
+                     moe_stream_t stream);
 
 /*
  * moe_capacity - slot assignment under the capacity limit ("Lab 18" section 3;
@@ -243,7 +251,8 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x,
  *     experts (all NULL when S = 0).
  *   Y_perm [moe_perm_rows, d] dtype out: FFN_e of each row of segment e.
  *   Y_shared [T, d] dtype out (NULL when S = 0): sum over s of FFN_s(x_t).
- *   ws: scratch (hidden activations), moe_stage_workspace_size bytes.
+ *   ws: scratch (hidden activations), moe_stage_workspace_size bytes; its
+ *     first word is the device status word (cleared by this call).
  * bf16 runs on the tensor cores (tcgen05, fp32 accumulation, hidden
  * activations rounded to bf16); fp32 runs on the CUDA cores in fp32.
  */
@@ -294,10 +303,11 @@ moe_status moe_forward(const moe_config *cfg, const moe_weights *w,
                        size_t ws_bytes, moe_stream_t stream);
 
 /*
- * moe_device_status - read the device status word that the expert GEMM's
- * bounded waits set when they give up (MOE_OK or MOE_ERR_DEVICE_TIMEOUT).
- * ws is the workspace passed to moe_expert_ffn / moe_forward; *status is host
- * memory.  Synchronises `stream` (a cudaMemcpyAsync followed by a stream
+ * moe_device_status - read the device status word that the bounded waits of
+ * the tensor-core kernels (router, expert GEMMs) set when they give up
+ * (MOE_OK or MOE_ERR_DEVICE_TIMEOUT).  moe_route and moe_expert_ffn clear it
+ * when they start, moe_forward once for the whole layer.  ws is the workspace
+ * passed to those calls; *status is host memory.  Synchronises `stream` (a cudaMemcpyAsync followed by a stream
  * synchronise) - the only call in this library that does.
  */
 moe_status moe_device_status(const void *ws, int32_t *status,

@@ -51,7 +51,8 @@ SIGNATURES = {
     "moe_loss_partials_count": (ctypes.c_int64, [_CFG]),
     "moe_stage_workspace_size": (ctypes.c_size_t, [_CFG]),
     "moe_workspace_size": (ctypes.c_size_t, [_CFG]),
-    "moe_route": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_route": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                 _P]),
     "moe_capacity": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                     _P]),
     "moe_capacity_noalloc": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),

@@ -76,10 +76,17 @@ void carve_stage_into(const moe_config &c, Carver &cv, StageScratch &s)
     const size_t esz = dtype_bytes(c.dtype);
     const size_t hk = (size_t)cap_blocks(c) * c.k * c.E * sizeof(int32_t);
     s.status = static_cast<int32_t *>(cv.take(kAlign));
-    s.hist = static_cast<int32_t *>(cv.take(hk));
-    s.base = static_cast<int32_t *>(cv.take(hk));
-    s.H = cv.take((size_t)R * c.d_ff * esz);
-    s.H_sh = cv.take((size_t)c.n_shared * c.T * (c.n_shared ? c.d_ff_shared : 0) * esz);
+    // one shared region: the largest of the three stages' scratch
+    const size_t off = cv.off;
+    Carver route_cv{cv.base, off}, cap_cv{cv.base, off}, ffn_cv{cv.base, off};
+    s.route = route_cv.take(route_scratch_bytes(c));
+    s.hist = static_cast<int32_t *>(cap_cv.take(hk));
+    s.base = static_cast<int32_t *>(cap_cv.take(hk));
+    s.H = ffn_cv.take((size_t)R * c.d_ff * esz);
+    s.H_sh = ffn_cv.take((size_t)c.n_shared * c.T * (c.n_shared ? c.d_ff_shared : 0) * esz);
+    cv.off = route_cv.off > cap_cv.off ? route_cv.off : cap_cv.off;
+    if (ffn_cv.off > cv.off)
+        cv.off = ffn_cv.off;
 }
 
 struct ForwardBufs {
@@ -204,19 +211,49 @@ size_t moe_workspace_size(const moe_config *cfg)
     return cv.off;
 }
 
-moe_status moe_route(const moe_config *cfg, const void *x, const float *W_r,
-                     const float *logit_bias, const float *select_bias, int32_t *topk_idx,
-                     float *gates, float *loss_partials, float *logits_out, float *scores_out,
-                     moe_stream_t stream)
+namespace {
+
+moe_status route_impl(const moe_config *cfg, const void *x, const float *W_r,
+                      const float *logit_bias, const float *select_bias, int32_t *topk_idx,
+                      float *gates, float *loss_partials, float *logits_out, float *scores_out,
+                      void *ws, size_t ws_bytes, moe_stream_t stream, bool clear_status)
 {
     moe_status st = check_cfg(cfg);
     if (st != MOE_OK)
         return st;
-    if (cfg->T > 0 && (!x || !W_r || !topk_idx || !gates || !loss_partials))
+    if (cfg->T == 0)
+        return MOE_OK;
+    if (!x || !W_r || !topk_idx || !gates || !loss_partials || !ws)
         return MOE_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return MOE_ERR_ALIGN;
+    if (ws_bytes < stage_scratch_bytes(*cfg))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (clear_status && cudaMemsetAsync(ws, 0, sizeof(int32_t), cs) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const RoutePlan plan = route_plan(*cfg);
+    if (plan.tensor_cores) {
+        if (!aligned16(x))
+            return MOE_ERR_ALIGN;
+        StageScratch s = carve_stage(*cfg, ws);
+        return cuda_status(launch_route_tc(*cfg, x, W_r, logit_bias, select_bias, topk_idx,
+                                           gates, loss_partials, logits_out, scores_out, s.route,
+                                           s.status, cs));
+    }
     return cuda_status(launch_route(*cfg, x, W_r, logit_bias, select_bias, topk_idx, gates,
-                                    loss_partials, logits_out, scores_out,
-                                    reinterpret_cast<cudaStream_t>(stream)));
+                                    loss_partials, logits_out, scores_out, cs));
+}
+
+}  // namespace
+
+moe_status moe_route(const moe_config *cfg, const void *x, const float *W_r,
+                     const float *logit_bias, const float *select_bias, int32_t *topk_idx,
+                     float *gates, float *loss_partials, float *logits_out, float *scores_out,
+                     void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    return route_impl(cfg, x, W_r, logit_bias, select_bias, topk_idx, gates, loss_partials,
+                      logits_out, scores_out, ws, ws_bytes, stream, true);
 }
 
 moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx, int32_t *counts,
@@ -257,10 +294,13 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *top
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
-moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
-                          const void *W1, const void *W3, const void *W2, const void *x,
-                          const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
-                          void *Y_shared, void *ws, size_t ws_bytes, moe_stream_t stream)
+namespace {
+
+moe_status expert_ffn_impl(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                           const void *W1, const void *W3, const void *W2, const void *x,
+                           const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
+                           void *Y_shared, void *ws, size_t ws_bytes, moe_stream_t stream,
+                           bool clear_status)
 {
     moe_status st = check_cfg(cfg);
     if (st != MOE_OK)
@@ -282,8 +322,8 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32
         return MOE_ERR_WORKSPACE;
     StageScratch s = carve_stage(c, ws);
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(s.status, 0, sizeof(int32_t), cs);
-    if (e != cudaSuccess)
+    cudaError_t e;
+    if (clear_status && cudaMemsetAsync(s.status, 0, sizeof(int32_t), cs) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (c.dtype == MOE_DTYPE_BF16)
         e = launch_ffn_tcgen05(c, x_perm, offsets, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
@@ -292,6 +332,17 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32
         e = launch_ffn_simt(c, x_perm, offsets, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm, Y_shared,
                             s.H, s.H_sh, cs);
     return cuda_status(e);
+}
+
+}  // namespace
+
+moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                          const void *W1, const void *W3, const void *W2, const void *x,
+                          const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
+                          void *Y_shared, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    return expert_ffn_impl(cfg, x_perm, offsets, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm, Y_shared,
+                           ws, ws_bytes, stream, true);
 }
 
 moe_status moe_combine(const moe_config *cfg, const void *Y_perm, const void *Y_shared,
@@ -355,16 +406,18 @@ moe_status moe_forward(const moe_config *cfg, const moe_weights *w, const void *
     if (out->counts) f.counts = out->counts;
     if (out->n_dropped) f.n_dropped = out->n_dropped;
     const size_t ssz = stage_scratch_bytes(c);
-    if ((st = moe_route(cfg, x, w->W_r, w->logit_bias, w->select_bias, f.topk, f.gates,
-                        f.partials, nullptr, nullptr, stream)) != MOE_OK)
+    if ((st = moe_clear_device_status(ws, stream)) != MOE_OK)
+        return st;
+    if ((st = route_impl(cfg, x, w->W_r, w->logit_bias, w->select_bias, f.topk, f.gates,
+                         f.partials, nullptr, nullptr, ws, ssz, stream, false)) != MOE_OK)
         return st;
     if ((st = moe_capacity(cfg, f.topk, f.counts, f.pos, f.keep, f.kept, f.offsets, f.dropped,
                            f.n_dropped, ws, ssz, stream)) != MOE_OK)
         return st;
     if ((st = moe_dispatch(cfg, x, f.topk, f.pos, f.keep, f.offsets, f.x_perm, stream)) != MOE_OK)
         return st;
-    if ((st = moe_expert_ffn(cfg, f.x_perm, f.offsets, w->W1, w->W3, w->W2, x, w->Ws1, w->Ws3,
-                             w->Ws2, f.Y_perm, f.Y_sh, ws, ssz, stream)) != MOE_OK)
+    if ((st = expert_ffn_impl(cfg, f.x_perm, f.offsets, w->W1, w->W3, w->W2, x, w->Ws1, w->Ws3,
+                              w->Ws2, f.Y_perm, f.Y_sh, ws, ssz, stream, false)) != MOE_OK)
         return st;
     if ((st = moe_combine(cfg, f.Y_perm, f.Y_sh, f.gates, f.topk, f.pos, f.keep, f.offsets,
                           nullptr, out->y, stream)) != MOE_OK)

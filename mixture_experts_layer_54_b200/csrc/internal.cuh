@@ -29,13 +29,25 @@ int route_blocks(const moe_config &c);   // blocks of the tiled route kernel
 int partial_rows(const moe_config &c);   // rows of the loss partials, ceil(T / 4)
 int cap_blocks(const moe_config &c);
 
-// Scratch carving of the stage workspace.
+// Tensor-core router layout (bf16 layers): experts padded to E_pad, split in
+// chunks of n_chunk per block, K split in k_parts.
+struct RoutePlan {
+    bool tensor_cores;
+    int E_pad, n_chunk, k_parts, kb_per_part;
+};
+RoutePlan route_plan(const moe_config &c);
+size_t route_scratch_bytes(const moe_config &c);
+
+// Scratch carving of the stage workspace: the status word, then one region
+// that the route, capacity and expert-FFN calls share (a call only uses it
+// while it runs, and calls on one stream do not overlap).
 struct StageScratch {
     int32_t *status;      // device status word (timeouts)
+    void *route;          // tensor-core router: split weights and partial logits
     int32_t *hist;        // [cap_blocks][k][E]
     int32_t *base;        // [cap_blocks][k][E]
     void *H;              // [perm_rows][F] dtype
-    void *H_sh;           // [T][S * Fs] dtype
+    void *H_sh;           // [S][T][Fs] dtype
 };
 size_t stage_scratch_bytes(const moe_config &c);
 StageScratch carve_stage(const moe_config &c, void *ws);
@@ -45,6 +57,11 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *W_r,
                          const float *logit_bias, const float *select_bias,
                          int32_t *topk, float *gates, float *partials,
                          float *logits_out, float *scores_out, cudaStream_t s);
+
+cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r,
+                            const float *logit_bias, const float *select_bias, int32_t *topk,
+                            float *gates, float *partials, float *logits_out, float *scores_out,
+                            void *scratch, int32_t *status, cudaStream_t s);
 
 cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep,

@@ -1,0 +1,124 @@
+// Device helpers shared by the two routers (fp32 tiled, bf16 tensor-core).
+#pragma once
+
+#include "internal.cuh"
+
+#include <math.h>
+
+namespace moe {
+
+struct RouteArgs {
+    const void *x;
+    const float *W_r, *logit_bias, *select_bias;
+    int32_t *topk;
+    float *gates, *partials, *logits_out, *scores_out;
+    int T, d, E, k, score, renorm;
+};
+
+// Better of two (key, index) candidates: larger key, then lower index.
+__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib)
+{
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+
+// Softmax / sigmoid, top-k, gates and loss partials of the TB tokens of one
+// batch: lane L holds the logit of (token L / E_T, expert L % E_T).
+template <int E_T>
+__device__ __forceinline__ void small_epilogue(const RouteArgs &a, float z, int t0, int lane,
+                                               bool renorm)
+{
+    constexpr int TB = 32 / E_T;
+    (void)TB;
+    const int E = a.E, T = a.T;
+    const int gl = lane % E_T;
+    const int gbase = lane - gl;
+    const int t = t0 + lane / E_T;
+    const bool tok = t < T;
+    const bool valid = tok && gl < E;
+    if (valid && a.logit_bias)
+        z += a.logit_bias[gl];
+    float m = valid ? z : -INFINITY;
+#pragma unroll
+    for (int o = 1; o < E_T; o <<= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ex = valid ? expf(z - m) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 1; o < E_T; o <<= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float lse = m + logf(sum);
+    float v, key;
+    if (a.score == MOE_SCORE_SOFTMAX) {
+        v = valid ? ex / sum : 0.f;
+        key = valid ? z : -INFINITY;
+    } else {
+        v = valid ? 1.f / (1.f + expf(-z)) : 0.f;
+        key = valid ? v + (a.select_bias ? a.select_bias[gl] : 0.f) : -INFINITY;
+    }
+    float ssum = v;
+#pragma unroll
+    for (int o = 1; o < E_T; o <<= 1)
+        ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+    if (valid && a.logits_out)
+        a.logits_out[(int64_t)t * E + gl] = z;
+    if (valid && a.scores_out)
+        a.scores_out[(int64_t)t * E + gl] = v;
+    // top-k: k rounds of a group argmax over (key, expert), lower index on ties
+    bool taken = false;
+    int sel_idx[kMaxK];
+    float sel_v[kMaxK];
+    float sel_sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        sel_idx[j] = 0;
+        sel_v[j] = 0.f;
+        if (j < a.k) {
+            float bk = (!taken && valid) ? key : -INFINITY;
+            int bi = (!taken && valid) ? gl : 0x7fffffff;
+#pragma unroll
+            for (int o = 1; o < E_T; o <<= 1) {
+                const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (better(ok, oi, bk, bi)) {
+                    bk = ok;
+                    bi = oi;
+                }
+            }
+            const float bv = __shfl_sync(0xffffffffu, v, gbase + (bi < E_T ? bi : 0));
+            if (gl == bi)
+                taken = true;
+            sel_idx[j] = bi;
+            sel_v[j] = bv;
+            sel_sum += bv;
+        }
+    }
+    if (tok && gl == 0) {
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (j < a.k) {
+                a.topk[(int64_t)t * a.k + j] = sel_idx[j];
+                a.gates[(int64_t)t * a.k + j] = renorm ? sel_v[j] / sel_sum : sel_v[j];
+            }
+    }
+    // loss partials: one row per 4 tokens (4 * E_T lanes), tokens in order
+    float pc = valid ? (a.score == MOE_SCORE_SOFTMAX ? v : v / ssum) : 0.f;
+    float zc = (tok && gl == 0) ? lse * lse : 0.f;
+#pragma unroll
+    for (int o = E_T; o < kPartialTokens * E_T; o <<= 1) {
+        pc += __shfl_xor_sync(0xffffffffu, pc, o);
+        zc += __shfl_xor_sync(0xffffffffu, zc, o);
+    }
+    const int row = t0 / kPartialTokens + lane / (kPartialTokens * E_T);
+    const bool row_lane = (lane % (kPartialTokens * E_T)) < E_T;
+    if (row_lane && row * kPartialTokens < T) {
+        float *out = a.partials + (int64_t)row * (E + 1);
+        if (gl < E)
+            out[gl] = pc;
+        if (gl == 0)
+            out[E] = zc;
+    }
+}
+
+
+}  // namespace moe

@@ -90,8 +90,10 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def moe_route(cfg: MoeConfig, x, W_r, logit_bias=None, select_bias=None, want_logits=False,
-              want_scores=False):
+              want_scores=False, ws=None):
     dev = _dev(x)
+    if ws is None:
+        ws = workspace(moe_stage_workspace_size(cfg), dev)
     T, k, E = cfg.T, cfg.k, cfg.E
     topk = torch.empty((T, k), dtype=torch.int32, device=dev)
     gates = torch.empty((T, k), dtype=torch.float32, device=dev)
@@ -100,8 +102,8 @@ def moe_route(cfg: MoeConfig, x, W_r, logit_bias=None, select_bias=None, want_lo
     logits = torch.empty((T, E), dtype=torch.float32, device=dev) if want_logits else None
     scores = torch.empty((T, E), dtype=torch.float32, device=dev) if want_scores else None
     check(lib().moe_route(ctypes.byref(cfg), _p(x), _p(W_r), _p(logit_bias), _p(select_bias),
-                          _p(topk), _p(gates), _p(partials), _p(logits), _p(scores), _stream()),
-          "moe_route")
+                          _p(topk), _p(gates), _p(partials), _p(logits), _p(scores), _p(ws),
+                          ws.numel(), _stream()), "moe_route")
     return topk, gates, partials, logits, scores
 
 
@@ -299,7 +301,8 @@ class StagedForward:
         rec = (lambda i: events[i].record()) if events is not None else (lambda i: None)
         rec(0)
         check(L.moe_route(c, _p(x), _p(W_r), _p(logit_bias), _p(select_bias), _p(self.topk),
-                          _p(self.gates), _p(self.partials), None, None, s), "moe_route")
+                          _p(self.gates), _p(self.partials), None, None, _p(self.ws),
+                          self.ws.numel(), s), "moe_route")
         rec(1)
         check(L.moe_capacity(c, _p(self.topk), _p(self.counts), _p(self.pos), _p(self.keep),
                              _p(self.kept), _p(self.offsets), _p(self.dropped),

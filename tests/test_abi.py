@@ -70,7 +70,7 @@ def test_null_pointers_are_rejected_before_any_launch():
     cfg = moe.moe_config(CONFIGS["tiny"])
     L = moe.lib()
     st = L.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None,
-                     None)
+                     None, 0, None)
     assert st == _abi.MOE_ERR_NULL
     st = L.moe_forward(ctypes.byref(cfg), None, None, None, None, 0, None)
     assert st == _abi.MOE_ERR_NULL
