@@ -190,13 +190,13 @@ def layer_work(shape, counts, kept_total, dropped_tokens):
     ffn_bytes = w_bytes + (N + (T if S else 0)) * d * b * 2 + (N + S * T) * F * b * 2
     routed_tokens = T - dropped_tokens
     return {
-        "route": {"bytes": T * d * b + d * E * 4 + T * k * 8 + math.ceil(T / 4) * (E + 1) * 4,
+        "route": {"bytes": T * d * b + d * E * 4 + T * k * 8 + math.ceil(T / 32) * (E + 1) * 4,
                   "flops": 2.0 * T * d * E},
         "dispatch": {"bytes": routed_tokens * d * b + N * d * b + T * k * 9},
         "expert_ffn": {"flops": ffn_flops, "bytes": ffn_bytes},
         "combine": {"bytes": N * d * b + (T * d * b if S else 0) + T * d * b + T * k * 9},
         "capacity": {"bytes": T * k * 4 * 3 + T * k + T},
-        "losses": {"bytes": math.ceil(T / 4) * (E + 1) * 4 + E * 4},
+        "losses": {"bytes": math.ceil(T / 32) * (E + 1) * 4 + E * 4},
     }
 
 

@@ -22,8 +22,9 @@
 // next.  SwiGLU tiles load 128 rows of W1 and the same 128 rows of W3 into one
 // 256-row B tile: accumulator columns [0,128) hold x W1^T, [128,256) x W3^T.
 //
-// Warps: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..5 = epilogue
-// (warp w reads TMEM lanes 32 (w mod 4) .. +31).  Every wait on an mbarrier is
+// Warps: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..9 = epilogue
+// (warp w reads TMEM lanes 32 (w mod 4) .. +31; warps 2..5 take the first half
+// of the tile's columns, warps 6..9 the second).  Every wait on an mbarrier is
 // bounded by a wall-clock limit; on expiry the CTA records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, every role leaves its loop, the
 // CTA drains what it issued (bounded as well), frees TMEM and returns.
@@ -37,8 +38,8 @@ namespace tc {
 constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
-constexpr int EPI_WARPS = 4;
-constexpr int THREADS = 64 + 32 * EPI_WARPS;         // 192
+constexpr int EPI_WARPS = 8;                          // two per TMEM lane quarter
+constexpr int THREADS = 64 + 32 * EPI_WARPS;         // 320
 constexpr int CHUNK = 32;                            // epilogue columns per step
 constexpr int STG_BYTES = 32 * CHUNK * 2;            // 32 rows x 32 bf16 = 2 KB
 constexpr uint32_t TMEM_COLS = 512;
@@ -46,7 +47,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
 constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_BAR = OFF_STG + EPI_WARPS * 2 * STG_BYTES;
+constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BYTES;
 constexpr int OFF_TILES = OFF_BAR + 256;
 constexpr int SMEM_BYTES = OFF_TILES + 2 * 4 * (kMaxE + 1) + 1024;   // + alignment slack
 
@@ -166,7 +167,7 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -279,9 +280,9 @@ __device__ __forceinline__ void epilogue_chunk(const float *g, const float *u, u
 #pragma unroll
     for (int i = 0; i < CHUNK; i += 2) {
         float a, b;
-        if (EPI == EPI_SWIGLU) {
-            a = g[i] / (1.f + __expf(-g[i])) * u[i];
-            b = g[i + 1] / (1.f + __expf(-g[i + 1])) * u[i + 1];
+        if (EPI == EPI_SWIGLU) {   // silu(g) * u, fast reciprocal (output is bf16)
+            a = __fdividef(g[i], 1.f + __expf(-g[i])) * u[i];
+            b = __fdividef(g[i + 1], 1.f + __expf(-g[i + 1])) * u[i + 1];
         } else if (EPI == EPI_GELU) {
             a = 0.5f * g[i] * (1.f + erff(g[i] * 0.70710678118654752f));
             b = 0.5f * g[i + 1] * (1.f + erff(g[i + 1] * 0.70710678118654752f));
@@ -465,23 +466,23 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             }
         }
     } else {
-        // ================= epilogue (warps 2..5) =================
+        // ================= epilogue (warps 2..9) =================
         const int q = warp & 3;                      // TMEM lane quarter
         const int ew = warp - 2;                     // staging buffer owner
-        const uint32_t stg0 = sStg + ew * 2 * STG_BYTES;
-        uint8_t *stg_ptr0 = smem + OFF_STG + ew * 2 * STG_BYTES;
+        const int half = ew >> 2;                    // which half of the columns
+        const uint32_t stg = sStg + ew * STG_BYTES;
+        uint8_t *stg_ptr = smem + OFF_STG + ew * STG_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
-        int buf = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
             if (!wait_bar(tfull_bar(acc), acc_phase, ctl))
                 break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            const int c_end = min(BN_OUT, p.set[t.set].c_cols - t.c_col);
+            const int c_end = min((half + 1) * (BN_OUT / 2), p.set[t.set].c_cols - t.c_col);
 #pragma unroll 1
-            for (int c = 0; c < c_end; c += CHUNK) {
+            for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
                 float g[CHUNK], u[CHUNK];
                 uint32_t packed[CHUNK / 2];
                 tmem_ld32(tbase + c, g);
@@ -494,9 +495,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                 // staging tile: 32 rows x 64 bytes, 64-byte swizzle (16-byte
                 // chunk index XOR bits 1-2 of the row), as the store map expects
                 if (lane == 0)
-                    bulk_wait_read1();
+                    bulk_wait_read0();
                 __syncwarp();
-                uint8_t *row = stg_ptr0 + buf * STG_BYTES + lane * 64;
+                uint8_t *row = stg_ptr + lane * 64;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
                     const int phys = ch ^ ((lane >> 1) & 3);
@@ -507,11 +508,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&p.tmC[t.set], stg0 + buf * STG_BYTES, t.c_col + c, t.m0 + q * 32,
-                                 t.c_group);
+                    tma_store_3d(&p.tmC[t.set], stg, t.c_col + c, t.m0 + q * 32, t.c_group);
                     bulk_commit();
                 }
-                buf ^= 1;
             }
             // this warp's reads of the accumulator are done
             tc_fence_before();
@@ -557,7 +556,7 @@ constexpr int HALF_BYTES = 128 * BK * 2;             // 16 KB: 128 rows x 64 bf1
 constexpr int OFF2_A = 0;
 constexpr int OFF2_B = OFF2_A + STAGES2 * HALF_BYTES;
 constexpr int OFF2_STG = OFF2_B + STAGES2 * HALF_BYTES;
-constexpr int OFF2_BAR = OFF2_STG + EPI_WARPS * 2 * STG_BYTES;
+constexpr int OFF2_BAR = OFF2_STG + EPI_WARPS * STG_BYTES;
 constexpr int OFF2_TILES = OFF2_BAR + 256;
 constexpr int SMEM2_BYTES = OFF2_TILES + 2 * 4 * (kMaxE + 1) + 1024;
 
@@ -846,14 +845,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
             }
         }
     } else {
-        // ================= epilogue (warps 2..5, both CTAs) =================
+        // ================= epilogue (warps 2..9, both CTAs) =================
         const int q = warp & 3;
         const int ew = warp - 2;
-        const uint32_t stg0 = sStg + ew * 2 * STG_BYTES;
-        uint8_t *stg_ptr0 = smem + OFF2_STG + ew * 2 * STG_BYTES;
+        const int half = ew >> 2;
+        const uint32_t stg = sStg + ew * STG_BYTES;
+        uint8_t *stg_ptr = smem + OFF2_STG + ew * STG_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
-        int buf = 0;
         for (int tile = cluster_id; tile < total; tile += nclusters) {
             const Tile2 t = decode2(p, tstart, mpairs, routed_total, tile);
             if (!wait_bar(tfull_bar(acc), acc_phase, ctl))
@@ -861,10 +860,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const int c_col = t.n_idx * BN_OUT;
-            const int c_end = (rank == 0 || t.second) ? min(BN_OUT, p.set[t.set].c_cols - c_col) : 0;
+            const int c_end = (rank == 0 || t.second)
+                                  ? min((half + 1) * (BN_OUT / 2), p.set[t.set].c_cols - c_col)
+                                  : 0;
             const int row = t.m0 + (int)rank * 128 + q * 32;
 #pragma unroll 1
-            for (int c = 0; c < c_end; c += CHUNK) {
+            for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
                 float g[CHUNK], u[CHUNK];
                 uint32_t packed[CHUNK / 2];
                 tmem_ld32(tbase + c, g);
@@ -875,9 +876,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                     epilogue_chunk<EPI>(g, g, packed);
                 }
                 if (lane == 0)
-                    bulk_wait_read1();
+                    bulk_wait_read0();
                 __syncwarp();
-                uint8_t *rowp = stg_ptr0 + buf * STG_BYTES + lane * 64;
+                uint8_t *rowp = stg_ptr + lane * 64;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
                     const int phys = ch ^ ((lane >> 1) & 3);
@@ -888,10 +889,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&p.tmC[t.set], stg0 + buf * STG_BYTES, c_col + c, row, t.c_group);
+                    tma_store_3d(&p.tmC[t.set], stg, c_col + c, row, t.c_group);
                     bulk_commit();
                 }
-                buf ^= 1;
             }
             tc_fence_before();
             __syncwarp();

@@ -13,7 +13,7 @@ namespace moe {
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 8;
 constexpr int kRouteTokens = 32;   // tokens per block of the tiled route kernel
-constexpr int kPartialTokens = 4;  // tokens per row of the loss partials
+constexpr int kPartialTokens = 32;  // tokens per row of the loss partials
 constexpr int kCapTokens = 256;    // tokens per capacity block
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -26,7 +26,7 @@ moe_status validate(const moe_config &c);
 int64_t capacity_of(const moe_config &c);          // valid config only
 int64_t perm_rows(const moe_config &c);            // valid config only
 int route_blocks(const moe_config &c);   // blocks of the tiled route kernel
-int partial_rows(const moe_config &c);   // rows of the loss partials, ceil(T / 4)
+int partial_rows(const moe_config &c);   // rows of the loss partials, ceil(T / 32)
 int cap_blocks(const moe_config &c);
 
 // Tensor-core router layout (bf16 layers): experts padded to E_pad, split in

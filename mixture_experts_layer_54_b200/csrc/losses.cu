@@ -11,34 +11,29 @@ namespace moe {
 namespace {
 
 constexpr int THREADS = 1024;
+constexpr int WARPS = THREADS / 32;
 
-// Column c of the partials (expert c < E, or the lse^2 column c = E) is
-// summed by ny threads, each over rows y, y + ny, ... in order, then the ny
-// partial sums in order: a fixed reduction tree, so the result does not depend
-// on timing.
+// Column c of the partials (expert c < E, or the lse^2 column c = E) belongs
+// to warp c mod 32; lane l sums rows l, l + 32, ... in order (double), then
+// the 32 lane sums meet by xor shuffles in a fixed pattern: a fixed reduction
+// tree, so the result does not depend on timing.
 __global__ void __launch_bounds__(THREADS)
-losses_kernel(const int32_t *counts, const float *partials, int rows, int T, int k, int E,
-              float *aux, float *zloss)
+losses_kernel(const int32_t *__restrict__ counts, const float *__restrict__ partials, int rows,
+              int T, int k, int E, float *aux, float *zloss)
 {
-    extern __shared__ double part[];   // [ny][C]
     __shared__ double term[kMaxE + 1];
     const int C = E + 1;
-    const int ny = THREADS / C;
-    const int tx = threadIdx.x % C, ty = threadIdx.x / C;
-    if (ty < ny) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int col = warp; col < C; col += WARPS) {
         double s = 0.0;
-        for (int r = ty; r < rows; r += ny)
-            s += (double)partials[(int64_t)r * C + tx];
-        part[ty * C + tx] = s;
-    }
-    __syncthreads();
-    if (threadIdx.x < C) {
-        double s = 0.0;
-        for (int y = 0; y < ny; ++y)
-            s += part[y * C + threadIdx.x];
-        term[threadIdx.x] = threadIdx.x < E
-                                ? ((double)counts[threadIdx.x] / ((double)T * (double)k)) *
-                                      (s / (double)T)
+#pragma unroll 4
+        for (int r = lane; r < rows; r += 32)
+            s += (double)__ldg(partials + (int64_t)r * C + col);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0)
+            term[col] = col < E ? ((double)counts[col] / ((double)T * (double)k)) * (s / (double)T)
                                 : s / (double)T;
     }
     __syncthreads();
@@ -56,10 +51,8 @@ losses_kernel(const int32_t *counts, const float *partials, int rows, int T, int
 cudaError_t launch_losses(const moe_config &c, const int32_t *counts, const float *partials,
                           float *aux, float *zloss, cudaStream_t s)
 {
-    const int C = c.E + 1;
-    const size_t smem = sizeof(double) * (THREADS / C) * C;
-    losses_kernel<<<1, THREADS, smem, s>>>(counts, partials, partial_rows(c),
-                                           c.T > 0 ? c.T : 1, c.k, c.E, aux, zloss);
+    losses_kernel<<<1, THREADS, 0, s>>>(counts, partials, partial_rows(c), c.T > 0 ? c.T : 1,
+                                        c.k, c.E, aux, zloss);
     return cudaGetLastError();
 }
 

@@ -9,38 +9,74 @@
 // Dispatch reads each token row once and writes it to each of its kept
 // destinations, so it moves T*d + N_kept*d elements.  Combine reads the k
 // expert rows of a token, its shared-expert row (and residual) and writes y,
-// summing in fp32 in slot order.  Rows move as 16-byte vectors; a block of 128
-// threads owns one token per iteration of a grid-stride loop.
+// summing in fp32 in slot order.  A warp owns one token at a time (grid-stride
+// over tokens): lanes 0..k-1 look up the slots, then the row moves as 16-byte
+// vectors, four per lane in flight.
 #include "internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;   // 8 warps, one token per warp at a time
+constexpr int WARPS = THREADS / 32;
+constexpr int UNROLL = 4;      // 16-byte vectors in flight per lane
+
+// The kept destinations of token t: lane j < k looks up slot j, then every lane
+// gets the k rows (or -1) by shuffle.
+__device__ __forceinline__ void slot_rows(int t, int k, int E, const int32_t *topk,
+                                          const int32_t *pos, const uint8_t *keep,
+                                          const int32_t *offsets, int lane, int64_t *rows)
+{
+    int64_t mine = -1;
+    if (lane < k) {
+        const int64_t a = (int64_t)t * k + lane;
+        const int e = topk[a];
+        if (keep[a] && e >= 0 && e < E)
+            mine = (int64_t)offsets[e] + pos[a];
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+        rows[j] = __shfl_sync(0xffffffffu, mine, j);
+}
 
 __global__ void __launch_bounds__(THREADS)
-dispatch_vec_kernel(const uint4 *x, int T, int k, int E, int nvec, const int32_t *topk,
-                    const int32_t *pos, const uint8_t *keep, const int32_t *offsets,
-                    uint4 *x_perm)
+dispatch_vec_kernel(const uint4 *__restrict__ x, int T, int k, int E, int nvec,
+                    const int32_t *__restrict__ topk, const int32_t *__restrict__ pos,
+                    const uint8_t *__restrict__ keep, const int32_t *__restrict__ offsets,
+                    uint4 *__restrict__ x_perm)
 {
-    for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        uint4 *dst[kMaxK];
-        int nd = 0;
-        for (int j = 0; j < k; ++j) {
-            int64_t a = (int64_t)t * k + j;
-            const int e = topk[a];
-            if (keep[a] && e >= 0 && e < E) {
-                int64_t row = (int64_t)offsets[e] + pos[a];
-                dst[nd++] = x_perm + row * nvec;
-            }
-        }
-        if (nd == 0)
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
+    for (int t = gw; t < T; t += gridDim.x * WARPS) {
+        int64_t rows[kMaxK];
+        slot_rows(t, k, E, topk, pos, keep, offsets, lane, rows);
+        bool any = false;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            any |= j < k && rows[j] >= 0;
+        if (!any)
             continue;
         const uint4 *src = x + (int64_t)t * nvec;
-        for (int v = threadIdx.x; v < nvec; v += THREADS) {
-            uint4 val = __ldg(src + v);
-            for (int j = 0; j < nd; ++j)
-                __stcs(dst[j] + v, val);
+        for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
+            uint4 val[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec)
+                    val[u] = __ldcs(src + v);
+            }
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j) {
+                if (j >= k || rows[j] < 0)
+                    continue;
+                uint4 *dst = x_perm + rows[j] * nvec;
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec)
+                        __stcs(dst + v, val[u]);
+                }
+            }
         }
     }
 }
@@ -87,60 +123,93 @@ template <> struct Vec<float> {
 
 template <typename Elem>
 __global__ void __launch_bounds__(THREADS)
-combine_vec_kernel(const uint4 *Y_perm, const uint4 *Y_sh, const float *gates,
-                   const int32_t *topk, const int32_t *pos, const uint8_t *keep,
-                   const int32_t *offsets, const uint4 *residual, uint4 *y, int T, int k,
-                   int E, int nvec)
+combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y_sh,
+                   const float *__restrict__ gates, const int32_t *__restrict__ topk,
+                   const int32_t *__restrict__ pos, const uint8_t *__restrict__ keep,
+                   const int32_t *__restrict__ offsets, const uint4 *__restrict__ residual,
+                   uint4 *__restrict__ y, int T, int k, int E, int nvec)
 {
     constexpr int N = Vec<Elem>::N;
-    for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        const uint4 *src[kMaxK];
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
+    for (int t = gw; t < T; t += gridDim.x * WARPS) {
+        int64_t rows[kMaxK];
+        slot_rows(t, k, E, topk, pos, keep, offsets, lane, rows);
+        const float mg = lane < k ? gates[(int64_t)t * k + lane] : 0.f;
         float g[kMaxK];
-        int ns = 0;
-        for (int j = 0; j < k; ++j) {
-            int64_t a = (int64_t)t * k + j;
-            const int e = topk[a];
-            if (keep[a] && e >= 0 && e < E) {
-                int64_t row = (int64_t)offsets[e] + pos[a];
-                src[ns] = Y_perm + row * nvec;
-                g[ns++] = gates[a];
-            }
-        }
-        for (int v = threadIdx.x; v < nvec; v += THREADS) {
-            float acc[N], f[N];
 #pragma unroll
-            for (int i = 0; i < N; ++i)
-                acc[i] = 0.f;
-            for (int j = 0; j < ns; ++j) {
-                Vec<Elem>::load(__ldcs(src[j] + v), f);
+        for (int j = 0; j < kMaxK; ++j)
+            g[j] = __shfl_sync(0xffffffffu, mg, j);
+        for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
+            float acc[UNROLL][N];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u)
 #pragma unroll
                 for (int i = 0; i < N; ++i)
-                    acc[i] = fmaf(g[j], f[i], acc[i]);
-            }
-            if (Y_sh) {
-                Vec<Elem>::load(__ldcs(Y_sh + (int64_t)t * nvec + v), f);
+                    acc[u][i] = 0.f;
+            // slots in order, then the shared experts, then the residual
 #pragma unroll
-                for (int i = 0; i < N; ++i)
-                    acc[i] += f[i];
-            }
-            if (residual) {
-                Vec<Elem>::load(__ldg(residual + (int64_t)t * nvec + v), f);
+            for (int j = 0; j < kMaxK; ++j) {
+                if (j >= k || rows[j] < 0)
+                    continue;
+                const uint4 *src = Y_perm + rows[j] * nvec;
+                uint4 raw[UNROLL];
 #pragma unroll
-                for (int i = 0; i < N; ++i)
-                    acc[i] += f[i];
+                for (int u = 0; u < UNROLL; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec)
+                        raw[u] = __ldcs(src + v);
+                }
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) {
+                    float f[N];
+                    Vec<Elem>::load(raw[u], f);
+#pragma unroll
+                    for (int i = 0; i < N; ++i)
+                        acc[u][i] = fmaf(g[j], f[i], acc[u][i]);
+                }
             }
-            y[(int64_t)t * nvec + v] = Vec<Elem>::store(acc);
+            const uint4 *extra[2] = {Y_sh ? Y_sh + (int64_t)t * nvec : nullptr,
+                                     residual ? residual + (int64_t)t * nvec : nullptr};
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                if (!extra[q])
+                    continue;
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) {
+                        float f[N];
+                        Vec<Elem>::load(__ldcs(extra[q] + v), f);
+#pragma unroll
+                        for (int i = 0; i < N; ++i)
+                            acc[u][i] += f[i];
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec)
+                    y[(int64_t)t * nvec + v] = Vec<Elem>::store(acc[u]);
+            }
         }
     }
 }
 
-int grid_for(int T)
+// As many blocks of 8 token-warps as are resident at once, fewer for small T.
+template <typename K>
+int grid_for(K kernel, int T)
 {
-    int dev = 0, sms = 148;
+    int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int g = sms * 16;
-    return T < g ? T : g;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, THREADS, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int need = (T + WARPS - 1) / WARPS;
+    const int g = sms * per_sm;
+    return need < g ? need : g;
 }
 
 }  // namespace
@@ -152,7 +221,7 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *t
     if (c.T == 0)
         return cudaSuccess;
     const int nvec = (int)((int64_t)c.d * dtype_bytes(c.dtype) / 16);
-    dispatch_vec_kernel<<<grid_for(c.T), THREADS, 0, s>>>(
+    dispatch_vec_kernel<<<grid_for(dispatch_vec_kernel, c.T), THREADS, 0, s>>>(
         static_cast<const uint4 *>(x), c.T, c.k, c.E, nvec, topk, pos, keep, offsets,
         static_cast<uint4 *>(x_perm));
     return cudaGetLastError();
@@ -167,7 +236,7 @@ cudaError_t launch_combine(const moe_config &c, const void *Y_perm, const void *
         return cudaSuccess;
     const int nvec = (int)((int64_t)c.d * dtype_bytes(c.dtype) / 16);
     auto args = [&](auto kern) {
-        kern<<<grid_for(c.T), THREADS, 0, s>>>(
+        kern<<<grid_for(kern, c.T), THREADS, 0, s>>>(
             static_cast<const uint4 *>(Y_perm), static_cast<const uint4 *>(Y_sh), gates, topk,
             pos, keep, offsets, static_cast<const uint4 *>(residual), static_cast<uint4 *>(y),
             c.T, c.k, c.E, nvec);

@@ -12,7 +12,7 @@
 // the block's x rows against W_r, staged through shared memory in chunks of 32
 // columns of d; phase 2 gives each warp whole tokens (the E logits of a token
 // spread over the lanes, max / sum / argmax as warp shuffles); phase 3 sums
-// each expert's probability over every 4 tokens in token order, so the loss
+// each expert's probability over the block's 32 tokens in token order, so the loss
 // partials are deterministic.
 #include "internal.cuh"
 #include "route_common.cuh"
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(THREADS) route_kernel(RouteArgs a)
     }
     __syncthreads();
 
-    // ---- phase 3: sums over each row of 4 tokens, in token order ----
+    // ---- phase 3: sums over the block's row of 32 tokens, in token order ----
     constexpr int G = RT / kPartialTokens;
     const int rows = (T + kPartialTokens - 1) / kPartialTokens;
     for (int i = tid; i < G * (E + 1); i += THREADS) {

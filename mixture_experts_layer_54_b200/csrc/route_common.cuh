@@ -24,12 +24,13 @@ __device__ __forceinline__ bool better(float ka, int ia, float kb, int ib)
 
 // Softmax / sigmoid, top-k, gates and loss partials of the TB tokens of one
 // batch: lane L holds the logit of (token L / E_T, expert L % E_T).
+// On return, lanes 0..E_T-1 hold in *pc the batch's sum of expert lane's
+// probability (sigmoid: s / sum s) and every lane holds in *zc the batch's sum
+// of lse^2, both summed over the tokens in a fixed order.
 template <int E_T>
 __device__ __forceinline__ void small_epilogue(const RouteArgs &a, float z, int t0, int lane,
-                                               bool renorm)
+                                               bool renorm, float *pc_out, float *zc_out)
 {
-    constexpr int TB = 32 / E_T;
-    (void)TB;
     const int E = a.E, T = a.T;
     const int gl = lane % E_T;
     const int gbase = lane - gl;
@@ -101,23 +102,17 @@ __device__ __forceinline__ void small_epilogue(const RouteArgs &a, float z, int 
                 a.gates[(int64_t)t * a.k + j] = renorm ? sel_v[j] / sel_sum : sel_v[j];
             }
     }
-    // loss partials: one row per 4 tokens (4 * E_T lanes), tokens in order
+    // loss sums over the batch's tokens (lanes of the same expert), fixed order
     float pc = valid ? (a.score == MOE_SCORE_SOFTMAX ? v : v / ssum) : 0.f;
     float zc = (tok && gl == 0) ? lse * lse : 0.f;
 #pragma unroll
-    for (int o = E_T; o < kPartialTokens * E_T; o <<= 1) {
+    for (int o = E_T; o < 32; o <<= 1)
         pc += __shfl_xor_sync(0xffffffffu, pc, o);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
         zc += __shfl_xor_sync(0xffffffffu, zc, o);
-    }
-    const int row = t0 / kPartialTokens + lane / (kPartialTokens * E_T);
-    const bool row_lane = (lane % (kPartialTokens * E_T)) < E_T;
-    if (row_lane && row * kPartialTokens < T) {
-        float *out = a.partials + (int64_t)row * (E + 1);
-        if (gl < E)
-            out[gl] = pc;
-        if (gl == 0)
-            out[E] = zc;
-    }
+    *pc_out = pc;
+    *zc_out = zc;
 }
 
 

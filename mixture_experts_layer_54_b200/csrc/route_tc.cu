@@ -19,8 +19,8 @@
 //            [K part][T][E_pad];
 //   select - sums the K parts in order, adds the logit bias, softmax or
 //            sigmoid, top-k by warp argmax, gates, and one loss-partials row per
-//            4 tokens: one warp per token, or for E <= 8 one warp per 4 (or 8)
-//            tokens with E_T lanes each.
+//            block of 32 tokens: one warp per token, or for E <= 8 one warp per
+//            4 (or 8) tokens with E_T lanes each.
 #include "internal.cuh"
 #include "route_common.cuh"
 
@@ -290,14 +290,14 @@ struct SelectArgs {
     int T, E, k, score, renorm;
 };
 
-// 8 warps, each one loss row of 4 consecutive tokens, one token at a time
+// One block = 32 tokens = one row of the loss partials; each of the 8 warps
+// takes 4 consecutive tokens, one token at a time, and the warps' sums meet in
+// shared memory in a fixed order.
 __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
 {
+    constexpr int PER_WARP = kPartialTokens / 8;
+    __shared__ float pw[8][kMaxE + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int row = blockIdx.x * 8 + warp;
-    const int rows = (a.T + kPartialTokens - 1) / kPartialTokens;
-    if (row >= rows)
-        return;
     const int E = a.E;
     const int per_lane = (E + 31) / 32;   // <= 8
     const bool renorm = a.renorm < 0 ? (a.k > 1) : (a.renorm != 0);
@@ -306,8 +306,8 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
     for (int i = 0; i < 8; ++i)
         pacc[i] = 0.f;
     float zacc = 0.f;
-    for (int tt = 0; tt < kPartialTokens; ++tt) {
-        const int t = row * kPartialTokens + tt;
+    for (int tt = 0; tt < PER_WARP; ++tt) {
+        const int t = blockIdx.x * kPartialTokens + warp * PER_WARP + tt;
         if (t >= a.T)
             break;
         float z[8], v[8], key[8];
@@ -413,26 +413,34 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
             if (i < per_lane && lane + 32 * i < E)
                 pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[i] : v[i] / ssum;
     }
-    float *out = a.loss_partials + (int64_t)row * (E + 1);
 #pragma unroll
     for (int i = 0; i < 8; ++i)
         if (i < per_lane && lane + 32 * i < E)
-            out[lane + 32 * i] = pacc[i];
+            pw[warp][lane + 32 * i] = pacc[i];
     if (lane == 0)
-        out[E] = zacc;
+        pw[warp][E] = zacc;
+    __syncthreads();
+    float *out = a.loss_partials + (int64_t)blockIdx.x * (E + 1);
+    for (int e = threadIdx.x; e <= E; e += 256) {
+        float acc = 0.f;
+        for (int w = 0; w < 8; ++w)
+            acc += pw[w][e];
+        out[e] = acc;
+    }
 }
 
 // Small E (<= 8): a warp holds 32 / E_T tokens at once, lane L = (token
-// L / E_T, expert L % E_T), so softmax, top-k and the loss row are segmented
-// shuffles over E_T lanes; one warp = one row of 4 loss-partial tokens.
+// L / E_T, expert L % E_T), so softmax, top-k and the loss sums are segmented
+// shuffles over E_T lanes; E_T warps make one block of 32 tokens, one row of
+// the loss partials.
 template <int E_T>
-__global__ void __launch_bounds__(256) select_small_kernel(SelectArgs s)
+__global__ void __launch_bounds__(32 * E_T) select_small_kernel(SelectArgs s)
 {
     constexpr int TB = 32 / E_T;
+    __shared__ float pw[E_T][E_T];
+    __shared__ float zw[E_T];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int t0 = (blockIdx.x * 8 + warp) * TB;
-    if (t0 >= s.T)
-        return;
+    const int t0 = blockIdx.x * kPartialTokens + warp * TB;
     const int gl = lane % E_T;
     const int t = t0 + lane / E_T;
     float z = -INFINITY;
@@ -444,7 +452,20 @@ __global__ void __launch_bounds__(256) select_small_kernel(SelectArgs s)
     RouteArgs a{nullptr, nullptr, s.logit_bias, s.select_bias, s.topk, s.gates,
                 s.loss_partials, s.logits_out, s.scores_out, s.T, 0, s.E, s.k, s.score, s.renorm};
     const bool renorm = s.renorm < 0 ? (s.k > 1) : (s.renorm != 0);
-    small_epilogue<E_T>(a, z, t0, lane, renorm);
+    float pc, zc;
+    small_epilogue<E_T>(a, z, t0, lane, renorm, &pc, &zc);
+    if (lane < E_T)
+        pw[warp][lane] = pc;
+    if (lane == 0)
+        zw[warp] = zc;
+    __syncthreads();
+    float *out = s.loss_partials + (int64_t)blockIdx.x * (s.E + 1);
+    if (threadIdx.x <= s.E) {
+        float acc = 0.f;
+        for (int w = 0; w < E_T; ++w)
+            acc += threadIdx.x < s.E ? pw[w][threadIdx.x] : zw[w];
+        out[threadIdx.x] = acc;
+    }
 }
 
 // ---------------------------------------------------------------- host
@@ -567,14 +588,13 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
         return err;
     SelectArgs a{plog, r.k_parts, r.E_pad, logit_bias, select_bias, topk, gates, partials,
                  logits_out, scores_out, c.T, c.E, c.k, c.score, c.renorm};
-    if (c.E <= 4) {
-        select_small_kernel<4><<<(unsigned)ceil_div(c.T, 8 * 8), 256, 0, s>>>(a);
-    } else if (c.E <= 8) {
-        select_small_kernel<8><<<(unsigned)ceil_div(c.T, 8 * 4), 256, 0, s>>>(a);
-    } else {
-        const int rows = (int)ceil_div(c.T, kPartialTokens);
-        select_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(a);
-    }
+    const unsigned rows = (unsigned)ceil_div(c.T, kPartialTokens);
+    if (c.E <= 4)
+        select_small_kernel<4><<<rows, 4 * 32, 0, s>>>(a);
+    else if (c.E <= 8)
+        select_small_kernel<8><<<rows, 8 * 32, 0, s>>>(a);
+    else
+        select_kernel<<<rows, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -61,7 +61,7 @@ def test_layer_work_counts_only_algorithmic_flops():
     shared = 2.0 * 3 * ds.n_shared * ds.T * ds.d * ds.d_ff_shared
     assert wd["expert_ffn"]["flops"] == 2.0 * 3 * ds.T * ds.k * ds.d * ds.d_ff + shared
     assert wd["route"]["bytes"] == ds.T * ds.d * 2 + ds.d * ds.E * 4 + ds.T * ds.k * 8 + \
-        math.ceil(ds.T / 4) * (ds.E + 1) * 4
+        math.ceil(ds.T / 32) * (ds.E + 1) * 4
 
 
 def test_clock_summary_flags_throttle_reasons():
