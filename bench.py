@@ -14,8 +14,10 @@ weak and no collective touches the data path; the per-step time is the max
 over ranks.
 
 Rank 0 prints one JSON line.  `value` is device-timed (CUDA events, inputs
-resident in HBM); `e2e` repeats the measurement with the step's input copied
-from pinned host memory and the result read back inside the timed region;
+resident in HBM); `e2e` repeats the measurement through HostStream: every
+step's input is copied in from pinned host memory and its output and losses
+copied back inside the timed region, the copies of neighbouring steps
+overlapping a step's kernels;
 `roofline` covers the dominant stage (the expert FFN: two grouped tcgen05
 GEMMs) from its own CUDA events in the same timed region; `cpu_baseline` times
 the CPU oracle on a bounded sample of the same workload.
@@ -56,7 +58,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture (profiles/gemm_2sm_mixtral.md), valid only for the GEMM source it was taken on.
 GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_54_b200", "csrc", "ffn_tcgen05.cu")
 MEASURED_TRAFFIC = {
-    ("mixtral", "2552d78e7c3833aa21e3be7d002760efa36ebea2f049ef2fced01ea7231f723c"): 5.752e9,
+    ("mixtral", "76528806f495b963bf05080db2666b5375ae3e33383fcce51776a9056bf3eb02"): 6.717e9,
 }
 
 
@@ -73,7 +75,7 @@ def measured_traffic(config: str):
 def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
@@ -349,32 +351,35 @@ def run_ours(args):
     del graph
     ms_per_step = max_over_ranks(total_ms / args.steps, dev)
 
-    # ---- end to end: pinned host input in, result out, inside the timed region ----
-    fwd = moe.MoEForward(cfg, dev, keep_routing=False)
+    # ---- end to end: pinned host input in, result out, inside the timed region.
+    # Batches stream through HostStream (public API): each step copies its x
+    # in and its y and losses out, overlapped with the neighbouring steps'
+    # kernels; the region ends when the last step's outputs are on the host ----
     w = moe.weights_struct(inp.W_r, inp.W1, inp.W2, inp.W3, inp.logit_bias, inp.select_bias,
                            inp.Ws1, inp.Ws3, inp.Ws2)
+    hs = moe.HostStream(cfg, dev, w)
     x_host = inp.x.cpu().pin_memory()
-    y_host = torch.empty(fwd.y.shape, dtype=fwd.y.dtype).pin_memory()
-    loss_host = torch.empty((2,), dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(inp.x)
-    for _ in range(max(args.warmup, 3)):
-        x_dev.copy_(x_host, non_blocking=True)
-        fwd(x_dev, w)
+    y_host = [torch.empty(x_host.shape, dtype=x_host.dtype).pin_memory() for _ in range(2)]
+    loss_host = [torch.empty((2,), dtype=torch.float32).pin_memory() for _ in range(2)]
+    for i in range(max(args.warmup, 3)):
+        hs.submit(x_host, y_host[i % 2], loss_host[i % 2])
+    hs.drain()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dev)
     torch.cuda.synchronize()
     e0.record()
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        fwd(x_dev, w)
-        y_host.copy_(fwd.y, non_blocking=True)
-        loss_host[0:1].copy_(fwd.aux, non_blocking=True)
-        loss_host[1:2].copy_(fwd.zloss, non_blocking=True)
+    hs.start_after(e0)
+    for i in range(args.steps):
+        hs.submit(x_host, y_host[i % 2], loss_host[i % 2])
+    hs.drain()
     e1.record()
     torch.cuda.synchronize()
     barrier(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    if not torch.equal(y_host[(args.steps - 1) % 2], hs.fwd[(args.steps - 1) % 2].y.cpu()):
+        raise SystemExit("e2e: the host copy of y differs from the device result")
+    del hs
 
     if world > 1:
         dist.destroy_process_group()
@@ -397,16 +402,19 @@ def run_ours(args):
         stages[name] = entry
     ffn = work["expert_ffn"]
     ach = ffn["flops"] / (st["expert_ffn"] / 1e3) / 1e12
-    roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
+    # the stage runs inside a step of a long graph replay, under the power cap:
+    # its peak is the sustained matmul figure (the burst one is kept beside it)
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4),
                 "traffic": measured_traffic(args.config),
                 "traffic_unit": "bytes per launch (ncu dram read + write, GEMM1 + GEMM2)",
                 "algorithmic_bytes": ffn["bytes"],
                 "kernel": "moe_expert_ffn: grouped tcgen05 GEMM1 (act fused) + GEMM2",
                 "flops_per_launch": ffn["flops"],
-                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
-                "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4)}
-    t_flop = ffn["flops"] / (peaks["bf16_tflops"] * 1e12)
+                "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
+                "frac_of_burst": round(ach / peaks["bf16_tflops"], 4)}
+    t_flop = ffn["flops"] / (peak * 1e12)
     all_bytes = sum(v.get("bytes", 0) for v in work.values())
     t_byte = all_bytes / (peaks["hbm_gbs"] * 1e9)
     layer_roof = {"t_flop_us": round(t_flop * 1e6, 1), "t_byte_us": round(t_byte * 1e6, 1),
@@ -428,7 +436,8 @@ def run_ours(args):
             "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": kernels_per_step(shape) * args.steps,
-            "timing": "device: one CUDA graph of the K steps; e2e: direct moe_forward calls",
+            "timing": "device: one CUDA graph of the K steps; e2e: HostStream (copies of step "
+                      "i +- 1 overlap step i's kernels)",
             "roofline": roofline, "layer_roofline": layer_roof, "stages": stages,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},

@@ -250,6 +250,64 @@ class MoEForward:
         return self.y
 
 
+class HostStream:
+    """Runs the layer over batches that live in pinned host memory, the way a
+    server feeds it: batch i + 1's copy to the device and batch i - 1's copy
+    back overlap batch i's kernels.  `depth` device slots (input buffer, layer
+    state, output) rotate; copies in run on one side stream, copies out on
+    another, the layer (moe_forward) on the caller's current stream, ordered by
+    events only.  This class orders copies; it computes nothing itself."""
+
+    def __init__(self, cfg: MoeConfig, device, weights: MoeWeights, depth: int = 2):
+        dev = torch.device(device)
+        self.weights = weights
+        self.depth = depth
+        self.fwd = [MoEForward(cfg, dev, keep_routing=False) for _ in range(depth)]
+        self.x_dev = [torch.empty((cfg.T, cfg.d), dtype=_tdtype(cfg), device=dev)
+                      for _ in range(depth)]
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(depth)]
+        self.ev_in, self.ev_done, self.ev_out = ev(), ev(), ev()
+        self.n = 0
+
+    def start_after(self, event):
+        """Make the next copies wait for `event` (e.g. the start of a timed region)."""
+        self.s_in.wait_event(event)
+        self.s_out.wait_event(event)
+
+    def submit(self, x_host, y_host, loss_host=None):
+        """Queue one batch: x_host [T, d] pinned in, y_host [T, d] (and loss_host
+        [2] = aux, z) pinned out.  Returns the event after which the outputs
+        hold this batch's results."""
+        slot = self.n % self.depth
+        comp = torch.cuda.current_stream()
+        fwd = self.fwd[slot]
+        with torch.cuda.stream(self.s_in):
+            self.s_in.wait_event(self.ev_done[slot])     # slot's input no longer read
+            self.x_dev[slot].copy_(x_host, non_blocking=True)
+            self.ev_in[slot].record(self.s_in)
+        comp.wait_event(self.ev_in[slot])
+        comp.wait_event(self.ev_out[slot])                # slot's output already copied out
+        fwd(self.x_dev[slot], self.weights)
+        self.ev_done[slot].record(comp)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.ev_done[slot])
+            y_host.copy_(fwd.y, non_blocking=True)
+            if loss_host is not None:
+                loss_host[0:1].copy_(fwd.aux, non_blocking=True)
+                loss_host[1:2].copy_(fwd.zloss, non_blocking=True)
+            self.ev_out[slot].record(self.s_out)
+        self.n += 1
+        return self.ev_out[slot]
+
+    def drain(self):
+        """Make the current stream wait until every queued batch is copied out."""
+        comp = torch.cuda.current_stream()
+        for e in self.ev_out:
+            comp.wait_event(e)
+
+
 def moe_forward(cfg: MoeConfig, x, W_r, W1, W2, W3=None, logit_bias=None, select_bias=None,
                 Ws1=None, Ws3=None, Ws2=None):
     """One-shot forward: returns (y, aux, zloss, MoEForward state with routing)."""
@@ -264,7 +322,7 @@ __all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
            "moe_loss_partials_count", "moe_stage_workspace_size", "moe_workspace_size",
            "workspace", "moe_route", "moe_capacity", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_losses", "moe_device_status", "weights_struct", "MoEForward",
-           "moe_forward", "CapacityOut", "StagedForward"]
+           "HostStream", "moe_forward", "CapacityOut", "StagedForward"]
 
 
 class StagedForward:
