@@ -61,8 +61,13 @@ def _load():
         lib.oracle_ffn_tokens.argtypes = [I, I, I, I, I, I, I, I, P, I, P, P, P,
                                           P, P, P, P, P, P, I, P, I, P]
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_capacity_walk_scored.argtypes = [I, I, I, ctypes.c_int64, P, P, P, P, P, P,
+                                                    P]
+        lib.oracle_seq_losses.argtypes = [I, I, I, I, I, P, P, P, P]
+        lib.oracle_bias_update.argtypes = [I, I, I, P, ctypes.c_float, P, P]
         for f in (lib.oracle_route, lib.oracle_capacity_value, lib.oracle_capacity,
-                  lib.oracle_capacity_walk,
+                  lib.oracle_capacity_walk, lib.oracle_capacity_walk_scored,
+                  lib.oracle_seq_losses, lib.oracle_bias_update,
                   lib.oracle_losses, lib.oracle_ffn_tokens, lib.oracle_num_threads):
             f.restype = ctypes.c_int
         _lib = lib
@@ -148,13 +153,16 @@ class Capacity:
 
 
 def capacity_walk(topk, E: int, cf: float | None = None, priority: int = 0,
-                  C: int | None = None) -> Capacity:
+                  C: int | None = None, sel_scores=None) -> Capacity:
     """Priority-order walk with one counter per expert ("Lab 18" section 3).
 
     C comes from the capacity factor cf, or is given directly as the pages'
     capacity_mask takes it.
     priority 0 = token order, first come first served ("Lab 01" step 4);
-    priority 1 = rank-major (GShard, "Lab 18" section 3).
+    priority 1 = rank-major (GShard, "Lab 18" section 3);
+    priority 2 = batch-prioritized (V-MoE, "Lab 18" section 3): highest router
+                 score first, ties in token then slot order; sel_scores [T, k]
+                 are the scores of the selected experts, taken as fp32.
     """
     topk = np.ascontiguousarray(topk, dtype=np.int32)
     T, k = topk.shape
@@ -165,9 +173,25 @@ def capacity_walk(topk, E: int, cf: float | None = None, priority: int = 0,
     pos = np.empty((T, k), np.int32)
     keep = np.empty((T, k), np.uint8)
     dropped = np.empty((T,), np.uint8)
-    _check(_load().oracle_capacity_walk(T, E, k, int(C), priority, _ptr(topk), _ptr(counts),
-                                        _ptr(pos), _ptr(keep), _ptr(dropped), ctypes.byref(nd)))
+    if priority == 2:
+        sel = np.ascontiguousarray(sel_scores, dtype=np.float32)
+        assert sel.shape == (T, k)
+        _check(_load().oracle_capacity_walk_scored(T, E, k, int(C), _ptr(topk), _ptr(sel),
+                                                   _ptr(counts), _ptr(pos), _ptr(keep),
+                                                   _ptr(dropped), ctypes.byref(nd)))
+    else:
+        _check(_load().oracle_capacity_walk(T, E, k, int(C), priority, _ptr(topk),
+                                            _ptr(counts), _ptr(pos), _ptr(keep), _ptr(dropped),
+                                            ctypes.byref(nd)))
     return Capacity(int(C), counts, pos, keep, dropped, int(nd.value))
+
+
+def selected_scores(scores, topk) -> np.ndarray:
+    """The router score of each selected expert, [T, k], rounded to fp32 (the
+    precision the batch-prioritized ranking is taken in)."""
+    scores = np.asarray(scores)
+    topk = np.asarray(topk)
+    return np.take_along_axis(scores, topk.astype(np.int64), axis=1).astype(np.float32)
 
 
 # --------------------------------------------------------------------------- losses
@@ -183,6 +207,37 @@ def losses(scores, counts, lse, k: int, score: int = 0):
     _check(_load().oracle_losses(T, E, k, score, _ptr(scores), _ptr(counts), _ptr(lse),
                                  ctypes.byref(aux), ctypes.byref(zl)))
     return float(aux.value), float(zl.value)
+
+
+def seq_losses(scores, topk, k: int, L: int, score: int = 0):
+    """Sequence-wise balance loss: the Switch loss per sequence of L tokens,
+    averaged over the T / L sequences (the balancing unit variant of the cs336
+    lecture 4 field map, "Training a router you cannot differentiate").
+    Returns (mean, per_sequence values)."""
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    T, E = scores.shape
+    topk = np.ascontiguousarray(topk, dtype=np.int32)
+    assert topk.shape == (T, k)
+    if L < 1 or T % L:
+        raise OracleError("bad shape")
+    mean = ctypes.c_double()
+    per = np.empty((T // L,), np.float64)
+    _check(_load().oracle_seq_losses(T, E, k, score, L, _ptr(scores), _ptr(topk),
+                                     ctypes.byref(mean), _ptr(per)))
+    return float(mean.value), per
+
+
+def bias_update(counts, T: int, k: int, gamma: float, bias) -> np.ndarray:
+    """DeepSeek-V3 auxiliary-loss-free balancing step ("Lab 18" section 2):
+    the selection bias of an overloaded expert moves down by gamma, of an
+    underloaded one up by gamma, in fp32."""
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    E = counts.shape[0]
+    bias = np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty((E,), np.float32)
+    _check(_load().oracle_bias_update(T, E, k, _ptr(counts), ctypes.c_float(gamma), _ptr(bias),
+                                      _ptr(out)))
+    return out
 
 
 # ------------------------------------------------------------------------------ FFN
@@ -246,7 +301,8 @@ def forward(x, W_r, W1, W3, W2, *, k: int, act: int, cf: float, score: int = 0,
     """MoE.forward of "Lab 18" ("What to implement" row 5), returning y (not x + y)."""
     r = route(x, W_r, k, score, renorm, logit_bias, select_bias)
     E = np.asarray(W_r).shape[1]
-    cap = capacity_walk(r.topk, E, cf, priority, C=capacity_override)
+    sel = selected_scores(r.scores, r.topk) if priority == 2 else None
+    cap = capacity_walk(r.topk, E, cf, priority, C=capacity_override, sel_scores=sel)
     aux, zl = losses(r.scores, cap.counts, r.lse, k, score)
     if tokens is None:
         tokens = np.arange(np.asarray(x).shape[0], dtype=np.int32)

@@ -227,6 +227,71 @@ int oracle_capacity(int T, int E, int k, double cf, int priority,
                                 dropped, n_dropped_assignments);
 }
 
+/*
+ * Batch-prioritized capacity ([Lab18 sec. 3]: V-MoE ranks the assignments by
+ * router score).  The T*k assignments are walked from the highest router
+ * score down, equal scores in token order and then slot order, with the same
+ * per-expert counters as above.  sel_scores[t*k + j] is the router's score of
+ * the expert chosen in slot j (softmax probability p, or sigmoid affinity s
+ * without the selection bias), given in fp32: the ranking is a decision and
+ * is taken in the precision the scores are stored in.
+ */
+struct scored_assignment {
+    float score;
+    int64_t a;
+};
+
+static int by_score_then_index(const void *l, const void *r)
+{
+    const struct scored_assignment *x = l, *y = r;
+    if (x->score != y->score)
+        return x->score > y->score ? -1 : 1;
+    return x->a < y->a ? -1 : (x->a > y->a ? 1 : 0);
+}
+
+int oracle_capacity_walk_scored(int T, int E, int k, int64_t C, const int32_t *topk,
+                                const float *sel_scores, int32_t *counts, int32_t *pos,
+                                uint8_t *keep, uint8_t *dropped,
+                                int64_t *n_dropped_assignments)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E || C < 0)
+        return OR_ERR_SHAPE;
+    int64_t A = (int64_t)T * k;
+    struct scored_assignment *order = malloc(sizeof *order * (A > 0 ? A : 1));
+    if (!order)
+        return OR_ERR_SHAPE;
+    for (int64_t a = 0; a < A; ++a) {
+        if (topk[a] < 0 || topk[a] >= E || sel_scores[a] != sel_scores[a]) {
+            free(order);
+            return OR_ERR_SHAPE;
+        }
+        order[a].score = sel_scores[a];
+        order[a].a = a;
+    }
+    qsort(order, (size_t)A, sizeof *order, by_score_then_index);
+    for (int e = 0; e < E; ++e)
+        counts[e] = 0;
+    for (int64_t n = 0; n < A; ++n) {
+        int64_t a = order[n].a;
+        int e = topk[a];
+        pos[a] = counts[e]++;
+        keep[a] = (uint8_t)(pos[a] < C);
+    }
+    free(order);
+    int64_t nd = 0;
+    for (int t = 0; t < T; ++t) {
+        int any = 0;
+        for (int j = 0; j < k; ++j) {
+            any |= keep[(int64_t)t * k + j];
+            nd += !keep[(int64_t)t * k + j];
+        }
+        dropped[t] = (uint8_t)!any;
+    }
+    if (n_dropped_assignments)
+        *n_dropped_assignments = nd;
+    return OR_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Balancing losses.                                                         */
 /* ------------------------------------------------------------------------ */
@@ -268,6 +333,84 @@ int oracle_losses(int T, int E, int k, int score, const double *scores,
     for (int t = 0; t < T; ++t)
         zs += lse[t] * lse[t];
     *zloss = zs / (double)T;
+    return OR_OK;
+}
+
+/*
+ * Sequence-wise balance loss: the loss above with one sequence as the
+ * balancing unit ([Lec4] "Training a router you cannot differentiate": the
+ * balancing unit is where the variants differ; DeepSeek-V3 keeps a small
+ * sequence-wise loss beside its bias-based balancing, [Lab18 sec. 2]).
+ * Tokens [b L, (b + 1) L) form sequence b; its f_i counts the assignments its
+ * tokens sent to expert i (before capacity) over its L k slots and its P_i
+ * averages its tokens' probabilities.  mean = average over the T / L
+ * sequences; per_seq[b] (optional) = each sequence's value.
+ */
+int oracle_seq_losses(int T, int E, int k, int score, int L, const double *scores,
+                      const int32_t *topk, double *mean, double *per_seq)
+{
+    if (T < 1 || E < 1 || k < 1 || k > E || L < 1 || T % L != 0)
+        return OR_ERR_SHAPE;
+    int B = T / L;
+    int32_t *counts = malloc(sizeof(int32_t) * E);
+    double *lse = calloc((size_t)L, sizeof(double));   /* z-loss part unused here */
+    if (!counts || !lse) {
+        free(counts);
+        free(lse);
+        return OR_ERR_SHAPE;
+    }
+    double total = 0.0;
+    int st = OR_OK;
+    for (int b = 0; b < B && st == OR_OK; ++b) {
+        for (int e = 0; e < E; ++e)
+            counts[e] = 0;
+        for (int64_t a = (int64_t)b * L * k; a < (int64_t)(b + 1) * L * k; ++a) {
+            if (topk[a] < 0 || topk[a] >= E) {
+                st = OR_ERR_SHAPE;
+                break;
+            }
+            counts[topk[a]]++;
+        }
+        if (st != OR_OK)
+            break;
+        double aux, zl;
+        st = oracle_losses(L, E, k, score, scores + (int64_t)b * L * E, counts, lse, &aux, &zl);
+        if (per_seq)
+            per_seq[b] = aux;
+        total += aux;
+    }
+    free(counts);
+    free(lse);
+    if (st == OR_OK)
+        *mean = total / (double)B;
+    return st;
+}
+
+/*
+ * Auxiliary-loss-free balancing ([Lab18 sec. 2], DeepSeek-V3; [Lec4] "Training
+ * a router you cannot differentiate"): after a step each expert's selection
+ * bias moves by a fixed step gamma against its load, down for an overloaded
+ * expert and up for an underloaded one, unchanged at exactly the balanced
+ * load.  Load = counts_i, the assignments routed to expert i before capacity;
+ * the balanced load T k / E is compared exactly, as E counts_i against T k.
+ * The bias is an fp32 vector and each step is one fp32 addition.
+ */
+int oracle_bias_update(int T, int E, int k, const int32_t *counts, float gamma,
+                       const float *bias_in, float *bias_out)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E)
+        return OR_ERR_SHAPE;
+    int64_t balanced = (int64_t)T * k;
+    for (int i = 0; i < E; ++i) {
+        int64_t load = (int64_t)E * counts[i];
+        float b = bias_in[i];
+        float nb = b;
+        if (load > balanced)
+            nb = b - gamma;
+        else if (load < balanced)
+            nb = b + gamma;
+        bias_out[i] = nb;
+    }
     return OR_OK;
 }
 
