@@ -243,6 +243,52 @@ def size_oracle_sample(shape, h, seconds):
     return int(max(4, min(shape.T, seconds / per)))
 
 
+def graph_time_us(fn, n=20):
+    """Device time of one call of fn: n calls captured in a CUDA graph,
+    replayed once between CUDA events (after three eager warm-up calls)."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        for _ in range(n):
+            fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / n
+
+
+def next_rows(moe, shape, inp, staged, seq_len):
+    """Device times of the rows past the forward, on the same batch: the
+    batch-prioritized capacity (from the router's scores), the sequence-wise
+    balance loss and one loss-free bias step."""
+    import dataclasses
+    cfg2 = moe.moe_config(dataclasses.replace(shape, priority=2))
+    cfg = moe.moe_config(shape)
+    _, _, _, _, scores = moe.moe_route(cfg, inp.x, inp.W_r, inp.logit_bias, inp.select_bias,
+                                       want_scores=True)
+    ws2 = moe.workspace(moe.moe_stage_workspace_size(cfg2), inp.x.device)
+    cap = moe.moe_capacity_scored(cfg2, staged.topk, scores, ws=ws2)
+    t_cap = graph_time_us(lambda: moe.moe_capacity_scored(cfg2, staged.topk, scores, ws=ws2))
+    loss, per = moe.moe_seq_balance_loss(cfg, seq_len, staged.topk, staged.partials)
+    t_seq = graph_time_us(lambda: moe.moe_seq_balance_loss(cfg, seq_len, staged.topk,
+                                                           staged.partials, per, loss))
+    bias = torch.zeros(shape.E, dtype=torch.float32, device=inp.x.device)
+    t_bias = graph_time_us(lambda: moe.moe_bias_update(cfg, staged.counts, 1e-3, bias))
+    torch.cuda.synchronize()
+    return {"capacity_scored": {"us": round(t_cap, 2), "launches": 6,
+                                "n_dropped": int(cap.n_dropped.item())},
+            "seq_balance_loss": {"us": round(t_seq, 2), "seq_len": seq_len, "launches": 2,
+                                 "value": round(float(loss.item()), 6)},
+            "bias_update": {"us": round(t_bias, 2), "launches": 1}}
+
+
 def cpu_baseline(shape, inp, seconds):
     import oracle
     h = oracle_inputs(inp)
@@ -381,6 +427,8 @@ def run_ours(args):
         raise SystemExit("e2e: the host copy of y differs from the device result")
     del hs
 
+    extra = next_rows(moe, shape, inp, staged, seq_len=min(shape.T, 1024)) \
+        if shape.T % 32 == 0 and shape.T > 0 else None
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -441,7 +489,8 @@ def run_ours(args):
             "roofline": roofline, "layer_roofline": layer_roof, "stages": stages,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
-            "device_status": status}
+            "device_status": status,
+            "next_rows": extra}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(shape, inp, args.cpu_seconds)
     print(json.dumps(line), flush=True)

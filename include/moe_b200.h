@@ -50,7 +50,7 @@ typedef enum moe_status {
 enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 };
 enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
-enum { MOE_PRIORITY_TOKEN = 0, MOE_PRIORITY_RANK = 1 };
+enum { MOE_PRIORITY_TOKEN = 0, MOE_PRIORITY_RANK = 1, MOE_PRIORITY_SCORE = 2 };
 
 /* Every expert's segment of the permuted row buffers starts on a multiple of
  * this many rows (the expert GEMM's M tile). */
@@ -68,8 +68,10 @@ enum { MOE_PRIORITY_TOKEN = 0, MOE_PRIORITY_RANK = 1 };
  *            1: renormalized.
  *   dtype    MOE_DTYPE_F32 or MOE_DTYPE_BF16 for x, y and all expert weights.
  *   priority order in which assignments claim expert slots: token order, first
- *            come first served ("Lab 01", where to start step 4), or rank-major
- *            (every first choice before any second, "Lab 18" section 3).
+ *            come first served ("Lab 01", where to start step 4), rank-major
+ *            (every first choice before any second, "Lab 18" section 3), or
+ *            MOE_PRIORITY_SCORE, batch-prioritized: highest router score first
+ *            (V-MoE, "Lab 18" section 3; see moe_capacity_scored).
  *   capacity_factor  C = ceil(capacity_factor * T * k / E) slots per expert
  *            ("Lab 18" section 3); +infinity = no limit.  Must be >= 1.0.
  * Limits: 1 <= k <= min(E, 8), E <= 256.  bf16 needs d, d_ff, d_ff_shared
@@ -196,13 +198,36 @@ moe_status moe_route(const moe_config *cfg, const void *x, const float *W_r,
  *   dropped [T] uint8 out: 1 when every slot of the token was dropped.
  *   n_dropped [1] int32 out: number of dropped assignments.
  *   ws: scratch of at least moe_stage_workspace_size bytes, 256-byte aligned.
- * Returns MOE_ERR_CAPACITY_FACTOR for capacity_factor < 1 ("Lab 01" traps).
+ * Returns MOE_ERR_CAPACITY_FACTOR for capacity_factor < 1 ("Lab 01" traps),
+ * MOE_ERR_DTYPE for MOE_PRIORITY_SCORE (that order needs the router scores:
+ * moe_capacity_scored).
  */
 moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx,
                         int32_t *counts, int32_t *pos, uint8_t *keep,
                         int32_t *kept, int32_t *offsets, uint8_t *dropped,
                         int32_t *n_dropped, void *ws, size_t ws_bytes,
                         moe_stream_t stream);
+
+/*
+ * moe_capacity_scored - moe_capacity in batch-prioritized order ("Lab 18"
+ * section 3: V-MoE ranks the assignments by router score).  The walk takes the
+ * T*k assignments from the highest router score of the selected expert down;
+ * equal scores go in token order, then slot order.  cfg->priority must be
+ * MOE_PRIORITY_SCORE (else MOE_ERR_DTYPE).
+ *   scores [T, E] fp32 in: the router scores, as moe_route writes them to
+ *     scores_out (softmax p, or sigmoid s without the selection bias); the
+ *     score of assignment (t, j) is scores[t, topk_idx[t, j]], compared as
+ *     fp32 (-0 equals +0; NaN scores give an unspecified order).
+ *   Every other argument as for moe_capacity; counts, kept, offsets and
+ *   n_dropped do not depend on the order.
+ *   ws: moe_stage_workspace_size bytes of a config with this priority (it
+ *     holds 8 T k bytes of sort keys).
+ */
+moe_status moe_capacity_scored(const moe_config *cfg, const int32_t *topk_idx,
+                               const float *scores, int32_t *counts, int32_t *pos,
+                               uint8_t *keep, int32_t *kept, int32_t *offsets,
+                               uint8_t *dropped, int32_t *n_dropped, void *ws,
+                               size_t ws_bytes, moe_stream_t stream);
 
 /*
  * moe_capacity_noalloc - moe_capacity with its scratch inside the library.
@@ -292,11 +317,44 @@ moe_status moe_losses(const moe_config *cfg, const int32_t *counts,
                       moe_stream_t stream);
 
 /*
+ * moe_seq_balance_loss - sequence-wise balance loss: the Switch loss of
+ * moe_losses with one sequence as the balancing unit (cs336 lecture 4 field
+ * map, "Training a router you cannot differentiate": the balancing unit is
+ * where the variants differ; DeepSeek-V3 keeps a small sequence-wise loss,
+ * "Lab 18" section 2).  Tokens [b L, (b + 1) L) form sequence b:
+ *   per_seq[b] = E * sum_i (count_i^b / (L k)) * P_i^b,
+ *   count_i^b = assignments of sequence b to expert i (before capacity),
+ *   P_i^b = (1/L) sum_{t in b} p_{t,i} (sigmoid: s_{t,i} / sum_j s_{t,j}),
+ *   loss = (1/B) sum_b per_seq[b], B = T / L.
+ *   seq_len L: a multiple of 32 that divides T (else MOE_ERR_SHAPE).
+ *   topk_idx [T, k] and loss_partials (moe_route) in; per_seq [T / L] fp32
+ *   and loss [1] fp32 out (device).  Fixed summation order (deterministic).
+ */
+moe_status moe_seq_balance_loss(const moe_config *cfg, int32_t seq_len,
+                                const int32_t *topk_idx, const float *loss_partials,
+                                float *per_seq, float *loss, moe_stream_t stream);
+
+/*
+ * moe_bias_update - one step of auxiliary-loss-free balancing ("Lab 18"
+ * section 2, DeepSeek-V3; cs336 lecture 4, "Training a router you cannot
+ * differentiate"): in place, select_bias[i] -= gamma when expert i is
+ * overloaded (E counts[i] > T k), += gamma when underloaded (E counts[i] <
+ * T k), unchanged at the balanced load; one fp32 addition each.
+ *   counts [E] int32 in (moe_capacity: assignments before capacity);
+ *   gamma: finite step (else MOE_ERR_SHAPE); select_bias [E] fp32 in/out,
+ *   the bias moe_route adds to the sigmoid scores for selection only.
+ */
+moe_status moe_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,
+                           float *select_bias, moe_stream_t stream);
+
+/*
  * moe_forward - the whole layer: route, capacity, dispatch, expert FFNs,
  * combine, losses ("Lab 18", MoE.forward row of "What to implement").
  *   x [T, d] dtype; weights; outputs as described at moe_outputs.
  *   ws: at least moe_workspace_size(cfg) bytes, 256-byte aligned.
  * Six kernel stages, no host synchronisation, safe to capture in a CUDA graph.
+ * With MOE_PRIORITY_SCORE the router also writes its scores [T, E] to the
+ * workspace and the capacity stage is moe_capacity_scored.
  */
 moe_status moe_forward(const moe_config *cfg, const moe_weights *w,
                        const void *x, const moe_outputs *out, void *ws,

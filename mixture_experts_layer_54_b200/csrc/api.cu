@@ -17,7 +17,8 @@ moe_status validate(const moe_config &c)
     if ((c.act != MOE_ACT_GELU && c.act != MOE_ACT_SWIGLU) ||
         (c.score != MOE_SCORE_SOFTMAX && c.score != MOE_SCORE_SIGMOID) ||
         (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16) ||
-        (c.priority != MOE_PRIORITY_TOKEN && c.priority != MOE_PRIORITY_RANK) || c.renorm < -1 ||
+        (c.priority != MOE_PRIORITY_TOKEN && c.priority != MOE_PRIORITY_RANK &&
+         c.priority != MOE_PRIORITY_SCORE) || c.renorm < -1 ||
         c.renorm > 1)
         return MOE_ERR_DTYPE;
     if (!(c.capacity_factor >= 1.0))   // also rejects NaN
@@ -82,6 +83,8 @@ void carve_stage_into(const moe_config &c, Carver &cv, StageScratch &s)
     s.route = route_cv.take(route_scratch_bytes(c));
     s.hist = static_cast<int32_t *>(cap_cv.take(hk));
     s.base = static_cast<int32_t *>(cap_cv.take(hk));
+    s.keys = static_cast<unsigned long long *>(
+        cap_cv.take(c.priority == MOE_PRIORITY_SCORE ? (size_t)c.T * c.k * 8 : 0));
     s.H = ffn_cv.take((size_t)R * c.d_ff * esz);
     s.H_sh = ffn_cv.take((size_t)c.n_shared * c.T * (c.n_shared ? c.d_ff_shared : 0) * esz);
     cv.off = route_cv.off > cap_cv.off ? route_cv.off : cap_cv.off;
@@ -91,7 +94,7 @@ void carve_stage_into(const moe_config &c, Carver &cv, StageScratch &s)
 
 struct ForwardBufs {
     int32_t *topk, *counts, *kept, *offsets, *n_dropped, *pos;
-    float *gates, *partials;
+    float *gates, *partials, *scores;
     uint8_t *keep, *dropped;
     void *x_perm, *Y_perm, *Y_sh;
 };
@@ -104,6 +107,9 @@ void carve_forward_into(const moe_config &c, Carver &cv, ForwardBufs &f)
     f.topk = static_cast<int32_t *>(cv.take(A * 4));
     f.gates = static_cast<float *>(cv.take(A * 4));
     f.partials = static_cast<float *>(cv.take((size_t)partial_rows(c) * (c.E + 1) * 4));
+    // router scores [T, E], kept only for the batch-prioritized capacity order
+    f.scores = static_cast<float *>(
+        cv.take(c.priority == MOE_PRIORITY_SCORE ? (size_t)c.T * c.E * 4 : 0));
     f.counts = static_cast<int32_t *>(cv.take((size_t)c.E * 4));
     f.kept = static_cast<int32_t *>(cv.take((size_t)c.E * 4));
     f.offsets = static_cast<int32_t *>(cv.take((size_t)(c.E + 1) * 4));
@@ -264,6 +270,8 @@ moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx, int32_t 
     moe_status st = check_cfg(cfg);
     if (st != MOE_OK)
         return st;
+    if (cfg->priority == MOE_PRIORITY_SCORE)
+        return MOE_ERR_DTYPE;   // the score order needs the scores: moe_capacity_scored
     if (!counts || !kept || !offsets || !n_dropped || !ws ||
         (cfg->T > 0 && (!topk_idx || !pos || !keep || !dropped)))
         return MOE_ERR_NULL;
@@ -275,6 +283,30 @@ moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx, int32_t 
     return cuda_status(launch_capacity(*cfg, capacity_of(*cfg), topk_idx, counts, pos, keep, kept,
                                        offsets, dropped, n_dropped, s.hist, s.base,
                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_capacity_scored(const moe_config *cfg, const int32_t *topk_idx,
+                               const float *scores, int32_t *counts, int32_t *pos, uint8_t *keep,
+                               int32_t *kept, int32_t *offsets, uint8_t *dropped,
+                               int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = check_cfg(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (cfg->priority != MOE_PRIORITY_SCORE)
+        return MOE_ERR_DTYPE;
+    if (!counts || !kept || !offsets || !n_dropped || !ws ||
+        (cfg->T > 0 && (!topk_idx || !scores || !pos || !keep || !dropped)))
+        return MOE_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return MOE_ERR_ALIGN;
+    if (ws_bytes < stage_scratch_bytes(*cfg))
+        return MOE_ERR_WORKSPACE;
+    StageScratch s = carve_stage(*cfg, ws);
+    return cuda_status(launch_capacity_scored(*cfg, capacity_of(*cfg), topk_idx, scores, counts,
+                                              pos, keep, kept, offsets, dropped, n_dropped,
+                                              s.hist, s.base, s.keys,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_idx,
@@ -379,6 +411,35 @@ moe_status moe_losses(const moe_config *cfg, const int32_t *counts, const float 
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_seq_balance_loss(const moe_config *cfg, int32_t seq_len, const int32_t *topk_idx,
+                                const float *loss_partials, float *per_seq, float *loss,
+                                moe_stream_t stream)
+{
+    moe_status st = check_cfg(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (seq_len < kPartialTokens || seq_len % kPartialTokens || cfg->T < 1 || cfg->T % seq_len)
+        return MOE_ERR_SHAPE;
+    if (!topk_idx || !loss_partials || !per_seq || !loss)
+        return MOE_ERR_NULL;
+    return cuda_status(launch_seq_loss(*cfg, seq_len, topk_idx, loss_partials, per_seq, loss,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,
+                           float *select_bias, moe_stream_t stream)
+{
+    moe_status st = check_cfg(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (!isfinite(gamma))
+        return MOE_ERR_SHAPE;
+    if (!counts || !select_bias)
+        return MOE_ERR_NULL;
+    return cuda_status(launch_bias_update(*cfg, counts, gamma, select_bias,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_forward(const moe_config *cfg, const moe_weights *w, const void *x,
                        const moe_outputs *out, void *ws, size_t ws_bytes, moe_stream_t stream)
 {
@@ -408,11 +469,16 @@ moe_status moe_forward(const moe_config *cfg, const moe_weights *w, const void *
     const size_t ssz = stage_scratch_bytes(c);
     if ((st = moe_clear_device_status(ws, stream)) != MOE_OK)
         return st;
+    const bool scored = c.priority == MOE_PRIORITY_SCORE;
     if ((st = route_impl(cfg, x, w->W_r, w->logit_bias, w->select_bias, f.topk, f.gates,
-                         f.partials, nullptr, nullptr, ws, ssz, stream, false)) != MOE_OK)
+                         f.partials, nullptr, scored ? f.scores : nullptr, ws, ssz, stream,
+                         false)) != MOE_OK)
         return st;
-    if ((st = moe_capacity(cfg, f.topk, f.counts, f.pos, f.keep, f.kept, f.offsets, f.dropped,
-                           f.n_dropped, ws, ssz, stream)) != MOE_OK)
+    st = scored ? moe_capacity_scored(cfg, f.topk, f.scores, f.counts, f.pos, f.keep, f.kept,
+                                      f.offsets, f.dropped, f.n_dropped, ws, ssz, stream)
+                : moe_capacity(cfg, f.topk, f.counts, f.pos, f.keep, f.kept, f.offsets, f.dropped,
+                               f.n_dropped, ws, ssz, stream);
+    if (st != MOE_OK)
         return st;
     if ((st = moe_dispatch(cfg, x, f.topk, f.pos, f.keep, f.offsets, f.x_perm, stream)) != MOE_OK)
         return st;

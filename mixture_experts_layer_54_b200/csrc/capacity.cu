@@ -17,6 +17,20 @@
 //            time, ranking equal experts inside a warp with __match_any_sync
 //            and across warps through a per-warp count table.
 // Integers only, so the result is bit-exact with the sequential walk.
+//
+// Batch-prioritized order ("Lab 18" section 3, V-MoE: assignments ranked by
+// router score) adds three launches after the token-order ones, which give
+// the counts, kept, offsets and drop total (the same for every order) and each
+// assignment's token-order place in its expert's list:
+//   list   - every assignment writes a 64-bit key into its expert's list at
+//            that place: high word the score's bits mapped to an unsigned
+//            order, low word ~a, so a larger key means a higher score, or an
+//            equal score and an earlier assignment;
+//   rank   - a block per 256 entries of one expert's list; each entry's queue
+//            position is the number of larger keys in the list (keys are
+//            distinct, so positions are a permutation), read from shared
+//            memory in tiles;
+//   drop   - a token is dropped when none of its k slots was kept.
 #include "internal.cuh"
 
 namespace moe {
@@ -189,7 +203,127 @@ cap_place_kernel(const int32_t *topk, int T, int k, int E, int priority, long lo
     }
 }
 
+// fp32 bits to an unsigned key with the same order (-0 and +0 equal)
+__device__ __forceinline__ uint32_t score_order(float v)
+{
+    uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// exclusive scan of the counts into shared memory (E <= 256, one warp)
+__device__ __forceinline__ void list_offsets(const int32_t *counts, int E, int32_t *lofs)
+{
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < E ? counts[e] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += n;
+            }
+            if (e < E)
+                lofs[e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(256)
+cap_list_kernel(const int32_t *__restrict__ topk, const float *__restrict__ scores, int T, int k,
+                int E, const int32_t *__restrict__ counts, const int32_t *__restrict__ pos_tok,
+                unsigned long long *__restrict__ keys)
+{
+    __shared__ int32_t lofs[kMaxE];
+    list_offsets(counts, E, lofs);
+    const int64_t A = (int64_t)T * k;
+    for (int64_t a = (int64_t)blockIdx.x * 256 + threadIdx.x; a < A; a += (int64_t)gridDim.x * 256) {
+        const int e = topk[a];
+        if (e < 0 || e >= E)
+            continue;
+        const float v = scores[(a / k) * E + e];
+        keys[lofs[e] + pos_tok[a]] =
+            ((unsigned long long)score_order(v) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)a);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+cap_rank_kernel(const unsigned long long *__restrict__ keys, const int32_t *__restrict__ counts,
+                int E, int k, long long C, int32_t *__restrict__ pos, uint8_t *__restrict__ keep)
+{
+    __shared__ int32_t lofs[kMaxE];
+    __shared__ unsigned long long tile[256];
+    const int e = blockIdx.y;
+    const int n = counts[e];
+    const int m = blockIdx.x * 256 + threadIdx.x;
+    if (blockIdx.x * 256 >= n)
+        return;   // whole block: no entries of this expert here
+    list_offsets(counts, E, lofs);
+    const unsigned long long *list = keys + lofs[e];
+    const unsigned long long mine = m < n ? list[m] : 0ull;
+    int ahead = 0;
+    for (int t0 = 0; t0 < n; t0 += 256) {
+        __syncthreads();
+        if (t0 + threadIdx.x < n)
+            tile[threadIdx.x] = list[t0 + threadIdx.x];
+        __syncthreads();
+        const int len = min(256, n - t0);
+        for (int j = 0; j < len; ++j)
+            ahead += tile[j] > mine ? 1 : 0;
+    }
+    if (m < n) {
+        const int64_t a = (int64_t)(0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull));
+        pos[a] = ahead;
+        keep[a] = (long long)ahead < C ? 1 : 0;
+    }
+}
+
+__global__ void cap_drop_kernel(const uint8_t *__restrict__ keep, int T, int k,
+                                uint8_t *__restrict__ dropped)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T)
+        return;
+    int any = 0;
+    for (int j = 0; j < k; ++j)
+        any |= keep[(int64_t)t * k + j];
+    dropped[t] = any ? 0 : 1;
+}
+
 }  // namespace
+
+cudaError_t launch_capacity_scored(const moe_config &c, int64_t C, const int32_t *topk,
+                                   const float *scores, int32_t *counts, int32_t *pos,
+                                   uint8_t *keep, int32_t *kept, int32_t *offsets,
+                                   uint8_t *dropped, int32_t *n_dropped, int32_t *hist,
+                                   int32_t *base, unsigned long long *keys, cudaStream_t s)
+{
+    // token order first: counts, kept, offsets, drop total, and each
+    // assignment's place in its expert's list (written to pos, then replaced)
+    moe_config tok = c;
+    tok.priority = MOE_PRIORITY_TOKEN;
+    cudaError_t err = launch_capacity(tok, C, topk, counts, pos, keep, kept, offsets, dropped,
+                                      n_dropped, hist, base, s);
+    if (err != cudaSuccess || c.T == 0)
+        return err;
+    const int64_t A = (int64_t)c.T * c.k;
+    const int list_blocks = (int)(ceil_div(A, 256) < 1184 ? ceil_div(A, 256) : 1184);
+    cap_list_kernel<<<list_blocks, 256, 0, s>>>(topk, scores, c.T, c.k, c.E, counts, pos, keys);
+    if ((err = cudaGetLastError()) != cudaSuccess)
+        return err;
+    // an expert holds at most T assignments (a token's k experts are distinct)
+    dim3 grid((unsigned)ceil_div(c.T, 256), (unsigned)c.E);
+    cap_rank_kernel<<<grid, 256, 0, s>>>(keys, counts, c.E, c.k, (long long)C, pos, keep);
+    if ((err = cudaGetLastError()) != cudaSuccess)
+        return err;
+    cap_drop_kernel<<<(unsigned)ceil_div(c.T, 256), 256, 0, s>>>(keep, c.T, c.k, dropped);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep, int32_t *kept,

@@ -62,6 +62,8 @@ extern "C" moe_status moe_capacity_noalloc(const moe_config *cfg, const int32_t 
     moe_status st = moe::validate(c);
     if (st != MOE_OK)
         return st;
+    if (c.priority == MOE_PRIORITY_SCORE)
+        return MOE_ERR_DTYPE;   // the score order needs scores and more scratch
     if (!counts || !kept || !offsets || !n_dropped ||
         (c.T > 0 && (!topk_idx || !pos || !keep || !dropped)))
         return MOE_ERR_NULL;

@@ -46,6 +46,7 @@ struct StageScratch {
     void *route;          // tensor-core router: split weights and partial logits
     int32_t *hist;        // [cap_blocks][k][E]
     int32_t *base;        // [cap_blocks][k][E]
+    unsigned long long *keys;   // [T k] batch-prioritized capacity: per-expert lists
     void *H;              // [perm_rows][F] dtype
     void *H_sh;           // [S][T][Fs] dtype
 };
@@ -68,6 +69,18 @@ cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *kept, int32_t *offsets, uint8_t *dropped,
                             int32_t *n_dropped, int32_t *hist, int32_t *base,
                             cudaStream_t s);
+
+cudaError_t launch_capacity_scored(const moe_config &c, int64_t C, const int32_t *topk,
+                                   const float *scores, int32_t *counts, int32_t *pos,
+                                   uint8_t *keep, int32_t *kept, int32_t *offsets,
+                                   uint8_t *dropped, int32_t *n_dropped, int32_t *hist,
+                                   int32_t *base, unsigned long long *keys, cudaStream_t s);
+
+cudaError_t launch_seq_loss(const moe_config &c, int L, const int32_t *topk,
+                            const float *partials, float *per_seq, float *loss, cudaStream_t s);
+
+cudaError_t launch_bias_update(const moe_config &c, const int32_t *counts, float gamma,
+                               float *bias, cudaStream_t s);
 
 cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *topk,
                             const int32_t *pos, const uint8_t *keep,

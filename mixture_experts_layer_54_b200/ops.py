@@ -137,6 +137,51 @@ def moe_capacity(cfg: MoeConfig, topk, ws=None) -> CapacityOut:
     return out
 
 
+def moe_capacity_scored(cfg: MoeConfig, topk, scores, ws=None) -> CapacityOut:
+    """Batch-prioritized capacity: scores [T, E] fp32 are moe_route's
+    scores_out; cfg.priority must be 2 (score order)."""
+    dev = _dev(topk)
+    T, k, E = cfg.T, cfg.k, cfg.E
+    out = CapacityOut(
+        counts=torch.empty((E,), dtype=torch.int32, device=dev),
+        pos=torch.empty((T, k), dtype=torch.int32, device=dev),
+        keep=torch.empty((T, k), dtype=torch.uint8, device=dev),
+        kept=torch.empty((E,), dtype=torch.int32, device=dev),
+        offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+        dropped=torch.empty((T,), dtype=torch.uint8, device=dev),
+        n_dropped=torch.empty((1,), dtype=torch.int32, device=dev))
+    if ws is None:
+        ws = workspace(moe_stage_workspace_size(cfg), dev)
+    check(lib().moe_capacity_scored(ctypes.byref(cfg), _p(topk), _p(scores), _p(out.counts),
+                                    _p(out.pos), _p(out.keep), _p(out.kept), _p(out.offsets),
+                                    _p(out.dropped), _p(out.n_dropped), _p(ws), ws.numel(),
+                                    _stream()), "moe_capacity_scored")
+    return out
+
+
+def moe_seq_balance_loss(cfg: MoeConfig, seq_len: int, topk, loss_partials, per_seq=None,
+                         loss=None):
+    """Sequence-wise balance loss over sequences of seq_len tokens; returns
+    (loss [1], per_seq [T / seq_len]) as device fp32 tensors."""
+    dev = _dev(topk)
+    if per_seq is None:
+        per_seq = torch.empty((max(cfg.T // max(seq_len, 1), 1),), dtype=torch.float32,
+                              device=dev)
+    if loss is None:
+        loss = torch.empty((1,), dtype=torch.float32, device=dev)
+    check(lib().moe_seq_balance_loss(ctypes.byref(cfg), int(seq_len), _p(topk),
+                                     _p(loss_partials), _p(per_seq), _p(loss), _stream()),
+          "moe_seq_balance_loss")
+    return loss, per_seq
+
+
+def moe_bias_update(cfg: MoeConfig, counts, gamma: float, select_bias):
+    """One auxiliary-loss-free balancing step on select_bias (in place)."""
+    check(lib().moe_bias_update(ctypes.byref(cfg), _p(counts), ctypes.c_float(gamma),
+                                _p(select_bias), _stream()), "moe_bias_update")
+    return select_bias
+
+
 def moe_capacity_noalloc(cfg: MoeConfig, topk) -> CapacityOut:
     """moe_capacity with the library's own static scratch instead of a
     workspace (for callers that cannot allocate device memory)."""
@@ -322,7 +367,8 @@ __all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
            "moe_loss_partials_count", "moe_stage_workspace_size", "moe_workspace_size",
            "workspace", "moe_route", "moe_capacity", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_losses", "moe_device_status", "weights_struct", "MoEForward",
-           "HostStream", "moe_forward", "CapacityOut", "StagedForward"]
+           "HostStream", "moe_forward", "CapacityOut", "StagedForward", "moe_capacity_scored",
+           "moe_seq_balance_loss", "moe_bias_update"]
 
 
 class StagedForward:
@@ -351,6 +397,8 @@ class StagedForward:
         self.Y_sh = e((T, d), dt) if cfg.n_shared > 0 else None
         self.y = e((T, d), dt)
         self.aux, self.zloss = e((1,), torch.float32), e((1,), torch.float32)
+        # batch-prioritized capacity ranks by the router scores [T, E]
+        self.scores = e((T, E), torch.float32) if cfg.priority == 2 else None
         self.ws = workspace(moe_stage_workspace_size(cfg), dev)
 
     def __call__(self, x, W_r, W1, W2, W3=None, logit_bias=None, select_bias=None, Ws1=None,
@@ -359,12 +407,19 @@ class StagedForward:
         rec = (lambda i: events[i].record()) if events is not None else (lambda i: None)
         rec(0)
         check(L.moe_route(c, _p(x), _p(W_r), _p(logit_bias), _p(select_bias), _p(self.topk),
-                          _p(self.gates), _p(self.partials), None, None, _p(self.ws),
+                          _p(self.gates), _p(self.partials), None, _p(self.scores), _p(self.ws),
                           self.ws.numel(), s), "moe_route")
         rec(1)
-        check(L.moe_capacity(c, _p(self.topk), _p(self.counts), _p(self.pos), _p(self.keep),
-                             _p(self.kept), _p(self.offsets), _p(self.dropped),
-                             _p(self.n_dropped), _p(self.ws), self.ws.numel(), s), "moe_capacity")
+        if self.scores is not None:
+            check(L.moe_capacity_scored(c, _p(self.topk), _p(self.scores), _p(self.counts),
+                                        _p(self.pos), _p(self.keep), _p(self.kept),
+                                        _p(self.offsets), _p(self.dropped), _p(self.n_dropped),
+                                        _p(self.ws), self.ws.numel(), s), "moe_capacity_scored")
+        else:
+            check(L.moe_capacity(c, _p(self.topk), _p(self.counts), _p(self.pos), _p(self.keep),
+                                 _p(self.kept), _p(self.offsets), _p(self.dropped),
+                                 _p(self.n_dropped), _p(self.ws), self.ws.numel(), s),
+                  "moe_capacity")
         rec(2)
         check(L.moe_dispatch(c, _p(x), _p(self.topk), _p(self.pos), _p(self.keep),
                              _p(self.offsets), _p(self.x_perm), s), "moe_dispatch")

@@ -31,7 +31,7 @@ import torch
 ACT_GELU, ACT_SWIGLU = 0, 1
 SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
 DTYPE_F32, DTYPE_BF16 = 0, 1
-PRIORITY_TOKEN, PRIORITY_RANK = 0, 1
+PRIORITY_TOKEN, PRIORITY_RANK, PRIORITY_SCORE = 0, 1, 2
 
 
 @dataclass(frozen=True)
@@ -222,4 +222,4 @@ def resample_rows(inp: Inputs, rows, attempt: int) -> None:
 __all__ = ["MoEShape", "CONFIGS", "CONFIG_ORDER", "Inputs", "generate", "mixtral_variant",
            "shrink", "resample_rows", "balanced_assignment", "seed_for", "torch_dtype",
            "ACT_GELU", "ACT_SWIGLU", "SCORE_SOFTMAX", "SCORE_SIGMOID", "DTYPE_F32",
-           "DTYPE_BF16", "PRIORITY_TOKEN", "PRIORITY_RANK"]
+           "DTYPE_BF16", "PRIORITY_TOKEN", "PRIORITY_RANK", "PRIORITY_SCORE"]

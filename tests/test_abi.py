@@ -58,12 +58,41 @@ def test_bad_shapes_are_rejected(kw):
 
 
 def test_bad_codes_are_rejected():
-    for kw in (dict(act=2), dict(score=5), dict(dtype=3), dict(priority=2), dict(renorm=4)):
+    for kw in (dict(act=2), dict(score=5), dict(dtype=3), dict(priority=3), dict(renorm=4)):
         base = dict(T=64, d=128, E=8, k=2, d_ff=128, dtype=1, cf=1.0)
         base.update(kw)
         with pytest.raises(moe.MoEError) as ei:
             moe.moe_validate(moe.moe_config(**base))
         assert ei.value.status == _abi.MOE_ERR_DTYPE
+
+
+def test_score_priority_is_only_taken_by_the_scored_capacity_call():
+    L = moe.lib()
+    scored = moe.moe_config(T=64, d=128, E=8, k=2, d_ff=128, dtype=1, cf=1.0, priority=2)
+    token = moe.moe_config(T=64, d=128, E=8, k=2, d_ff=128, dtype=1, cf=1.0, priority=0)
+    nul = [None] * 8
+    assert L.moe_capacity(ctypes.byref(scored), *nul, None, 0, None) == _abi.MOE_ERR_DTYPE
+    assert L.moe_capacity_noalloc(ctypes.byref(scored), *nul, None) == _abi.MOE_ERR_DTYPE
+    assert L.moe_capacity_scored(ctypes.byref(token), *nul, None, None, 0,
+                                 None) == _abi.MOE_ERR_DTYPE
+    assert L.moe_capacity_scored(ctypes.byref(scored), *nul, None, None, 0,
+                                 None) == _abi.MOE_ERR_NULL
+    # the score order needs room for its sort keys
+    assert moe.moe_stage_workspace_size(scored) >= moe.moe_stage_workspace_size(token)
+
+
+def test_seq_loss_and_bias_step_check_their_arguments_before_any_launch():
+    L = moe.lib()
+    cfg = moe.moe_config(T=256, d=128, E=8, k=2, d_ff=128, dtype=1, cf=1.0)
+    for seq_len in (0, 16, 48, 96, 512):   # not a multiple of 32, or not dividing T
+        assert L.moe_seq_balance_loss(ctypes.byref(cfg), seq_len, None, None, None, None,
+                                      None) == _abi.MOE_ERR_SHAPE
+    assert L.moe_seq_balance_loss(ctypes.byref(cfg), 64, None, None, None, None,
+                                  None) == _abi.MOE_ERR_NULL
+    assert L.moe_bias_update(ctypes.byref(cfg), None, ctypes.c_float(float("nan")), None,
+                             None) == _abi.MOE_ERR_SHAPE
+    assert L.moe_bias_update(ctypes.byref(cfg), None, ctypes.c_float(1e-3), None,
+                             None) == _abi.MOE_ERR_NULL
 
 
 def test_null_pointers_are_rejected_before_any_launch():
