@@ -374,6 +374,16 @@ moe_status moe_device_status(const void *ws, int32_t *status,
 /* Clear the device status word (asynchronous, on `stream`). */
 moe_status moe_clear_device_status(void *ws, moe_stream_t stream);
 
+/*
+ * moe_probe_wait_timeout - diagnostic of the failure path: launches one
+ * thread that waits, with the bounded wait the expert GEMMs' roles use, on an
+ * mbarrier that nothing arrives on.  After timeout_ns (at most 2 s, else
+ * MOE_ERR_SHAPE) it gives up and writes MOE_ERR_DEVICE_TIMEOUT to the status
+ * word at the start of ws; nothing else is touched and the CUDA context stays
+ * usable.  Read the result with moe_device_status.
+ */
+moe_status moe_probe_wait_timeout(void *ws, uint64_t timeout_ns, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -69,6 +69,7 @@ SIGNATURES = {
                                    ctypes.POINTER(MoeOutputs), _P, ctypes.c_size_t, _P]),
     "moe_device_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
     "moe_clear_device_status": (ctypes.c_int, [_P, _P]),
+    "moe_probe_wait_timeout": (ctypes.c_int, [_P, ctypes.c_uint64, _P]),
 }
 
 _lib = None

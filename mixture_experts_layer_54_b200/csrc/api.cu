@@ -501,6 +501,16 @@ moe_status moe_device_status(const void *ws, int32_t *status, moe_stream_t strea
     return cuda_status(cudaStreamSynchronize(cs));
 }
 
+moe_status moe_probe_wait_timeout(void *ws, uint64_t timeout_ns, moe_stream_t stream)
+{
+    if (!ws)
+        return MOE_ERR_NULL;
+    if (timeout_ns > 2000000000ull)
+        return MOE_ERR_SHAPE;
+    return cuda_status(launch_wait_probe(static_cast<int32_t *>(ws), timeout_ns,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_clear_device_status(void *ws, moe_stream_t stream)
 {
     if (!ws)

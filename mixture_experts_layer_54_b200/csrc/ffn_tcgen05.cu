@@ -1010,7 +1010,29 @@ cudaError_t launch(const Params &p, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// Diagnostic for the timeout path: one thread waits, with the same bounded
+// wait the GEMM roles use, on an mbarrier that nothing ever arrives on.  The
+// wait must give up after timeout_ns and record MOE_ERR_DEVICE_TIMEOUT; no
+// copy or MMA is in flight, so the kernel simply returns.
+__global__ void wait_probe_kernel(int32_t *status, unsigned long long timeout_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const Ctl ctl{&abort_flag, status, timeout_ns};
+    wait_bar(b, 0, ctl);
+}
+
 }  // namespace tc
+
+cudaError_t launch_wait_probe(int32_t *status, unsigned long long timeout_ns, cudaStream_t s)
+{
+    tc::wait_probe_kernel<<<1, 1, 0, s>>>(status, timeout_ns);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const int32_t *offsets,
                                const void *W1, const void *W3, const void *W2, const void *x,

@@ -95,6 +95,9 @@ cudaError_t launch_losses(const moe_config &c, const int32_t *counts,
                           const float *partials, float *aux, float *zloss,
                           cudaStream_t s);
 
+// one bounded wait on a barrier nobody arrives on (diagnostic)
+cudaError_t launch_wait_probe(int32_t *status, unsigned long long timeout_ns, cudaStream_t s);
+
 // fp32 expert FFNs on the CUDA cores
 cudaError_t launch_ffn_simt(const moe_config &c, const void *x_perm, const int32_t *offsets,
                             const void *W1, const void *W3, const void *W2,

@@ -250,6 +250,16 @@ def moe_device_status(ws) -> int:
     return int(st.value)
 
 
+def moe_clear_device_status(ws):
+    check(lib().moe_clear_device_status(_p(ws), _stream()), "moe_clear_device_status")
+
+
+def moe_probe_wait_timeout(ws, timeout_ns: int):
+    """Diagnostic: one bounded wait that must run out and set the status word."""
+    check(lib().moe_probe_wait_timeout(_p(ws), int(timeout_ns), _stream()),
+          "moe_probe_wait_timeout")
+
+
 def weights_struct(W_r, W1, W2, W3=None, logit_bias=None, select_bias=None, Ws1=None, Ws3=None,
                    Ws2=None) -> MoeWeights:
     def v(t):
@@ -368,7 +378,8 @@ __all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
            "workspace", "moe_route", "moe_capacity", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_losses", "moe_device_status", "weights_struct", "MoEForward",
            "HostStream", "moe_forward", "CapacityOut", "StagedForward", "moe_capacity_scored",
-           "moe_seq_balance_loss", "moe_bias_update"]
+           "moe_seq_balance_loss", "moe_bias_update", "moe_clear_device_status",
+           "moe_probe_wait_timeout"]
 
 
 class StagedForward:

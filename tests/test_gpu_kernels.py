@@ -222,3 +222,28 @@ def test_status_word_is_clear_after_a_normal_call():
     Y, _, ws = moe.moe_expert_ffn(cfg, x_perm, off, W, W, W)
     assert moe.moe_device_status(ws) == 0
     assert torch.count_nonzero(Y[:128]).item() == 0
+
+
+def test_a_wait_that_runs_out_sets_the_status_and_leaves_the_context_usable():
+    """The bounded wait of the expert GEMMs' roles, on a barrier nothing
+    arrives on, gives up after its limit and records MOE_ERR_DEVICE_TIMEOUT;
+    afterwards the same workspace, cleared, serves a normal call."""
+    from mixture_experts_layer_54_b200 import _abi
+    cfg = moe.moe_config(T=128, d=128, E=2, k=1, d_ff=128, act=1, dtype=1, cf=math.inf)
+    ws = moe.workspace(moe.moe_stage_workspace_size(cfg), DEV)
+    moe.moe_clear_device_status(ws)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    moe.moe_probe_wait_timeout(ws, 50_000_000)   # 50 ms
+    end.record()
+    assert moe.moe_device_status(ws) == _abi.MOE_ERR_DEVICE_TIMEOUT
+    assert 40.0 <= start.elapsed_time(end) < 1000.0
+    R = moe.moe_perm_rows(cfg)
+    g = torch.Generator(device=DEV).manual_seed(1)
+    x_perm = torch.randn((R, 128), generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn((2, 128, 128), generator=g, device=DEV) / 12).to(torch.bfloat16)
+    off = torch.tensor([0, 128, 128], dtype=torch.int32, device=DEV)
+    Y, _, _ = moe.moe_expert_ffn(cfg, x_perm, off, W, W, W, ws=ws)   # clears the word
+    assert moe.moe_device_status(ws) == 0
+    _close_bf16(Y[:128], _ffn_ref(x_perm[:128], W[0], W[0], W[0], 1))
