@@ -58,7 +58,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture (profiles/gemm_2sm_mixtral.md), valid only for the GEMM source it was taken on.
 GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_54_b200", "csrc", "ffn_tcgen05.cu")
 MEASURED_TRAFFIC = {
-    ("mixtral", "76528806f495b963bf05080db2666b5375ae3e33383fcce51776a9056bf3eb02"): 6.717e9,
+    ("mixtral", "08ae4c3a6308cecf9ae9b989daf9ff4b24a9fde50c41e13a8b341ad90fc61747"): 4.975e9,
 }
 
 
@@ -450,9 +450,13 @@ def run_ours(args):
         stages[name] = entry
     ffn = work["expert_ffn"]
     ach = ffn["flops"] / (st["expert_ffn"] / 1e3) / 1e12
-    # the stage runs inside a step of a long graph replay, under the power cap:
-    # its peak is the sustained matmul figure (the burst one is kept beside it)
-    peak = peaks["bf16_tflops_sustained"]
+    # The stage runs inside a step of one graph replay.  A timed region long
+    # enough for the 1 kW power cap to settle (>= 0.2 s) is compared with the
+    # sustained matmul figure, a shorter one with the burst figure; both
+    # fractions are reported.
+    region_s = ms_per_step * args.steps / 1e3
+    peak_kind = "sustained" if region_s >= 0.2 else "burst"
+    peak = peaks["bf16_tflops_sustained" if peak_kind == "sustained" else "bf16_tflops"]
     roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(ach / peak, 4),
                 "traffic": measured_traffic(args.config),
@@ -460,8 +464,10 @@ def run_ours(args):
                 "algorithmic_bytes": ffn["bytes"],
                 "kernel": "moe_expert_ffn: grouped tcgen05 GEMM1 (act fused) + GEMM2",
                 "flops_per_launch": ffn["flops"],
-                "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
-                "frac_of_burst": round(ach / peaks["bf16_tflops"], 4)}
+                "peak_source": f"{peak_src} bf16 {peak_kind} (MEASURED_PEAKS.json)",
+                "timed_region_s": round(region_s, 3),
+                "frac_of_burst": round(ach / peaks["bf16_tflops"], 4),
+                "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4)}
     t_flop = ffn["flops"] / (peak * 1e12)
     all_bytes = sum(v.get("bytes", 0) for v in work.values())
     t_byte = all_bytes / (peaks["hbm_gbs"] * 1e9)
