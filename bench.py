@@ -179,6 +179,13 @@ class ClockSampler:
 
 # ------------------------------------------------------------ work accounting
 
+def perm_rows(shape) -> int:
+    """Rows of the permuted buffers: kept slots plus per-expert padding to 128."""
+    C = shape.T if math.isinf(shape.cf) else math.ceil(shape.cf * shape.T * shape.k / shape.E)
+    kept = min(shape.T * shape.k, C * shape.E)
+    return (kept + shape.E * 127 + 127) // 128 * 128
+
+
 def layer_work(shape, counts, kept_total, dropped_tokens):
     """Algorithmic FLOPs and bytes of one step (no padding rows, no dense E-way
     work), per stage."""
@@ -195,6 +202,8 @@ def layer_work(shape, counts, kept_total, dropped_tokens):
         "route": {"bytes": T * d * b + d * E * 4 + T * k * 8 + math.ceil(T / 32) * (E + 1) * 4,
                   "flops": 2.0 * T * d * E},
         "dispatch": {"bytes": routed_tokens * d * b + N * d * b + T * k * 9},
+        # the dispatch fused into GEMM1 instead: the row table (cleared, one entry per kept slot)
+        "dispatch_rows": {"bytes": perm_rows(shape) * 4 + T * k * 9 + N * 4},
         "expert_ffn": {"flops": ffn_flops, "bytes": ffn_bytes},
         "combine": {"bytes": N * d * b + (T * d * b if S else 0) + T * d * b + T * k * 9},
         "capacity": {"bytes": T * k * 4 * 3 + T * k + T},
@@ -287,6 +296,32 @@ def next_rows(moe, shape, inp, staged, seq_len):
             "seq_balance_loss": {"us": round(t_seq, 2), "seq_len": seq_len, "launches": 2,
                                  "value": round(float(loss.item()), 6)},
             "bias_update": {"us": round(t_bias, 2), "launches": 1}}
+
+
+def fused_dispatch(moe, cfg, inp, staged):
+    """The dispatch fused into GEMM1 (row table + gathered expert FFN) against
+    the permuted copy + expert FFN that the step runs, same batch, same box."""
+    R = moe.moe_perm_rows(cfg)
+    dev = inp.x.device
+    rows = torch.empty((R,), dtype=torch.int32, device=dev)
+    Y = torch.empty_like(staged.Y_perm)
+    Ysh = None if staged.Y_sh is None else torch.empty_like(staged.Y_sh)
+
+    def fused():
+        moe.moe_dispatch_rows(cfg, staged.topk, staged.pos, staged.keep, staged.offsets, rows)
+        moe.moe_expert_ffn_gather(cfg, inp.x, rows, staged.offsets, inp.W1, inp.W3, inp.W2,
+                                  inp.Ws1, inp.Ws3, inp.Ws2, ws=staged.ws, Y_perm=Y, Y_shared=Ysh)
+
+    def unfused():
+        moe.moe_dispatch(cfg, inp.x, staged.topk, staged.pos, staged.keep, staged.offsets,
+                         staged.x_perm)
+        moe.moe_expert_ffn(cfg, staged.x_perm, staged.offsets, inp.W1, inp.W3, inp.W2, inp.x,
+                           inp.Ws1, inp.Ws3, inp.Ws2, ws=staged.ws, Y_perm=Y, Y_shared=Ysh)
+    t_fused = graph_time_us(fused, n=5)
+    t_unfused = graph_time_us(unfused, n=5)
+    return {"us": round(t_fused, 1), "unfused_us": round(t_unfused, 1), "launches": 3,
+            "note": "moe_dispatch_rows + moe_expert_ffn_gather (TMA gather4 rows) vs "
+                    "moe_dispatch + moe_expert_ffn"}
 
 
 def cpu_baseline(shape, inp, seconds):
@@ -429,6 +464,8 @@ def run_ours(args):
 
     extra = next_rows(moe, shape, inp, staged, seq_len=min(shape.T, 1024)) \
         if shape.T % 32 == 0 and shape.T > 0 else None
+    if extra is not None:
+        extra["fused_dispatch"] = fused_dispatch(moe, cfg, inp, staged)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -469,7 +506,7 @@ def run_ours(args):
                 "frac_of_burst": round(ach / peaks["bf16_tflops"], 4),
                 "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4)}
     t_flop = ffn["flops"] / (peak * 1e12)
-    all_bytes = sum(v.get("bytes", 0) for v in work.values())
+    all_bytes = sum(work[n].get("bytes", 0) for n in moe.StagedForward.STAGES)
     t_byte = all_bytes / (peaks["hbm_gbs"] * 1e9)
     layer_roof = {"t_flop_us": round(t_flop * 1e6, 1), "t_byte_us": round(t_byte * 1e6, 1),
                   "bound": "tensor" if t_flop >= t_byte else "hbm",

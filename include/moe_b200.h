@@ -268,6 +268,18 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x,
                         void *x_perm, moe_stream_t stream);
 
 /*
+ * moe_dispatch_rows - the dispatch as a row table, for moe_expert_ffn_gather
+ * (the dispatch fused into the expert GEMM): src_rows[offsets[e] + pos[t, j]]
+ * = t for every kept (t, j); every other row (segment padding) = 0.
+ *   topk_idx, pos, keep, offsets from moe_capacity; src_rows [moe_perm_rows]
+ *   int32 out (device).  Moves T k small entries instead of the rows.
+ */
+moe_status moe_dispatch_rows(const moe_config *cfg, const int32_t *topk_idx,
+                             const int32_t *pos, const uint8_t *keep,
+                             const int32_t *offsets, int32_t *src_rows,
+                             moe_stream_t stream);
+
+/*
  * moe_expert_ffn - the expert FFNs over the expert segments, and the shared
  * experts over all tokens ("Lab 18" section 1 expert definitions, tips: one
  * grouped matrix multiply over all experts).
@@ -287,6 +299,22 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm,
                           const void *Ws1, const void *Ws3, const void *Ws2,
                           void *Y_perm, void *Y_shared, void *ws,
                           size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn_gather - moe_expert_ffn with the dispatch fused in: row r of
+ * segment e is token src_rows[r] of x, read by GEMM1 straight from x (bf16:
+ * TMA row gathers into each tile; fp32: indexed loads), so x_perm is never
+ * written.  Results are those of moe_dispatch + moe_expert_ffn on the same
+ * rows.
+ *   x [T, d] dtype in; src_rows [moe_perm_rows] from moe_dispatch_rows;
+ *   every other argument as for moe_expert_ffn.
+ */
+moe_status moe_expert_ffn_gather(const moe_config *cfg, const void *x,
+                                 const int32_t *src_rows, const int32_t *offsets,
+                                 const void *W1, const void *W3, const void *W2,
+                                 const void *Ws1, const void *Ws3, const void *Ws2,
+                                 void *Y_perm, void *Y_shared, void *ws,
+                                 size_t ws_bytes, moe_stream_t stream);
 
 /*
  * moe_combine - gate-weighted sum plus shared experts ("Lab 18" section 1,

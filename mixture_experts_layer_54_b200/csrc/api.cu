@@ -309,6 +309,19 @@ moe_status moe_capacity_scored(const moe_config *cfg, const int32_t *topk_idx,
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_dispatch_rows(const moe_config *cfg, const int32_t *topk_idx, const int32_t *pos,
+                             const uint8_t *keep, const int32_t *offsets, int32_t *src_rows,
+                             moe_stream_t stream)
+{
+    moe_status st = check_cfg(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (!offsets || !src_rows || (cfg->T > 0 && (!topk_idx || !pos || !keep)))
+        return MOE_ERR_NULL;
+    return cuda_status(launch_dispatch_rows(*cfg, topk_idx, pos, keep, offsets, src_rows,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_idx,
                         const int32_t *pos, const uint8_t *keep, const int32_t *offsets,
                         void *x_perm, moe_stream_t stream)
@@ -329,8 +342,9 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *top
 namespace {
 
 moe_status expert_ffn_impl(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
-                           const void *W1, const void *W3, const void *W2, const void *x,
-                           const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
+                           const int32_t *src_rows, const void *W1, const void *W3,
+                           const void *W2, const void *x, const void *Ws1, const void *Ws3,
+                           const void *Ws2, void *Y_perm,
                            void *Y_shared, void *ws, size_t ws_bytes, moe_stream_t stream,
                            bool clear_status)
 {
@@ -340,7 +354,9 @@ moe_status expert_ffn_impl(const moe_config *cfg, const void *x_perm, const int3
     const moe_config &c = *cfg;
     const bool swiglu = c.act == MOE_ACT_SWIGLU;
     const bool shared = c.n_shared > 0;
-    if (!x_perm || !offsets || !W1 || !W2 || !Y_perm || !ws || (swiglu && !W3))
+    if (!offsets || !W1 || !W2 || !Y_perm || !ws || (swiglu && !W3))
+        return MOE_ERR_NULL;
+    if (src_rows ? (c.T > 0 && !x) : !x_perm)   // routed rows: gathered from x, or x_perm
         return MOE_ERR_NULL;
     if (shared && (!x || !Ws1 || !Ws2 || !Y_shared || (swiglu && !Ws3)))
         return MOE_ERR_NULL;
@@ -358,10 +374,11 @@ moe_status expert_ffn_impl(const moe_config *cfg, const void *x_perm, const int3
     if (clear_status && cudaMemsetAsync(s.status, 0, sizeof(int32_t), cs) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (c.dtype == MOE_DTYPE_BF16)
-        e = launch_ffn_tcgen05(c, x_perm, offsets, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
+        e = launch_ffn_tcgen05(c, x_perm, offsets, src_rows, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
                                Y_shared, s.H, s.H_sh, s.status, cs);
     else
-        e = launch_ffn_simt(c, x_perm, offsets, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm, Y_shared,
+        e = launch_ffn_simt(c, x_perm, offsets, src_rows, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
+                            Y_shared,
                             s.H, s.H_sh, cs);
     return cuda_status(e);
 }
@@ -373,8 +390,20 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32
                           const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
                           void *Y_shared, void *ws, size_t ws_bytes, moe_stream_t stream)
 {
-    return expert_ffn_impl(cfg, x_perm, offsets, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm, Y_shared,
-                           ws, ws_bytes, stream, true);
+    return expert_ffn_impl(cfg, x_perm, offsets, nullptr, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
+                           Y_shared, ws, ws_bytes, stream, true);
+}
+
+moe_status moe_expert_ffn_gather(const moe_config *cfg, const void *x, const int32_t *src_rows,
+                                 const int32_t *offsets, const void *W1, const void *W3,
+                                 const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
+                                 void *Y_perm, void *Y_shared, void *ws, size_t ws_bytes,
+                                 moe_stream_t stream)
+{
+    if (!src_rows)
+        return MOE_ERR_NULL;
+    return expert_ffn_impl(cfg, nullptr, offsets, src_rows, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
+                           Y_shared, ws, ws_bytes, stream, true);
 }
 
 moe_status moe_combine(const moe_config *cfg, const void *Y_perm, const void *Y_shared,
@@ -482,8 +511,8 @@ moe_status moe_forward(const moe_config *cfg, const moe_weights *w, const void *
         return st;
     if ((st = moe_dispatch(cfg, x, f.topk, f.pos, f.keep, f.offsets, f.x_perm, stream)) != MOE_OK)
         return st;
-    if ((st = expert_ffn_impl(cfg, f.x_perm, f.offsets, w->W1, w->W3, w->W2, x, w->Ws1, w->Ws3,
-                              w->Ws2, f.Y_perm, f.Y_sh, ws, ssz, stream, false)) != MOE_OK)
+    if ((st = expert_ffn_impl(cfg, f.x_perm, f.offsets, nullptr, w->W1, w->W3, w->W2, x, w->Ws1,
+                              w->Ws3, w->Ws2, f.Y_perm, f.Y_sh, ws, ssz, stream, false)) != MOE_OK)
         return st;
     if ((st = moe_combine(cfg, f.Y_perm, f.Y_sh, f.gates, f.topk, f.pos, f.keep, f.offsets,
                           nullptr, out->y, stream)) != MOE_OK)

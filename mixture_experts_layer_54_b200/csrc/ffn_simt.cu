@@ -37,6 +37,7 @@ struct SimtGemm {
     float *C;
     int64_t ldc;
     int64_t c_group_col;         // dense, blockIdx.z = group: C column offset per group
+    const int32_t *a_rows;       // non-null: row r of A is row a_rows[r] of the A tensor
 };
 
 __device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(THREADS) simt_gemm_kernel(SimtGemm p)
             for (int i = threadIdx.x; i < TILE * KC; i += THREADS) {
                 int r = i / KC, c = i % KC;
                 int row = m0 + r, kk = k0 + c, n = n0 + r;
-                As[r][c] = (row < row_end && kk < p.Kg) ? p.A[(int64_t)row * p.lda + a_col0 + kk] : 0.f;
+                const int64_t arow = (row < row_end && p.a_rows) ? p.a_rows[row] : row;
+                As[r][c] = (row < row_end && kk < p.Kg) ? p.A[arow * p.lda + a_col0 + kk] : 0.f;
                 Bs[r][c] = (n < p.N && kk < p.Kg) ? B[(int64_t)n * p.Kg + kk] : 0.f;
                 if (ACT == ACT_SWIGLU)
                     B3s[r][c] = (n < p.N && kk < p.Kg) ? B3[(int64_t)n * p.Kg + kk] : 0.f;
@@ -137,7 +139,7 @@ cudaError_t run(const SimtGemm &p, int act, int grid_m, int grid_z, cudaStream_t
 }  // namespace
 
 cudaError_t launch_ffn_simt(const moe_config &c, const void *x_perm, const int32_t *offsets,
-                            const void *W1, const void *W3, const void *W2, const void *x,
+                            const int32_t *src_rows, const void *W1, const void *W3, const void *W2, const void *x,
                             const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
                             void *Y_sh, void *H, void *H_sh, cudaStream_t s)
 {
@@ -145,10 +147,11 @@ cudaError_t launch_ffn_simt(const moe_config &c, const void *x_perm, const int32
     const int R = (int)perm_rows(c);
     const int gm = (int)ceil_div(R, TILE);
     cudaError_t err;
-    // routed GEMM1: H = act(x_perm W1^T)
-    SimtGemm g1{static_cast<const float *>(x_perm), c.d, 0, offsets, c.E,
+    // routed GEMM1: H = act(x_perm W1^T), or with src_rows the rows of x
+    SimtGemm g1{static_cast<const float *>(src_rows ? x : x_perm), c.d, 0, offsets, c.E,
                 static_cast<const float *>(W1), static_cast<const float *>(W3),
-                (int64_t)c.d_ff * c.d, c.d_ff, c.d, 1, static_cast<float *>(H), c.d_ff, 0};
+                (int64_t)c.d_ff * c.d, c.d_ff, c.d, 1, static_cast<float *>(H), c.d_ff, 0,
+                src_rows};
     if ((err = run(g1, act1, gm, 1, s)) != cudaSuccess)
         return err;
     // routed GEMM2: Y_perm = H W2^T

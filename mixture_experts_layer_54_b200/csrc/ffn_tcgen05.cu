@@ -8,7 +8,11 @@
 // ("Lab 18" section 1, DeepSeekMoE row).
 //
 // Two launches: GEMM1 (hidden = act(A W1^T), SwiGLU fuses W3) and GEMM2
-// (out = hidden W2^T).  Each launch covers two tile sets:
+// (out = hidden W2^T).  GEMM1's routed A rows come either from the permuted
+// buffer x_perm or, with the dispatch fused in, straight from x: each tile's
+// 128 rows are gathered by TMA (tile::gather4, four rows per copy, one copy
+// per lane of the producer warp) through the per-row source table that
+// moe_dispatch_rows writes.  Each launch covers two tile sets:
 //   set 0, routed: for expert e the rows [offsets[e], offsets[e+1]) of the
 //          permuted buffer, read from device memory (no host sync); segments
 //          start on multiples of 128 rows, so a 128-row tile has one expert;
@@ -65,9 +69,13 @@ struct SetDesc {
 
 struct __align__(64) Params {
     CUtensorMap tmA[2], tmB[2], tmB3[2], tmC[2];
+    CUtensorMap tmX;             // x as a 2-D [T][d] map with one-row boxes (gathered A)
     SetDesc set[2];
     int nsets;
     int E;
+    int gather;                  // 1: routed A rows gathered from x through src_rows
+    int n_rows;                  // rows of the permuted buffers (entries of src_rows)
+    const int32_t *src_rows;     // [n_rows] token of each permuted row
     const int32_t *offsets;
     int32_t *status;
     unsigned long long timeout_ns;
@@ -155,6 +163,27 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
         : "memory");
+}
+
+// Four rows (r0..r3) of a 2-D map, one 64-element box each, into 512
+// consecutive bytes of shared memory (the same swizzled layout a 4-row box
+// would give at that offset).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int col, int r0, int r1, int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "r"(bar)
+        : "memory");
+}
+
+// the source row of permuted row r (rows past the table read token 0; their
+// results are never used)
+__device__ __forceinline__ int gather_row(const Params &p, int r)
+{
+    return r < p.n_rows ? p.src_rows[r] : 0;
 }
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
@@ -295,7 +324,7 @@ __device__ __forceinline__ void epilogue_chunk(const float *g, const float *u, u
     }
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p)
 {
     constexpr int BN_B = EPI == EPI_SWIGLU ? BN / 2 : BN;     // B rows per tensor per tile
@@ -372,7 +401,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
 
     if (warp == 0) {
         // ================= TMA producer =================
-        if (lane == 0) {
+        // Lane 0 owns the barrier waits and the box copies; with gathered A
+        // rows (GATHER) the whole warp runs and every lane copies four of the
+        // tile's 128 rows.  The other lanes of the warp stay in this branch.
+        if (GATHER || lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int issued[STAGES];
@@ -383,8 +415,24 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
                 const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
                 const SetDesc &sd = p.set[t.set];
+                const bool gath = GATHER && t.set == 0;
+                int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
+                if (gath) {
+                    const int r = t.m0 + lane * 4;
+                    g0 = gather_row(p, r);
+                    g1 = gather_row(p, r + 1);
+                    g2 = gather_row(p, r + 2);
+                    g3 = gather_row(p, r + 3);
+                }
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
-                    if (!wait_bar(empty_bar(stage), phase ^ 1u, ctl)) {
+                    int okw = 1;
+                    if (lane == 0)
+                        okw = wait_bar(empty_bar(stage), phase ^ 1u, ctl) ? 1 : 0;
+                    if (GATHER) {
+                        okw = __shfl_sync(0xffffffffu, okw, 0);
+                        __syncwarp();
+                    }
+                    if (!okw) {
                         ok = false;
                         break;
                     }
@@ -394,14 +442,20 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                         kcol = (kb % sd.kbg) * BK;
                     }
                     const uint32_t fb = full_bar(stage);
-                    mbar_expect_tx(fb, A_BYTES + B_BYTES);
-                    tma_load_3d(sA + stage * A_BYTES, &p.tmA[t.set], fb, kcol, t.m0, ga);
-                    if (EPI == EPI_SWIGLU) {
-                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
-                        tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &p.tmB3[t.set], fb, kcol,
-                                    t.b_row, gb);
-                    } else {
-                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                    if (lane == 0)
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                    if (gath)
+                        tma_gather4(sA + stage * A_BYTES + lane * 512, &p.tmX, fb, kcol, g0, g1, g2, g3);
+                    if (lane == 0) {
+                        if (!gath)
+                            tma_load_3d(sA + stage * A_BYTES, &p.tmA[t.set], fb, kcol, t.m0, ga);
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                            tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &p.tmB3[t.set], fb, kcol,
+                                        t.b_row, gb);
+                        } else {
+                            tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                        }
                     }
                     issued[stage] = 1;
                     last_phase[stage] = phase;
@@ -411,10 +465,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                     }
                 }
             }
-            // drain: every load this thread issued has landed before the CTA exits
-            for (int s = 0; s < STAGES; ++s)
-                if (issued[s])
-                    wait_bar(full_bar(s), last_phase[s], ctl, false);
+            // drain: every load this warp issued has landed before the CTA exits
+            if (lane == 0)
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s])
+                        wait_bar(full_bar(s), last_phase[s], ctl, false);
+            if (GATHER)
+                __syncwarp();
         }
     } else if (warp == 1) {
         // ================= MMA issuer =================
@@ -600,6 +657,19 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
+// tma_gather4 with the completion reported to the leader CTA's barrier
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t bar_leader, int col, int r0, int r1,
+                                                 int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+        "complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "r"(bar_leader)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                               uint32_t accumulate)
 {
@@ -677,7 +747,7 @@ __device__ __forceinline__ Tile2 decode2(const Params &p, const int *tstart, con
     return t;
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __grid_constant__ Params p)
 {
     constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;   // output columns per tile
@@ -756,7 +826,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
 
     if (warp == 0) {
         // ================= TMA producer (both CTAs) =================
-        if (lane == 0) {
+        // Lane 0 owns the barrier waits and the box copies; with gathered A
+        // rows (GATHER) the whole warp runs and every lane copies four of its
+        // CTA's 128 rows.  The other lanes of the warp stay in this branch.
+        if (GATHER || lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int issued[STAGES2];
@@ -771,8 +844,24 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                                                    : t.n_idx * BN + (int)rank * (BN / 2);
                 const CUtensorMap *bmap =
                     (EPI == EPI_SWIGLU && rank == 1) ? &p.tmB3[t.set] : &p.tmB[t.set];
+                const bool gath = GATHER && t.set == 0;
+                int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
+                if (gath) {
+                    const int r = t.m0 + (int)rank * 128 + lane * 4;
+                    g0 = gather_row(p, r);
+                    g1 = gather_row(p, r + 1);
+                    g2 = gather_row(p, r + 2);
+                    g3 = gather_row(p, r + 3);
+                }
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
-                    if (!wait_bar(empty_bar(stage), phase ^ 1u, ctl)) {
+                    int okw = 1;
+                    if (lane == 0)
+                        okw = wait_bar(empty_bar(stage), phase ^ 1u, ctl) ? 1 : 0;
+                    if (GATHER) {
+                        okw = __shfl_sync(0xffffffffu, okw, 0);
+                        __syncwarp();
+                    }
+                    if (!okw) {
                         ok = false;
                         break;
                     }
@@ -781,14 +870,21 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                         ga = gb = kb / sd.kbg;
                         kcol = (kb % sd.kbg) * BK * KSUB;
                     }
-                    if (leader)
+                    if (leader && lane == 0)
                         mbar_expect_tx(full_bar(stage), 4 * KSUB * HALF_BYTES);
                     const uint32_t fb = map_to_rank(full_bar(stage), 0);
                     for (int ks = 0; ks < KSUB; ++ks) {
-                        tma_load_3d_pair(sA + (stage * KSUB + ks) * HALF_BYTES, &p.tmA[t.set], fb,
-                                         kcol + ks * BK, t.m0 + (int)rank * 128, ga);
-                        tma_load_3d_pair(sB + (stage * KSUB + ks) * HALF_BYTES, bmap, fb,
-                                         kcol + ks * BK, brow, gb);
+                        const uint32_t a_dst = sA + (stage * KSUB + ks) * HALF_BYTES;
+                        if (gath)
+                            tma_gather4_pair(a_dst + lane * 512, &p.tmX, fb, kcol + ks * BK, g0, g1,
+                                             g2, g3);
+                        if (lane == 0) {
+                            if (!gath)
+                                tma_load_3d_pair(a_dst, &p.tmA[t.set], fb, kcol + ks * BK,
+                                                 t.m0 + (int)rank * 128, ga);
+                            tma_load_3d_pair(sB + (stage * KSUB + ks) * HALF_BYTES, bmap, fb,
+                                             kcol + ks * BK, brow, gb);
+                        }
                     }
                     issued[stage] = 1;
                     last_phase[stage] = phase;
@@ -799,10 +895,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                 }
             }
             // the leader's full barriers count both CTAs' bytes: drain there
-            if (leader)
+            if (leader && lane == 0)
                 for (int s = 0; s < STAGES2; ++s)
                     if (issued[s])
                         wait_bar(full_bar(s), last_phase[s], ctl, false);
+            if (GATHER)
+                __syncwarp();
         }
     } else if (warp == 1) {
         // ================= MMA issuer (leader CTA only) =================
@@ -970,6 +1068,23 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64
     return r == CUDA_SUCCESS;
 }
 
+// 2-D bf16 tensor (d0 contiguous x d1 rows, row pitch s1 bytes)
+bool make_map2d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t s1,
+                uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw)
+{
+    EncodeTiled enc = encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {d0, d1 > 0 ? d1 : 1};
+    cuuint64_t strides[1] = {s1};
+    cuuint32_t box[2] = {b0, b1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int sm_count()
 {
     int dev = 0, n = 148;
@@ -978,10 +1093,10 @@ int sm_count()
     return n;
 }
 
-template <int EPI>
+template <int EPI, bool GATHER = false>
 cudaError_t launch_2sm(const Params &p, cudaStream_t s)
 {
-    auto kern = grouped_gemm_2sm_kernel<EPI>;
+    auto kern = grouped_gemm_2sm_kernel<EPI, GATHER>;
     cudaError_t err =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
     if (err != cudaSuccess)
@@ -1011,10 +1126,10 @@ cudaError_t launch_2sm(const Params &p, cudaStream_t s)
     return cudaGetLastError();
 }
 
-template <int EPI>
+template <int EPI, bool GATHER = false>
 cudaError_t launch(const Params &p, cudaStream_t s)
 {
-    auto kern = grouped_gemm_kernel<EPI>;
+    auto kern = grouped_gemm_kernel<EPI, GATHER>;
     cudaError_t err =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess)
@@ -1048,7 +1163,7 @@ cudaError_t launch_wait_probe(int32_t *status, unsigned long long timeout_ns, cu
 }
 
 cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const int32_t *offsets,
-                               const void *W1, const void *W3, const void *W2, const void *x,
+                               const int32_t *src_rows, const void *W1, const void *W3, const void *W2, const void *x,
                                const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
                                void *Y_sh, void *H, void *H_sh, int32_t *status, cudaStream_t s)
 {
@@ -1079,7 +1194,15 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     p1.timeout_ns = 2000000000ull;
     p1.nsets = shared ? 2 : 1;
     bool ok = true;
-    ok &= make_map(&p1.tmA[0], x_perm, d, R, 1, d * 2, 0, BK, BM, SW128);
+    if (src_rows) {
+        // dispatch fused in: tile rows gathered from x, one-row boxes (gather4)
+        p1.gather = 1;
+        p1.src_rows = src_rows;
+        p1.n_rows = (int)R;
+        ok &= make_map2d(&p1.tmX, x, d, T, d * 2, BK, 1, SW128);
+    } else {
+        ok &= make_map(&p1.tmA[0], x_perm, d, R, 1, d * 2, 0, BK, BM, SW128);
+    }
     ok &= make_map(&p1.tmB[0], W1, d, F, E, d * 2, F * d * 2, BK, bn_b, SW128);
     if (swiglu)
         ok &= make_map(&p1.tmB3[0], W3, d, F, E, d * 2, F * d * 2, BK, bn_b, SW128);
@@ -1098,8 +1221,13 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     }
     if (!ok)
         return cudaErrorInvalidValue;
-    cudaError_t err = pair ? (swiglu ? launch_2sm<EPI_SWIGLU>(p1, s) : launch_2sm<EPI_GELU>(p1, s))
-                           : (swiglu ? launch<EPI_SWIGLU>(p1, s) : launch<EPI_GELU>(p1, s));
+    cudaError_t err;
+    if (p1.gather)
+        err = pair ? (swiglu ? launch_2sm<EPI_SWIGLU, true>(p1, s) : launch_2sm<EPI_GELU, true>(p1, s))
+                   : (swiglu ? launch<EPI_SWIGLU, true>(p1, s) : launch<EPI_GELU, true>(p1, s));
+    else
+        err = pair ? (swiglu ? launch_2sm<EPI_SWIGLU>(p1, s) : launch_2sm<EPI_GELU>(p1, s))
+                   : (swiglu ? launch<EPI_SWIGLU>(p1, s) : launch<EPI_GELU>(p1, s));
     if (err != cudaSuccess)
         return err;
 

@@ -82,6 +82,10 @@ cudaError_t launch_seq_loss(const moe_config &c, int L, const int32_t *topk,
 cudaError_t launch_bias_update(const moe_config &c, const int32_t *counts, float gamma,
                                float *bias, cudaStream_t s);
 
+cudaError_t launch_dispatch_rows(const moe_config &c, const int32_t *topk, const int32_t *pos,
+                                 const uint8_t *keep, const int32_t *offsets, int32_t *src_rows,
+                                 cudaStream_t s);
+
 cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *topk,
                             const int32_t *pos, const uint8_t *keep,
                             const int32_t *offsets, void *x_perm, cudaStream_t s);
@@ -100,14 +104,15 @@ cudaError_t launch_wait_probe(int32_t *status, unsigned long long timeout_ns, cu
 
 // fp32 expert FFNs on the CUDA cores
 cudaError_t launch_ffn_simt(const moe_config &c, const void *x_perm, const int32_t *offsets,
-                            const void *W1, const void *W3, const void *W2,
+                            const int32_t *src_rows, const void *W1, const void *W3, const void *W2,
                             const void *x, const void *Ws1, const void *Ws3,
                             const void *Ws2, void *Y_perm, void *Y_sh, void *H,
                             void *H_sh, cudaStream_t s);
 
 // bf16 expert FFNs on the tensor cores (tcgen05 + TMEM + TMA)
 cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm,
-                               const int32_t *offsets, const void *W1, const void *W3,
+                               const int32_t *offsets, const int32_t *src_rows,
+                               const void *W1, const void *W3,
                                const void *W2, const void *x, const void *Ws1,
                                const void *Ws3, const void *Ws2, void *Y_perm,
                                void *Y_sh, void *H, void *H_sh, int32_t *status,

@@ -81,6 +81,23 @@ dispatch_vec_kernel(const uint4 *__restrict__ x, int T, int k, int E, int nvec,
     }
 }
 
+// Dispatch fused into the expert GEMM: instead of copying rows, record for
+// every kept assignment (t, j) that permuted row offsets[e] + pos[t, j] holds
+// token t.  Padding rows keep the 0 the table was cleared to.
+__global__ void dispatch_rows_kernel(const int32_t *__restrict__ topk,
+                                     const int32_t *__restrict__ pos,
+                                     const uint8_t *__restrict__ keep,
+                                     const int32_t *__restrict__ offsets, int64_t A, int k, int E,
+                                     int32_t *__restrict__ src_rows)
+{
+    for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < A;
+         a += (int64_t)gridDim.x * blockDim.x) {
+        const int e = topk[a];
+        if (keep[a] && e >= 0 && e < E)
+            src_rows[offsets[e] + pos[a]] = (int32_t)(a / k);
+    }
+}
+
 // 8 values of a 16-byte vector, widened to fp32
 template <typename T> struct Vec;
 template <> struct Vec<__nv_bfloat16> {
@@ -224,6 +241,19 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *t
     dispatch_vec_kernel<<<grid_for(dispatch_vec_kernel, c.T), THREADS, 0, s>>>(
         static_cast<const uint4 *>(x), c.T, c.k, c.E, nvec, topk, pos, keep, offsets,
         static_cast<uint4 *>(x_perm));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_rows(const moe_config &c, const int32_t *topk, const int32_t *pos,
+                                 const uint8_t *keep, const int32_t *offsets, int32_t *src_rows,
+                                 cudaStream_t s)
+{
+    cudaError_t err = cudaMemsetAsync(src_rows, 0, sizeof(int32_t) * (size_t)perm_rows(c), s);
+    if (err != cudaSuccess || c.T == 0)
+        return err;
+    const int64_t A = (int64_t)c.T * c.k;
+    const int blocks = (int)(ceil_div(A, 256) < 1184 ? ceil_div(A, 256) : 1184);
+    dispatch_rows_kernel<<<blocks, 256, 0, s>>>(topk, pos, keep, offsets, A, c.k, c.E, src_rows);
     return cudaGetLastError();
 }
 

@@ -210,6 +210,34 @@ def moe_dispatch(cfg: MoeConfig, x, topk, pos, keep, offsets, x_perm=None):
     return x_perm
 
 
+def moe_dispatch_rows(cfg: MoeConfig, topk, pos, keep, offsets, src_rows=None):
+    """The dispatch as a row table: src_rows[r] = token whose row goes to
+    permuted row r (0 for padding rows), for moe_expert_ffn_gather."""
+    if src_rows is None:
+        src_rows = torch.empty((moe_perm_rows(cfg),), dtype=torch.int32, device=_dev(offsets))
+    check(lib().moe_dispatch_rows(ctypes.byref(cfg), _p(topk), _p(pos), _p(keep), _p(offsets),
+                                  _p(src_rows), _stream()), "moe_dispatch_rows")
+    return src_rows
+
+
+def moe_expert_ffn_gather(cfg: MoeConfig, x, src_rows, offsets, W1, W3, W2, Ws1=None, Ws3=None,
+                          Ws2=None, ws=None, Y_perm=None, Y_shared=None):
+    """moe_expert_ffn with the dispatch fused in: routed rows read from x
+    through src_rows."""
+    dev = _dev(x)
+    if Y_perm is None:
+        Y_perm = torch.empty((moe_perm_rows(cfg), cfg.d), dtype=_tdtype(cfg), device=dev)
+    if cfg.n_shared > 0 and Y_shared is None:
+        Y_shared = torch.empty((cfg.T, cfg.d), dtype=_tdtype(cfg), device=dev)
+    if ws is None:
+        ws = workspace(moe_stage_workspace_size(cfg), dev)
+    check(lib().moe_expert_ffn_gather(ctypes.byref(cfg), _p(x), _p(src_rows), _p(offsets),
+                                      _p(W1), _p(W3), _p(W2), _p(Ws1), _p(Ws3), _p(Ws2),
+                                      _p(Y_perm), _p(Y_shared), _p(ws), ws.numel(), _stream()),
+          "moe_expert_ffn_gather")
+    return Y_perm, Y_shared, ws
+
+
 def moe_expert_ffn(cfg: MoeConfig, x_perm, offsets, W1, W3, W2, x=None, Ws1=None, Ws3=None,
                    Ws2=None, ws=None, Y_perm=None, Y_shared=None):
     dev = _dev(x_perm)
@@ -379,7 +407,7 @@ __all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
            "moe_combine", "moe_losses", "moe_device_status", "weights_struct", "MoEForward",
            "HostStream", "moe_forward", "CapacityOut", "StagedForward", "moe_capacity_scored",
            "moe_seq_balance_loss", "moe_bias_update", "moe_clear_device_status",
-           "moe_probe_wait_timeout"]
+           "moe_probe_wait_timeout", "moe_dispatch_rows", "moe_expert_ffn_gather"]
 
 
 class StagedForward:

@@ -56,6 +56,9 @@ def test_layer_work_counts_only_algorithmic_flops():
     # three matrices of d x d_ff per kept assignment, 2 FLOP per multiply-add
     assert w["expert_ffn"]["flops"] == 2.0 * 3 * (2 * s.T) * s.d * s.d_ff
     assert w["dispatch"]["bytes"] == s.T * s.d * 2 + 2 * s.T * s.d * 2 + s.T * s.k * 9
+    # the fused alternative moves a row table instead
+    assert w["dispatch_rows"]["bytes"] == bench.perm_rows(s) * 4 + s.T * s.k * 9 + 2 * s.T * 4
+    assert bench.perm_rows(s) == (2 * s.T + 127 * s.E + 127) // 128 * 128
     ds = CONFIGS["deepseekmoe"]
     wd = bench.layer_work(ds, None, kept_total=ds.T * ds.k, dropped_tokens=0)
     shared = 2.0 * 3 * ds.n_shared * ds.T * ds.d * ds.d_ff_shared

@@ -247,3 +247,55 @@ def test_a_wait_that_runs_out_sets_the_status_and_leaves_the_context_usable():
     Y, _, _ = moe.moe_expert_ffn(cfg, x_perm, off, W, W, W, ws=ws)   # clears the word
     assert moe.moe_device_status(ws) == 0
     _close_bf16(Y[:128], _ffn_ref(x_perm[:128], W[0], W[0], W[0], 1))
+
+
+@pytest.mark.parametrize("case", [
+    # T, d, E, k, F, act, S, dtype (pair tiles when T k >= 512 E)
+    (2048, 256, 8, 2, 384, 1, 0, 1),     # SM-pair tiles, SwiGLU
+    (2048, 192, 4, 2, 256, 0, 1, 1),     # SM-pair tiles, GELU, shared expert
+    (333, 128, 16, 3, 128, 1, 2, 1),     # single-SM tiles, shared experts
+    (97, 32, 4, 2, 64, 0, 1, 0),         # fp32 SIMT
+], ids=["pair_swiglu", "pair_gelu_shared", "1sm_shared", "fp32"])
+def test_gathered_expert_ffn_equals_dispatch_then_ffn(case):
+    """The dispatch fused into GEMM1 (rows gathered from x through the row
+    table) gives exactly the result of the permuted copy followed by the GEMM,
+    on every kept row; the row table matches one built on the host."""
+    T, d, E, k, F, act, S, dt = case
+    cfg = moe.moe_config(T=T, d=d, E=E, k=k, d_ff=F, act=act, dtype=dt, cf=1.0, n_shared=S,
+                         d_ff_shared=128 if S else 0)
+    tdt = torch.bfloat16 if dt == 1 else torch.float32
+    g = torch.Generator(device=DEV).manual_seed(T + E)
+    rnd = lambda *s, sc=1.0: (torch.randn(s, generator=g, device=DEV) * sc).to(tdt)
+    x = rnd(T, d)
+    W1, W2 = rnd(E, F, d, sc=d ** -0.5), rnd(E, d, F, sc=F ** -0.5)
+    W3 = rnd(E, F, d, sc=d ** -0.5) if act == 1 else None
+    Ws1 = rnd(S, 128, d, sc=d ** -0.5) if S else None
+    Ws3 = rnd(S, 128, d, sc=d ** -0.5) if S and act == 1 else None
+    Ws2 = rnd(S, d, 128, sc=128 ** -0.5) if S else None
+    # skewed random top-k so that some assignments are dropped (cf = 1)
+    pick = torch.rand((T, E), generator=g, device=DEV) + torch.linspace(0.5, 0, E, device=DEV)
+    topk = pick.argsort(dim=1, descending=True)[:, :k].to(torch.int32).contiguous()
+    cap = moe.moe_capacity(cfg, topk)
+    x_perm = moe.moe_dispatch(cfg, x, topk, cap.pos, cap.keep, cap.offsets)
+    Y_ref, Ysh_ref, ws1 = moe.moe_expert_ffn(cfg, x_perm, cap.offsets, W1, W3, W2, x, Ws1, Ws3,
+                                             Ws2)
+    rows = moe.moe_dispatch_rows(cfg, topk, cap.pos, cap.keep, cap.offsets)
+    Y, Ysh, ws2 = moe.moe_expert_ffn_gather(cfg, x, rows, cap.offsets, W1, W3, W2, Ws1, Ws3, Ws2)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status(ws1) == 0 and moe.moe_device_status(ws2) == 0
+    tk, pos, keep = topk.cpu().numpy(), cap.pos.cpu().numpy(), cap.keep.cpu().numpy()
+    off = cap.offsets.cpu().numpy()
+    assert keep.sum() < T * k   # something was dropped
+    want = np.zeros(moe.moe_perm_rows(cfg), np.int32)
+    kept_rows = []
+    for t in range(T):
+        for j in range(k):
+            if keep[t, j]:
+                r = off[tk[t, j]] + pos[t, j]
+                want[r] = t
+                kept_rows.append(r)
+    np.testing.assert_array_equal(rows.cpu().numpy(), want)
+    kr = torch.as_tensor(kept_rows, device=DEV, dtype=torch.long)
+    assert torch.equal(Y[kr], Y_ref[kr])
+    if S:
+        assert torch.equal(Ysh, Ysh_ref)
