@@ -58,7 +58,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture (profiles/gemm_2sm_mixtral.md), valid only for the GEMM source it was taken on.
 GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_54_b200", "csrc", "ffn_tcgen05.cu")
 MEASURED_TRAFFIC = {
-    ("mixtral", "08ae4c3a6308cecf9ae9b989daf9ff4b24a9fde50c41e13a8b341ad90fc61747"): 4.975e9,
+    ("mixtral", "872c0a36b644350c28d3aa0b8c0abd44d4e57e623453bff990cab6d72699abde"): 4.964e9,
 }
 
 
