@@ -290,67 +290,98 @@ struct SelectArgs {
     int T, E, k, score, renorm;
 };
 
+// fp32 -> unsigned integer of the same order (-0 made +0; keys are never NaN),
+// and back: lets a warp take a max with one redux.sync instead of a shuffle
+// tree.
+__device__ __forceinline__ uint32_t ord_key(float f)
+{
+    const uint32_t u = __float_as_uint(f + 0.f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unord_key(uint32_t u)
+{
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// The token's logits: the K parts summed in order, plus the logit bias.
+template <int PL>
+__device__ __forceinline__ void load_logits(const SelectArgs &a, int t, int lane, float *z)
+{
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+        const int e = lane + 32 * i;
+        z[i] = -INFINITY;
+        if (t < a.T && e < a.E) {
+            float s = 0.f;
+            for (int q = 0; q < a.parts; ++q)
+                s += a.partial[((int64_t)q * a.T + t) * a.E_pad + e];
+            if (a.logit_bias)
+                s += a.logit_bias[e];
+            z[i] = s;
+        }
+    }
+}
+
 // One block = 32 tokens = one row of the loss partials; each of the 8 warps
-// takes 4 consecutive tokens, one token at a time, and the warps' sums meet in
-// shared memory in a fixed order.
+// takes 4 consecutive tokens, one at a time (the next token's logits load
+// while the current one is processed), and the warps' sums meet in shared
+// memory in a fixed order.  Lane l holds experts l, l + 32, ... (PL of them).
+// Each top-k round is two integer warp reductions: the largest key, then the
+// lowest expert index holding it (ties go to the lower index).
+template <int PL>
 __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
 {
     constexpr int PER_WARP = kPartialTokens / 8;
     __shared__ float pw[8][kMaxE + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = a.E;
-    const int per_lane = (E + 31) / 32;   // <= 8
     const bool renorm = a.renorm < 0 ? (a.k > 1) : (a.renorm != 0);
-    float pacc[8];
+    const int t0 = blockIdx.x * kPartialTokens + warp * PER_WARP;
+    float pacc[PL];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < PL; ++i)
         pacc[i] = 0.f;
     float zacc = 0.f;
+    float z[PL];
+    load_logits<PL>(a, t0, lane, z);
     for (int tt = 0; tt < PER_WARP; ++tt) {
-        const int t = blockIdx.x * kPartialTokens + warp * PER_WARP + tt;
+        const int t = t0 + tt;
         if (t >= a.T)
             break;
-        float z[8], v[8], key[8];
-        float m = -INFINITY;
+        float zn[PL];
+        load_logits<PL>(a, t + 1 < t0 + PER_WARP ? t + 1 : a.T, lane, zn);
+        uint32_t mo = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane + 32 * i;
-            z[i] = -INFINITY;
-            if (i < per_lane && e < E) {
-                float s = 0.f;
-                for (int q = 0; q < a.parts; ++q)
-                    s += a.partial[((int64_t)q * a.T + t) * a.E_pad + e];
-                if (a.logit_bias)
-                    s += a.logit_bias[e];
-                z[i] = s;
-            }
-            m = fmaxf(m, z[i]);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        for (int i = 0; i < PL; ++i)
+            if (lane + 32 * i < E)
+                mo = max(mo, ord_key(z[i]));
+        const float m = unord_key(__reduce_max_sync(0xffffffffu, mo));
         float sum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i < per_lane && lane + 32 * i < E)
+        for (int i = 0; i < PL; ++i)
+            if (lane + 32 * i < E)
                 sum += expf(z[i] - m);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             sum += __shfl_xor_sync(0xffffffffu, sum, o);
         const float lse = m + logf(sum);
+        float v[PL];
+        uint32_t okey[PL];   // 0: not an expert of this layer
         float ssum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < PL; ++i) {
             const int e = lane + 32 * i;
-            const bool okk = i < per_lane && e < E;
+            const bool okk = e < E;
+            float key;
             if (a.score == MOE_SCORE_SOFTMAX) {
                 v[i] = okk ? expf(z[i] - m) / sum : 0.f;
-                key[i] = okk ? z[i] : -INFINITY;
+                key = z[i];
             } else {
                 v[i] = okk ? 1.f / (1.f + expf(-z[i])) : 0.f;
-                key[i] = okk ? v[i] + (a.select_bias ? a.select_bias[e] : 0.f) : -INFINITY;
+                key = v[i] + (a.select_bias && okk ? a.select_bias[e] : 0.f);
                 ssum += v[i];
             }
+            okey[i] = okk ? ord_key(key) : 0u;
             if (okk && a.logits_out)
                 a.logits_out[(int64_t)t * E + e] = z[i];
             if (okk && a.scores_out)
@@ -361,7 +392,6 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
             for (int o = 16; o > 0; o >>= 1)
                 ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
         }
-        unsigned taken = 0;
         int sel_idx[kMaxK];
         float sel_v[kMaxK];
         float sel_sum = 0.f;
@@ -371,31 +401,31 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
             sel_v[j] = 0.f;
             if (j >= a.k)
                 continue;
-            float bk = -INFINITY, bv = 0.f;
-            int bi = 0x7fffffff;
+            uint32_t lk = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                if (i < per_lane && e < E && !((taken >> i) & 1u) && better(key[i], e, bk, bi)) {
-                    bk = key[i];
-                    bi = e;
-                    bv = v[i];
-                }
-            }
+            for (int i = 0; i < PL; ++i)
+                lk = max(lk, okey[i]);
+            const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
+            uint32_t li = 0xffffffffu;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ok2 = __shfl_xor_sync(0xffffffffu, bk, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                if (better(ok2, oi, bk, bi)) {
-                    bk = ok2;
-                    bi = oi;
-                    bv = ov;
-                }
+            for (int i = PL - 1; i >= 0; --i)
+                if (okey[i] == mk && mk != 0u)
+                    li = (uint32_t)(lane + 32 * i);
+            const uint32_t bi = __reduce_min_sync(0xffffffffu, li);
+            const int slot = (int)(bi >> 5);
+            float mine = v[0];
+#pragma unroll
+            for (int i = 1; i < PL; ++i)
+                if (slot == i)
+                    mine = v[i];
+            const float bv = __shfl_sync(0xffffffffu, mine, (int)(bi & 31u));
+            if ((int)(bi & 31u) == lane) {
+#pragma unroll
+                for (int i = 0; i < PL; ++i)
+                    if (slot == i)
+                        okey[i] = 0u;   // taken
             }
-            if ((bi & 31) == lane)
-                taken |= 1u << (bi >> 5);
-            sel_idx[j] = bi;
+            sel_idx[j] = (int)bi;
             sel_v[j] = bv;
             sel_sum += bv;
         }
@@ -409,13 +439,16 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
             zacc += lse * lse;
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i < per_lane && lane + 32 * i < E)
+        for (int i = 0; i < PL; ++i)
+            if (lane + 32 * i < E)
                 pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[i] : v[i] / ssum;
+#pragma unroll
+        for (int i = 0; i < PL; ++i)
+            z[i] = zn[i];
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (i < per_lane && lane + 32 * i < E)
+    for (int i = 0; i < PL; ++i)
+        if (lane + 32 * i < E)
             pw[warp][lane + 32 * i] = pacc[i];
     if (lane == 0)
         pw[warp][E] = zacc;
@@ -593,8 +626,14 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
         select_small_kernel<4><<<rows, 4 * 32, 0, s>>>(a);
     else if (c.E <= 8)
         select_small_kernel<8><<<rows, 8 * 32, 0, s>>>(a);
+    else if (c.E <= 32)
+        select_kernel<1><<<rows, 256, 0, s>>>(a);
+    else if (c.E <= 64)
+        select_kernel<2><<<rows, 256, 0, s>>>(a);
+    else if (c.E <= 128)
+        select_kernel<4><<<rows, 256, 0, s>>>(a);
     else
-        select_kernel<<<rows, 256, 0, s>>>(a);
+        select_kernel<8><<<rows, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

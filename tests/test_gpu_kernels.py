@@ -299,3 +299,34 @@ def test_gathered_expert_ffn_equals_dispatch_then_ffn(case):
     assert torch.equal(Y[kr], Y_ref[kr])
     if S:
         assert torch.equal(Ysh, Ysh_ref)
+
+
+@pytest.mark.parametrize("E,k", [(9, 2), (16, 4), (32, 8), (33, 3), (64, 6), (96, 8), (128, 1),
+                                 (129, 5), (200, 8), (256, 8)])
+@pytest.mark.parametrize("score", [0, 1], ids=["softmax", "sigmoid"])
+def test_route_selection_every_width(E, k, score):
+    """The selection kernel at every lane width (1, 2, 4 or 8 experts per
+    lane), ragged expert counts included: top-k of the kernel's own fp32 keys
+    with ties to the lower index, gates, and the loss partials."""
+    T, d = 1000, 256
+    g = torch.Generator(device=DEV).manual_seed(E * 10 + k + score)
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    W_r = torch.randn((d, E), generator=g, device=DEV) * 0.05
+    sb = ((torch.rand(E, generator=g, device=DEV) - 0.5) * 0.2) if score == 1 else None
+    cfg = moe.moe_config(T=T, d=d, E=E, k=k, d_ff=64, dtype=1, cf=1.0, score=score)
+    topk, gates, part, logits, scores = moe.moe_route(cfg, x, W_r, None, sb, want_logits=True,
+                                                      want_scores=True)
+    torch.cuda.synchronize()
+    key = logits if score == 0 else scores + sb   # fp32, as the kernel ranks
+    ref = np.argsort(-key.double().cpu().numpy(), axis=1, kind="stable")[:, :k]
+    np.testing.assert_array_equal(topk.cpu().numpy(), ref)
+    sel = torch.gather(scores.double(), 1, topk.long())
+    want = sel / sel.sum(1, keepdim=True) if k > 1 else sel
+    assert (gates.double() - want).abs().max().item() < 1e-6
+    # loss partials: the probability mass per expert and lse^2, summed over the batch
+    rows = part.view(-1, E + 1).double()
+    p = scores.double() if score == 0 else scores.double() / scores.double().sum(1, keepdim=True)
+    np.testing.assert_allclose(rows[:, :E].sum(0).cpu().numpy(), p.sum(0).cpu().numpy(),
+                               rtol=1e-5, atol=1e-4)
+    lse = torch.logsumexp(logits.double(), dim=1)
+    assert rows[:, E].sum().item() == pytest.approx((lse ** 2).sum().item(), rel=1e-5)
