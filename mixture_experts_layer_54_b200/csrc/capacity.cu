@@ -13,9 +13,10 @@
 //   scan   - one block turns the histograms into, for every block, the number
 //            of assignments to each expert that come before the block in
 //            priority order, plus counts, kept, offsets and the drop total;
-//   place  - each block walks its own assignments in priority order, 256 at a
-//            time, ranking equal experts inside a warp with __match_any_sync
-//            and across warps through a per-warp count table.
+//   place  - each warp of a block walks its 32 tokens' assignments in
+//            priority order, 32 at a time, ranking equal experts with
+//            __match_any_sync; one scan over the block's warps gives each
+//            warp's start per expert.
 // Integers only, so the result is bit-exact with the sequential walk.
 //
 // Batch-prioritized order ("Lab 18" section 3, V-MoE: assignments ranked by
@@ -64,17 +65,25 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
                 int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
                 int32_t *__restrict__ n_dropped)
 {
+    constexpr int BATCH = 32;   // blocks' histogram entries in flight per column
     __shared__ int32_t total[kMaxK * kMaxE];   // per (j, e), all blocks
     __shared__ int32_t cnt[kMaxE];
+    __shared__ long long drop_w[32];
     const int cols = k * E;
-    // exclusive scan over blocks of each (j, e) column
+    // exclusive scan over blocks of each (j, e) column, BATCH loads at a time
     for (int col = threadIdx.x; col < cols; col += blockDim.x) {
         int run = 0;
-#pragma unroll 8
-        for (int b = 0; b < nblk; ++b) {
-            int v = hist[(int64_t)b * cols + col];
-            base[(int64_t)b * cols + col] = run;
-            run += v;
+        for (int b0 = 0; b0 < nblk; b0 += BATCH) {
+            int v[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i)
+                v[i] = b0 + i < nblk ? hist[(int64_t)(b0 + i) * cols + col] : 0;
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                if (b0 + i < nblk)
+                    base[(int64_t)(b0 + i) * cols + col] = run;
+                run += v[i];
+            }
         }
         total[col] = run;
     }
@@ -89,12 +98,18 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
     }
     __syncthreads();
     if (priority == MOE_PRIORITY_TOKEN) {
-        // assignments to e in earlier blocks, any rank: stored in the j = 0 slot
+        // assignments to e in earlier blocks, any rank: stored in the j = 0
+        // slot (every slot of the item read before it is written)
         for (int i = threadIdx.x; i < nblk * E; i += blockDim.x) {
-            int b = i / E, e = i % E;
+            const int b = i / E, e = i % E;
+            int v[kMaxK];
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j)
+                v[j] = j < k ? base[(int64_t)b * cols + j * E + e] : 0;
             int s = 0;
-            for (int j = 0; j < k; ++j)
-                s += base[(int64_t)b * cols + j * E + e];
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j)
+                s += v[j];
             base[(int64_t)b * cols + e] = s;
         }
     } else {
@@ -108,98 +123,136 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
             base[i] += s;
         }
     }
-    if (threadIdx.x == 0) {
-        int off = 0;
+    // segment offsets: kept counts rounded up to MOE_ROW_ALIGN, exclusive scan
+    // by one warp; the drop total summed in a fixed order
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int carry = 0;
         long long drop = 0;
-        for (int e = 0; e < E; ++e) {
-            offsets[e] = off;
-            int kv = (long long)cnt[e] < C ? cnt[e] : (int)C;
-            drop += cnt[e] - kv;
-            off += (kv + MOE_ROW_ALIGN - 1) / MOE_ROW_ALIGN * MOE_ROW_ALIGN;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            int padded = 0;
+            if (e < E) {
+                const int kv = (long long)cnt[e] < C ? cnt[e] : (int)C;
+                drop += cnt[e] - kv;
+                padded = (kv + MOE_ROW_ALIGN - 1) / MOE_ROW_ALIGN * MOE_ROW_ALIGN;
+            }
+            int incl = padded;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += n;
+            }
+            if (e < E)
+                offsets[e] = carry + incl - padded;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        offsets[E] = off;
-        *n_dropped = (int32_t)drop;
+        drop_w[lane] = drop;
+        __syncwarp();
+        if (lane == 0) {
+            long long d = 0;
+            for (int l = 0; l < 32; ++l)
+                d += drop_w[l];
+            offsets[E] = carry;
+            *n_dropped = (int32_t)d;
+        }
     }
 }
 
+// Each warp owns 32 consecutive tokens of the block.  Per pass (token order:
+// one pass over all slots; rank-major: one pass per slot j): (A) the warp
+// counts its assignments per expert; (B) one exclusive scan over the warps
+// turns the counts into each warp's start inside the block; (C) the warp walks
+// its assignments in priority order, 32 at a time, ranking equal experts with
+// __match_any_sync and keeping its own running count per expert.
 __global__ void __launch_bounds__(CT)
 cap_place_kernel(const int32_t *topk, int T, int k, int E, int priority, long long C,
                  const int32_t *base, int32_t *pos, uint8_t *keep, uint8_t *dropped)
 {
-    __shared__ int32_t run[kMaxE];
-    __shared__ int32_t wcnt[CT / 32][kMaxE];
+    __shared__ int32_t wrun[CT / 32][kMaxE];
     __shared__ uint8_t keep_s[CT * kMaxK];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t0 = blockIdx.x * CT;
-    const int ntok = min(CT, T - t0);
     const int cols = k * E;
     const int32_t *bb = base + (int64_t)blockIdx.x * cols;
-    for (int i = tid; i < (CT / 32) * kMaxE; i += CT)
-        (&wcnt[0][0])[i] = 0;
     const unsigned lt_mask = (1u << lane) - 1u;
-
-    // one pass = a sequence of `len` assignments, element n -> (t_local, j)
-    const int passes = priority == MOE_PRIORITY_TOKEN ? 1 : k;
+    const int tw = blockIdx.x * CT + warp * 32;   // this warp's first token
+    const int nw = max(0, min(32, T - tw));       // its tokens
+    const bool token_order = priority == MOE_PRIORITY_TOKEN;
+    const int passes = token_order ? 1 : k;
     for (int p = 0; p < passes; ++p) {
-        for (int e = tid; e < E; e += CT)
-            run[e] = 0;
-        __syncthreads();
-        const int len = priority == MOE_PRIORITY_TOKEN ? ntok * k : ntok;
-        for (int c0 = 0; c0 < len; c0 += CT) {
-            const int n = c0 + tid;
-            const bool valid = n < len;
-            int tl = 0, j = 0, e = E;   // E = sentinel for idle lanes
-            if (valid) {
-                if (priority == MOE_PRIORITY_TOKEN) {
-                    tl = n / k;
-                    j = n % k;
-                } else {
-                    tl = n;
-                    j = p;
-                }
-                e = topk[(int64_t)(t0 + tl) * k + j];
+        const int len = token_order ? nw * k : nw;
+        // (A) this warp's assignments per expert
+        for (int i = lane; i < E; i += 32)
+            wrun[warp][i] = 0;
+        __syncwarp();
+        for (int c0 = 0; c0 < len; c0 += 32) {
+            const int n = c0 + lane;
+            int e = E;   // sentinel for idle lanes and invalid experts
+            if (n < len) {
+                const int tl = token_order ? n / k : n, j = token_order ? n % k : p;
+                e = topk[(int64_t)(tw + tl) * k + j];
                 if (e < 0 || e >= E)
                     e = E;
             }
             const unsigned peers = __match_any_sync(0xffffffffu, e);
-            const int inwarp = __popc(peers & lt_mask);
-            const bool leader = (peers & lt_mask) == 0;
-            if (leader && e < E)
-                wcnt[warp][e] = __popc(peers);
-            __syncthreads();
-            if (valid) {
-                if (e < E) {
-                    int prior = 0;
-                    for (int w = 0; w < warp; ++w)
-                        prior += wcnt[w][e];
-                    const int boff = priority == MOE_PRIORITY_TOKEN ? e : j * E + e;
-                    const long long position = (long long)bb[boff] + run[e] + prior + inwarp;
-                    pos[(int64_t)(t0 + tl) * k + j] = (int32_t)position;
-                    keep_s[tl * k + j] = position < C ? 1 : 0;
-                } else {
-                    pos[(int64_t)(t0 + tl) * k + j] = -1;
-                    keep_s[tl * k + j] = 0;
-                }
-            }
-            __syncthreads();
-            for (int ee = tid; ee < E; ee += CT) {
-                int s = 0;
-                for (int w = 0; w < CT / 32; ++w) {
-                    s += wcnt[w][ee];
-                    wcnt[w][ee] = 0;
-                }
-                run[ee] += s;
-            }
-            __syncthreads();
+            if ((peers & lt_mask) == 0 && e < E)
+                wrun[warp][e] += __popc(peers);
+            __syncwarp();
         }
+        __syncthreads();
+        // (B) earlier warps' assignments to each expert
+        for (int e = tid; e < E; e += CT) {
+            int run = 0;
+#pragma unroll
+            for (int w = 0; w < CT / 32; ++w) {
+                const int v = wrun[w][e];
+                wrun[w][e] = run;
+                run += v;
+            }
+        }
+        __syncthreads();
+        // (C) positions, in priority order
+        for (int c0 = 0; c0 < len; c0 += 32) {
+            const int n = c0 + lane;
+            int e = E, tl = 0, j = 0;
+            if (n < len) {
+                tl = token_order ? n / k : n;
+                j = token_order ? n % k : p;
+                e = topk[(int64_t)(tw + tl) * k + j];
+                if (e < 0 || e >= E)
+                    e = E;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            if (n < len) {
+                const int64_t a = (int64_t)(tw + tl) * k + j;
+                uint8_t kv = 0;
+                if (e < E) {
+                    const int boff = token_order ? e : j * E + e;
+                    const long long position =
+                        (long long)bb[boff] + wrun[warp][e] + __popc(peers & lt_mask);
+                    pos[a] = (int32_t)position;
+                    kv = position < C ? 1 : 0;
+                } else {
+                    pos[a] = -1;
+                }
+                keep_s[(warp * 32 + tl) * k + j] = kv;
+            }
+            __syncwarp();
+            if ((peers & lt_mask) == 0 && e < E)
+                wrun[warp][e] += __popc(peers);
+            __syncwarp();
+        }
+        __syncthreads();   // every warp done with the tables before the next pass
     }
-    if (tid < ntok) {
+    if (lane < nw) {
         int any = 0;
         for (int j = 0; j < k; ++j) {
-            any |= keep_s[tid * k + j];
-            keep[(int64_t)(t0 + tid) * k + j] = keep_s[tid * k + j];
+            const uint8_t kv = keep_s[(warp * 32 + lane) * k + j];
+            any |= kv;
+            keep[(int64_t)(tw + lane) * k + j] = kv;
         }
-        dropped[t0 + tid] = any ? 0 : 1;
+        dropped[tw + lane] = any ? 0 : 1;
     }
 }
 
