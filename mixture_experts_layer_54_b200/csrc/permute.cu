@@ -138,49 +138,55 @@ template <> struct Vec<float> {
     }
 };
 
-template <typename Elem>
+// KS = the layer's k (slots per token).  A chunk of U vectors per lane is
+// loaded for every slot before any arithmetic (U * KS >= 8 loads in flight,
+// at least two per slot), then summed in fp32 in slot order, then the shared
+// experts and the residual.
+template <typename Elem, int KS>
 __global__ void __launch_bounds__(THREADS)
 combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y_sh,
                    const float *__restrict__ gates, const int32_t *__restrict__ topk,
                    const int32_t *__restrict__ pos, const uint8_t *__restrict__ keep,
                    const int32_t *__restrict__ offsets, const uint4 *__restrict__ residual,
-                   uint4 *__restrict__ y, int T, int k, int E, int nvec)
+                   uint4 *__restrict__ y, int T, int E, int nvec)
 {
     constexpr int N = Vec<Elem>::N;
+    constexpr int U = KS >= 4 ? 2 : 8 / KS;
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
     for (int t = gw; t < T; t += gridDim.x * WARPS) {
         int64_t rows[kMaxK];
-        slot_rows(t, k, E, topk, pos, keep, offsets, lane, rows);
-        const float mg = lane < k ? gates[(int64_t)t * k + lane] : 0.f;
-        float g[kMaxK];
+        slot_rows(t, KS, E, topk, pos, keep, offsets, lane, rows);
+        const float mg = lane < KS ? gates[(int64_t)t * KS + lane] : 0.f;
+        float g[KS];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
+        for (int j = 0; j < KS; ++j)
             g[j] = __shfl_sync(0xffffffffu, mg, j);
-        for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
-            float acc[UNROLL][N];
+        for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
+            uint4 raw[KS][U];
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u)
+            for (int j = 0; j < KS; ++j)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    raw[j][u] = (rows[j] >= 0 && v < nvec) ? __ldcs(Y_perm + rows[j] * nvec + v)
+                                                           : make_uint4(0u, 0u, 0u, 0u);
+                }
+            float acc[U][N];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int i = 0; i < N; ++i)
                     acc[u][i] = 0.f;
             // slots in order, then the shared experts, then the residual
 #pragma unroll
-            for (int j = 0; j < kMaxK; ++j) {
-                if (j >= k || rows[j] < 0)
+            for (int j = 0; j < KS; ++j) {
+                if (rows[j] < 0)
                     continue;
-                const uint4 *src = Y_perm + rows[j] * nvec;
-                uint4 raw[UNROLL];
 #pragma unroll
-                for (int u = 0; u < UNROLL; ++u) {
-                    const int v = v0 + u * 32 + lane;
-                    if (v < nvec)
-                        raw[u] = __ldcs(src + v);
-                }
-#pragma unroll
-                for (int u = 0; u < UNROLL; ++u) {
+                for (int u = 0; u < U; ++u) {
                     float f[N];
-                    Vec<Elem>::load(raw[u], f);
+                    Vec<Elem>::load(raw[j][u], f);
 #pragma unroll
                     for (int i = 0; i < N; ++i)
                         acc[u][i] = fmaf(g[j], f[i], acc[u][i]);
@@ -193,7 +199,7 @@ combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y
                 if (!extra[q])
                     continue;
 #pragma unroll
-                for (int u = 0; u < UNROLL; ++u) {
+                for (int u = 0; u < U; ++u) {
                     const int v = v0 + u * 32 + lane;
                     if (v < nvec) {
                         float f[N];
@@ -205,7 +211,7 @@ combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y
                 }
             }
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int v = v0 + u * 32 + lane;
                 if (v < nvec)
                     y[(int64_t)t * nvec + v] = Vec<Elem>::store(acc[u]);
@@ -269,12 +275,25 @@ cudaError_t launch_combine(const moe_config &c, const void *Y_perm, const void *
         kern<<<grid_for(kern, c.T), THREADS, 0, s>>>(
             static_cast<const uint4 *>(Y_perm), static_cast<const uint4 *>(Y_sh), gates, topk,
             pos, keep, offsets, static_cast<const uint4 *>(residual), static_cast<uint4 *>(y),
-            c.T, c.k, c.E, nvec);
+            c.T, c.E, nvec);
+    };
+    auto by_k = [&](auto elem) {
+        using El = decltype(elem);
+        switch (c.k) {
+        case 1: args(combine_vec_kernel<El, 1>); break;
+        case 2: args(combine_vec_kernel<El, 2>); break;
+        case 3: args(combine_vec_kernel<El, 3>); break;
+        case 4: args(combine_vec_kernel<El, 4>); break;
+        case 5: args(combine_vec_kernel<El, 5>); break;
+        case 6: args(combine_vec_kernel<El, 6>); break;
+        case 7: args(combine_vec_kernel<El, 7>); break;
+        default: args(combine_vec_kernel<El, 8>); break;
+        }
     };
     if (c.dtype == MOE_DTYPE_BF16)
-        args(combine_vec_kernel<__nv_bfloat16>);
+        by_k(__nv_bfloat16());
     else
-        args(combine_vec_kernel<float>);
+        by_k(float());
     return cudaGetLastError();
 }
 
