@@ -1,5 +1,6 @@
 """Host-side logic of the benchmark on CPU: two gloo ranks agree on the slowest
-rank's time, and the workload accounting is what the design doc states."""
+rank's time, and the workload accounting counts only algorithmic bytes and
+FLOPs."""
 import math
 import os
 import socket
