@@ -322,17 +322,19 @@ __device__ __forceinline__ void load_logits(const SelectArgs &a, int t, int lane
     }
 }
 
-// One block = 32 tokens = one row of the loss partials; each of the 8 warps
-// takes 4 consecutive tokens, one at a time (the next token's logits load
-// while the current one is processed), and the warps' sums meet in shared
-// memory in a fixed order.  Lane l holds experts l, l + 32, ... (PL of them).
-// Each top-k round is two integer warp reductions: the largest key, then the
-// lowest expert index holding it (ties go to the lower index).
-template <int PL>
-__global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
+// One block = 32 tokens = one row of the loss partials; each of the W warps
+// takes 32 / W consecutive tokens, one at a time (the next token's logits
+// load while the current one is processed), and the warps' sums meet in
+// shared memory in a fixed order.  Lane l holds experts l, l + 32, ... (PL of
+// them).  Each top-k round is two integer warp reductions: the largest key,
+// then the lowest expert index holding it (ties go to the lower index).  W = 8
+// for up to 128 experts; W = 32 (one token per warp) for more, where the
+// per-token work is long and eight warps per block left the schedulers idle.
+template <int PL, int W>
+__global__ void __launch_bounds__(32 * W, 1) select_kernel(SelectArgs a)
 {
-    constexpr int PER_WARP = kPartialTokens / 8;
-    __shared__ float pw[8][kMaxE + 1];
+    constexpr int PER_WARP = kPartialTokens / W;
+    __shared__ float pw[W][kMaxE + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = a.E;
     const bool renorm = a.renorm < 0 ? (a.k > 1) : (a.renorm != 0);
@@ -349,7 +351,8 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
         if (t >= a.T)
             break;
         float zn[PL];
-        load_logits<PL>(a, t + 1 < t0 + PER_WARP ? t + 1 : a.T, lane, zn);
+        if (PER_WARP > 1)
+            load_logits<PL>(a, t + 1 < t0 + PER_WARP ? t + 1 : a.T, lane, zn);
         uint32_t mo = 0;
 #pragma unroll
         for (int i = 0; i < PL; ++i)
@@ -442,9 +445,11 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
         for (int i = 0; i < PL; ++i)
             if (lane + 32 * i < E)
                 pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[i] : v[i] / ssum;
+        if (PER_WARP > 1) {
 #pragma unroll
-        for (int i = 0; i < PL; ++i)
-            z[i] = zn[i];
+            for (int i = 0; i < PL; ++i)
+                z[i] = zn[i];
+        }
     }
 #pragma unroll
     for (int i = 0; i < PL; ++i)
@@ -454,9 +459,9 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a)
         pw[warp][E] = zacc;
     __syncthreads();
     float *out = a.loss_partials + (int64_t)blockIdx.x * (E + 1);
-    for (int e = threadIdx.x; e <= E; e += 256) {
+    for (int e = threadIdx.x; e <= E; e += 32 * W) {
         float acc = 0.f;
-        for (int w = 0; w < 8; ++w)
+        for (int w = 0; w < W; ++w)
             acc += pw[w][e];
         out[e] = acc;
     }
@@ -627,13 +632,13 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
     else if (c.E <= 8)
         select_small_kernel<8><<<rows, 8 * 32, 0, s>>>(a);
     else if (c.E <= 32)
-        select_kernel<1><<<rows, 256, 0, s>>>(a);
+        select_kernel<1, 8><<<rows, 256, 0, s>>>(a);
     else if (c.E <= 64)
-        select_kernel<2><<<rows, 256, 0, s>>>(a);
+        select_kernel<2, 8><<<rows, 256, 0, s>>>(a);
     else if (c.E <= 128)
-        select_kernel<4><<<rows, 256, 0, s>>>(a);
+        select_kernel<4, 8><<<rows, 256, 0, s>>>(a);
     else
-        select_kernel<8><<<rows, 256, 0, s>>>(a);
+        select_kernel<8, 32><<<rows, 1024, 0, s>>>(a);
     return cudaGetLastError();
 }
 
