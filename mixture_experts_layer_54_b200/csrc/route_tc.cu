@@ -322,37 +322,29 @@ __device__ __forceinline__ void load_logits(const SelectArgs &a, int t, int lane
     }
 }
 
-// One block = 32 tokens = one row of the loss partials; each of the W warps
-// takes 32 / W consecutive tokens, one at a time (the next token's logits
-// load while the current one is processed), and the warps' sums meet in
-// shared memory in a fixed order.  Lane l holds experts l, l + 32, ... (PL of
-// them).  Each top-k round is two integer warp reductions: the largest key,
-// then the lowest expert index holding it (ties go to the lower index).  W = 8
-// for up to 128 experts; W = 32 (one token per warp) for more, where the
-// per-token work is long and eight warps per block left the schedulers idle.
-template <int PL, int W>
-__global__ void __launch_bounds__(32 * W, 1) select_kernel(SelectArgs a)
+// One block = 32 tokens = one row of the loss partials, one warp per token
+// (with four tokens per warp in series, eight warps per block left the
+// schedulers half idle); the warps' sums meet in shared memory in warp order.
+// Lane l holds experts l, l + 32, ... (PL of them).  Each top-k round is two
+// integer warp reductions: the largest key, then the lowest expert index
+// holding it (ties go to the lower index).
+template <int PL>
+__global__ void __launch_bounds__(32 * kPartialTokens, 1) select_kernel(SelectArgs a)
 {
-    constexpr int PER_WARP = kPartialTokens / W;
+    constexpr int W = kPartialTokens;   // warps per block, one token each
     __shared__ float pw[W][kMaxE + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = a.E;
     const bool renorm = a.renorm < 0 ? (a.k > 1) : (a.renorm != 0);
-    const int t0 = blockIdx.x * kPartialTokens + warp * PER_WARP;
+    const int t = blockIdx.x * kPartialTokens + warp;
     float pacc[PL];
 #pragma unroll
     for (int i = 0; i < PL; ++i)
         pacc[i] = 0.f;
     float zacc = 0.f;
-    float z[PL];
-    load_logits<PL>(a, t0, lane, z);
-    for (int tt = 0; tt < PER_WARP; ++tt) {
-        const int t = t0 + tt;
-        if (t >= a.T)
-            break;
-        float zn[PL];
-        if (PER_WARP > 1)
-            load_logits<PL>(a, t + 1 < t0 + PER_WARP ? t + 1 : a.T, lane, zn);
+    if (t < a.T) {
+        float z[PL];
+        load_logits<PL>(a, t, lane, z);
         uint32_t mo = 0;
 #pragma unroll
         for (int i = 0; i < PL; ++i)
@@ -445,11 +437,6 @@ __global__ void __launch_bounds__(32 * W, 1) select_kernel(SelectArgs a)
         for (int i = 0; i < PL; ++i)
             if (lane + 32 * i < E)
                 pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[i] : v[i] / ssum;
-        if (PER_WARP > 1) {
-#pragma unroll
-            for (int i = 0; i < PL; ++i)
-                z[i] = zn[i];
-        }
     }
 #pragma unroll
     for (int i = 0; i < PL; ++i)
@@ -632,13 +619,13 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
     else if (c.E <= 8)
         select_small_kernel<8><<<rows, 8 * 32, 0, s>>>(a);
     else if (c.E <= 32)
-        select_kernel<1, 8><<<rows, 256, 0, s>>>(a);
+        select_kernel<1><<<rows, 32 * kPartialTokens, 0, s>>>(a);
     else if (c.E <= 64)
-        select_kernel<2, 8><<<rows, 256, 0, s>>>(a);
+        select_kernel<2><<<rows, 32 * kPartialTokens, 0, s>>>(a);
     else if (c.E <= 128)
-        select_kernel<4, 8><<<rows, 256, 0, s>>>(a);
+        select_kernel<4><<<rows, 32 * kPartialTokens, 0, s>>>(a);
     else
-        select_kernel<8, 32><<<rows, 1024, 0, s>>>(a);
+        select_kernel<8><<<rows, 32 * kPartialTokens, 0, s>>>(a);
     return cudaGetLastError();
 }
 
