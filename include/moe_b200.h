@@ -209,6 +209,33 @@ moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx,
                         moe_stream_t stream);
 
 /*
+ * moe_capacity_sharded - moe_capacity for one shard of a batch split across
+ * data-parallel ranks in token order (rank r holds the tokens after those of
+ * ranks 0..r-1), keeping the capacity of the whole batch ("Lab 18" section 3:
+ * C per expert per batch, first come first served in token order).
+ *   capacity: C of the whole batch (moe_capacity_value of its config).
+ *   shard_counts [n_shards][E] int32 in (device): every shard's assignments
+ *     per expert (moe_capacity's counts, all-gathered in rank order); this
+ *     shard is number `shard`.  The library sums the rows before it:
+ *     count_base[e] = sum_{r < shard} shard_counts[r][e].
+ *   cfg: this shard's shape; priority must be MOE_PRIORITY_TOKEN (else
+ *     MOE_ERR_DTYPE: the other orders are not a prefix over shards).
+ *   Outputs as for moe_capacity, for this shard: counts = its assignments per
+ *   expert; pos = place in this shard's segment of the expert; keep = 1 while
+ *   count_base[e] + pos < capacity; kept = min(counts, max(0, capacity -
+ *   count_base)); offsets, dropped and n_dropped follow.  With one shard and
+ *   capacity = moe_capacity_value(cfg) the results equal moe_capacity's.
+ *   Returns MOE_ERR_SHAPE for capacity < 0 or shard outside [0, n_shards).
+ */
+moe_status moe_capacity_sharded(const moe_config *cfg, int64_t capacity,
+                                const int32_t *shard_counts, int32_t n_shards,
+                                int32_t shard, const int32_t *topk_idx,
+                                int32_t *counts, int32_t *pos, uint8_t *keep,
+                                int32_t *kept, int32_t *offsets, uint8_t *dropped,
+                                int32_t *n_dropped, void *ws, size_t ws_bytes,
+                                moe_stream_t stream);
+
+/*
  * moe_capacity_scored - moe_capacity in batch-prioritized order ("Lab 18"
  * section 3: V-MoE ranks the assignments by router score).  The walk takes the
  * T*k assignments from the highest router score of the selected expert down;

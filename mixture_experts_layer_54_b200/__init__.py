@@ -8,7 +8,8 @@ from ._abi import (MOE_ROW_ALIGN, CapacityFactorError, MoEError, MoeConfig, MoeO
                    MoeWeights, LIB_PATH, lib)
 from .ops import (HostStream, MoEForward, moe_bias_update, moe_capacity, moe_capacity_scored,
                   moe_seq_balance_loss, moe_clear_device_status, moe_probe_wait_timeout,
-                  moe_dispatch_rows, moe_expert_ffn_gather, moe_capacity_noalloc, moe_capacity_value, moe_combine, moe_config,
+                  moe_dispatch_rows, moe_expert_ffn_gather, moe_capacity_sharded,
+                  gather_shard_counts, shard_losses, moe_capacity_noalloc, moe_capacity_value, moe_combine, moe_config,
                   moe_device_status, moe_dispatch, moe_expert_ffn, moe_forward,
                   moe_loss_partials_count, moe_losses, moe_perm_rows, moe_route,
                   moe_stage_workspace_size, moe_validate, moe_workspace_size, weights_struct,
@@ -18,7 +19,8 @@ from .ops import (HostStream, MoEForward, moe_bias_update, moe_capacity, moe_cap
 __all__ = ["MOE_ROW_ALIGN", "CapacityFactorError", "MoEError", "MoeConfig", "MoeOutputs",
            "MoeWeights", "LIB_PATH", "lib", "HostStream", "MoEForward", "moe_bias_update",
            "moe_capacity_scored", "moe_seq_balance_loss", "moe_clear_device_status",
-           "moe_probe_wait_timeout", "moe_dispatch_rows", "moe_expert_ffn_gather", "moe_capacity", "moe_capacity_noalloc", "moe_capacity_value",
+           "moe_probe_wait_timeout", "moe_dispatch_rows", "moe_expert_ffn_gather",
+           "moe_capacity_sharded", "gather_shard_counts", "shard_losses", "moe_capacity", "moe_capacity_noalloc", "moe_capacity_value",
            "moe_combine", "moe_config", "moe_device_status", "moe_dispatch", "moe_expert_ffn",
            "moe_forward", "moe_loss_partials_count", "moe_losses", "moe_perm_rows", "moe_route",
            "moe_stage_workspace_size", "moe_validate", "moe_workspace_size", "weights_struct",

@@ -58,6 +58,9 @@ SIGNATURES = {
     "moe_capacity_noalloc": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_capacity_scored": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.c_size_t, _P]),
+    "moe_capacity_sharded": (ctypes.c_int, [_CFG, ctypes.c_int64, _P, ctypes.c_int32,
+                                            ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P,
+                                            _P, ctypes.c_size_t, _P]),
     "moe_seq_balance_loss": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _P, _P, _P, _P]),
     "moe_bias_update": (ctypes.c_int, [_CFG, _P, ctypes.c_float, _P, _P]),
     "moe_dispatch": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),

@@ -83,6 +83,7 @@ void carve_stage_into(const moe_config &c, Carver &cv, StageScratch &s)
     s.route = route_cv.take(route_scratch_bytes(c));
     s.hist = static_cast<int32_t *>(cap_cv.take(hk));
     s.base = static_cast<int32_t *>(cap_cv.take(hk));
+    s.count_base = static_cast<int32_t *>(cap_cv.take((size_t)c.E * 4));
     s.keys = static_cast<unsigned long long *>(
         cap_cv.take(c.priority == MOE_PRIORITY_SCORE ? (size_t)c.T * c.k * 8 : 0));
     s.H = ffn_cv.take((size_t)R * c.d_ff * esz);
@@ -283,6 +284,36 @@ moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx, int32_t 
     return cuda_status(launch_capacity(*cfg, capacity_of(*cfg), topk_idx, counts, pos, keep, kept,
                                        offsets, dropped, n_dropped, s.hist, s.base,
                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_capacity_sharded(const moe_config *cfg, int64_t capacity,
+                                const int32_t *shard_counts, int32_t n_shards, int32_t shard,
+                                const int32_t *topk_idx,
+                                int32_t *counts, int32_t *pos, uint8_t *keep, int32_t *kept,
+                                int32_t *offsets, uint8_t *dropped, int32_t *n_dropped, void *ws,
+                                size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = check_cfg(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (cfg->priority != MOE_PRIORITY_TOKEN)
+        return MOE_ERR_DTYPE;   // across shards only the token order is a prefix sum
+    if (capacity < 0 || n_shards < 1 || shard < 0 || shard >= n_shards)
+        return MOE_ERR_SHAPE;
+    if (!shard_counts || !counts || !kept || !offsets || !n_dropped || !ws ||
+        (cfg->T > 0 && (!topk_idx || !pos || !keep || !dropped)))
+        return MOE_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return MOE_ERR_ALIGN;
+    if (ws_bytes < stage_scratch_bytes(*cfg))
+        return MOE_ERR_WORKSPACE;
+    StageScratch s = carve_stage(*cfg, ws);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_shard_base(*cfg, shard_counts, shard, s.count_base, cs);
+    if (e != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cuda_status(launch_capacity(*cfg, capacity, topk_idx, counts, pos, keep, kept, offsets,
+                                       dropped, n_dropped, s.hist, s.base, cs, s.count_base));
 }
 
 moe_status moe_capacity_scored(const moe_config *cfg, const int32_t *topk_idx,

@@ -61,13 +61,14 @@ __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int 
 
 __global__ void __launch_bounds__(1024)
 cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int priority,
-                long long C, int32_t *__restrict__ base, int32_t *__restrict__ counts,
-                int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
-                int32_t *__restrict__ n_dropped)
+                long long C, const int32_t *__restrict__ count_base, int32_t *__restrict__ base,
+                int32_t *__restrict__ counts, int32_t *__restrict__ kept,
+                int32_t *__restrict__ offsets, int32_t *__restrict__ n_dropped)
 {
     constexpr int BATCH = 32;   // blocks' histogram entries in flight per column
     __shared__ int32_t total[kMaxK * kMaxE];   // per (j, e), all blocks
     __shared__ int32_t cnt[kMaxE];
+    __shared__ int32_t kept_s[kMaxE];
     __shared__ long long drop_w[32];
     const int cols = k * E;
     // exclusive scan over blocks of each (j, e) column, BATCH loads at a time
@@ -92,9 +93,15 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
         int s = 0;
         for (int j = 0; j < k; ++j)
             s += total[j * E + e];
+        // slots left for this batch: C, less what earlier shards of the same
+        // global batch already took (count_base, sharded capacity only)
+        long long room = C - (count_base ? (long long)count_base[e] : 0LL);
+        room = room < 0 ? 0 : room;
+        const int32_t kv = (long long)s < room ? s : (int32_t)room;
         cnt[e] = s;
         counts[e] = s;
-        kept[e] = (long long)s < C ? s : (int32_t)C;
+        kept_s[e] = kv;
+        kept[e] = kv;
     }
     __syncthreads();
     if (priority == MOE_PRIORITY_TOKEN) {
@@ -133,7 +140,7 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
             const int e = e0 + lane;
             int padded = 0;
             if (e < E) {
-                const int kv = (long long)cnt[e] < C ? cnt[e] : (int)C;
+                const int kv = kept_s[e];
                 drop += cnt[e] - kv;
                 padded = (kv + MOE_ROW_ALIGN - 1) / MOE_ROW_ALIGN * MOE_ROW_ALIGN;
             }
@@ -168,7 +175,8 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
 // __match_any_sync and keeping its own running count per expert.
 __global__ void __launch_bounds__(CT)
 cap_place_kernel(const int32_t *topk, int T, int k, int E, int priority, long long C,
-                 const int32_t *base, int32_t *pos, uint8_t *keep, uint8_t *dropped)
+                 const int32_t *count_base, const int32_t *base, int32_t *pos, uint8_t *keep,
+                 uint8_t *dropped)
 {
     __shared__ int32_t wrun[CT / 32][kMaxE];
     __shared__ uint8_t keep_s[CT * kMaxK];
@@ -232,7 +240,8 @@ cap_place_kernel(const int32_t *topk, int T, int k, int E, int priority, long lo
                     const long long position =
                         (long long)bb[boff] + wrun[warp][e] + __popc(peers & lt_mask);
                     pos[a] = (int32_t)position;
-                    kv = position < C ? 1 : 0;
+                    // kept while the slot's place in the whole (global) batch is below C
+                    kv = position + (count_base ? count_base[e] : 0) < C ? 1 : 0;
                 } else {
                     pos[a] = -1;
                 }
@@ -378,10 +387,31 @@ cudaError_t launch_capacity_scored(const moe_config &c, int64_t C, const int32_t
     return cudaGetLastError();
 }
 
+// count_base[e] = sum over the shards before `shard` of their counts
+// (shard_counts [n_shards][E]), in shard order.
+__global__ void shard_base_kernel(const int32_t *__restrict__ shard_counts, int shard, int E,
+                                  int32_t *__restrict__ count_base)
+{
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int s = 0;
+        for (int r = 0; r < shard; ++r)
+            s += shard_counts[(int64_t)r * E + e];
+        count_base[e] = s;
+    }
+}
+
+cudaError_t launch_shard_base(const moe_config &c, const int32_t *shard_counts, int shard,
+                              int32_t *count_base, cudaStream_t s)
+{
+    shard_base_kernel<<<1, 256, 0, s>>>(shard_counts, shard, c.E, count_base);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep, int32_t *kept,
                             int32_t *offsets, uint8_t *dropped, int32_t *n_dropped,
-                            int32_t *hist, int32_t *base, cudaStream_t s)
+                            int32_t *hist, int32_t *base, cudaStream_t s,
+                            const int32_t *count_base)
 {
     const int nblk = cap_blocks(c);
     if (nblk > 0) {
@@ -390,13 +420,13 @@ cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
         if (err != cudaSuccess)
             return err;
     }
-    cap_scan_kernel<<<1, 1024, 0, s>>>(hist, nblk, c.k, c.E, c.priority, (long long)C, base,
-                                       counts, kept, offsets, n_dropped);
+    cap_scan_kernel<<<1, 1024, 0, s>>>(hist, nblk, c.k, c.E, c.priority, (long long)C, count_base,
+                                       base, counts, kept, offsets, n_dropped);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess || nblk == 0)
         return err;
-    cap_place_kernel<<<nblk, CT, 0, s>>>(topk, c.T, c.k, c.E, c.priority, (long long)C, base, pos,
-                                         keep, dropped);
+    cap_place_kernel<<<nblk, CT, 0, s>>>(topk, c.T, c.k, c.E, c.priority, (long long)C, count_base,
+                                         base, pos, keep, dropped);
     return cudaGetLastError();
 }
 

@@ -46,6 +46,7 @@ struct StageScratch {
     void *route;          // tensor-core router: split weights and partial logits
     int32_t *hist;        // [cap_blocks][k][E]
     int32_t *base;        // [cap_blocks][k][E]
+    int32_t *count_base;  // [E] sharded capacity: earlier shards' assignments
     unsigned long long *keys;   // [T k] batch-prioritized capacity: per-expert lists
     void *H;              // [perm_rows][F] dtype
     void *H_sh;           // [S][T][Fs] dtype
@@ -64,11 +65,16 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
                             float *gates, float *partials, float *logits_out, float *scores_out,
                             void *scratch, int32_t *status, cudaStream_t s);
 
+cudaError_t launch_shard_base(const moe_config &c, const int32_t *shard_counts, int shard,
+                              int32_t *count_base, cudaStream_t s);
+
+// count_base (nullable, [E]): assignments to each expert in earlier shards of
+// the same global batch (token order); C is then the global batch's capacity.
 cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep,
                             int32_t *kept, int32_t *offsets, uint8_t *dropped,
                             int32_t *n_dropped, int32_t *hist, int32_t *base,
-                            cudaStream_t s);
+                            cudaStream_t s, const int32_t *count_base = nullptr);
 
 cudaError_t launch_capacity_scored(const moe_config &c, int64_t C, const int32_t *topk,
                                    const float *scores, int32_t *counts, int32_t *pos,

@@ -159,6 +159,53 @@ def moe_capacity_scored(cfg: MoeConfig, topk, scores, ws=None) -> CapacityOut:
     return out
 
 
+def moe_capacity_sharded(cfg: MoeConfig, capacity: int, shard_counts, shard: int, topk,
+                         ws=None) -> CapacityOut:
+    """Capacity of one shard of a token-ordered batch split across ranks:
+    shard_counts [n_shards, E] int32 are every shard's per-expert counts (see
+    gather_shard_counts), `capacity` the whole batch's C."""
+    dev = _dev(topk)
+    T, k, E = cfg.T, cfg.k, cfg.E
+    out = CapacityOut(
+        counts=torch.empty((E,), dtype=torch.int32, device=dev),
+        pos=torch.empty((T, k), dtype=torch.int32, device=dev),
+        keep=torch.empty((T, k), dtype=torch.uint8, device=dev),
+        kept=torch.empty((E,), dtype=torch.int32, device=dev),
+        offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+        dropped=torch.empty((T,), dtype=torch.uint8, device=dev),
+        n_dropped=torch.empty((1,), dtype=torch.int32, device=dev))
+    if ws is None:
+        ws = workspace(moe_stage_workspace_size(cfg), dev)
+    check(lib().moe_capacity_sharded(ctypes.byref(cfg), int(capacity), _p(shard_counts),
+                                     int(shard_counts.shape[0]), int(shard), _p(topk),
+                                     _p(out.counts), _p(out.pos), _p(out.keep), _p(out.kept),
+                                     _p(out.offsets), _p(out.dropped), _p(out.n_dropped), _p(ws),
+                                     ws.numel(), _stream()), "moe_capacity_sharded")
+    return out
+
+
+def gather_shard_counts(counts, group=None):
+    """All-gather of every rank's per-expert counts [E] into [world, E], rank
+    order (the one exchange the token-order capacity needs across shards)."""
+    import torch.distributed as dist
+    parts = [torch.empty_like(counts) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, counts, group=group)
+    return torch.stack(parts)
+
+
+def shard_losses(cfg_global: MoeConfig, counts, loss_partials, group=None):
+    """Switch loss and z-loss of the whole batch from the shards' own counts and
+    loss partials: counts all-reduced (sum), partial rows all-gathered in rank
+    order (every shard's token count a multiple of 32, so the rows line up
+    with the whole batch's), then moe_losses on the whole batch's config."""
+    import torch.distributed as dist
+    total = counts.clone()
+    dist.all_reduce(total, group=group)
+    rows = [torch.empty_like(loss_partials) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(rows, loss_partials, group=group)
+    return moe_losses(cfg_global, total, torch.cat(rows))
+
+
 def moe_seq_balance_loss(cfg: MoeConfig, seq_len: int, topk, loss_partials, per_seq=None,
                          loss=None):
     """Sequence-wise balance loss over sequences of seq_len tokens; returns
@@ -407,7 +454,8 @@ __all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
            "moe_combine", "moe_losses", "moe_device_status", "weights_struct", "MoEForward",
            "HostStream", "moe_forward", "CapacityOut", "StagedForward", "moe_capacity_scored",
            "moe_seq_balance_loss", "moe_bias_update", "moe_clear_device_status",
-           "moe_probe_wait_timeout", "moe_dispatch_rows", "moe_expert_ffn_gather"]
+           "moe_probe_wait_timeout", "moe_dispatch_rows", "moe_expert_ffn_gather",
+           "moe_capacity_sharded", "gather_shard_counts", "shard_losses"]
 
 
 class StagedForward:

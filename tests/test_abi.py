@@ -95,6 +95,18 @@ def test_seq_loss_and_bias_step_check_their_arguments_before_any_launch():
                              None) == _abi.MOE_ERR_NULL
 
 
+def test_sharded_capacity_checks_its_arguments_before_any_launch():
+    L = moe.lib()
+    tok = moe.moe_config(T=64, d=128, E=8, k=2, d_ff=128, dtype=1, cf=1.0)
+    rank = moe.moe_config(T=64, d=128, E=8, k=2, d_ff=128, dtype=1, cf=1.0, priority=1)
+    nul = [None] * 8
+    args = lambda cfg, C, n, i: (ctypes.byref(cfg), C, None, n, i, *nul, None, 0, None)
+    assert L.moe_capacity_sharded(*args(rank, 10, 2, 0)) == _abi.MOE_ERR_DTYPE
+    for C, n, i in ((-1, 2, 0), (10, 0, 0), (10, 2, 2), (10, 2, -1)):
+        assert L.moe_capacity_sharded(*args(tok, C, n, i)) == _abi.MOE_ERR_SHAPE
+    assert L.moe_capacity_sharded(*args(tok, 10, 2, 1)) == _abi.MOE_ERR_NULL
+
+
 def test_null_pointers_are_rejected_before_any_launch():
     cfg = moe.moe_config(CONFIGS["tiny"])
     L = moe.lib()

@@ -212,3 +212,52 @@ def test_bias_steps_balance_the_gpu_router():
         spread.append(int(c.max() - c.min()))
         moe.moe_bias_update(cfg, cap.counts, 0.01, bias)
     assert spread[-1] < spread[0] / 3, spread[::20]
+
+
+@pytest.mark.parametrize("shards,cf", [(3, 1.0), (2, 1.25), (4, math.inf)])
+def test_sharded_capacity_equals_the_whole_batch(shards, cf):
+    """A token-ordered batch split into shards (run one after another on this
+    GPU, the all-gather of counts done by stacking): each shard's keep, drop
+    and positions equal the whole batch's bit for bit, and the losses from the
+    shards' counts and loss rows match the whole batch's within 1e-5 (the
+    router splits K differently for a shard, so its loss rows may differ in
+    the last bits)."""
+    Tl, E, k, d = 1024, 16, 4, 256
+    shape = shrink(CONFIGS["deepseekmoe"], T=Tl * shards, d=d, E=E, k=k, d_ff=128,
+                   d_ff_shared=128, cf=cf, zipf_s=1.1)
+    inp = remove_near_ties(generate(shape, device="cuda"))
+    cfg_all = moe.moe_config(shape)
+    topk, _, part, _, _ = moe.moe_route(cfg_all, inp.x, inp.W_r, inp.logit_bias, inp.select_bias)
+    whole = moe.moe_capacity(cfg_all, topk)
+    C = moe.moe_capacity_value(cfg_all)
+    cfg_one = moe.moe_config(shape, T=Tl)
+    local = [moe.moe_capacity(cfg_one, topk[i * Tl:(i + 1) * Tl].contiguous())
+             for i in range(shards)]
+    shard_counts = torch.stack([c.counts for c in local])
+    base = torch.zeros(E, dtype=torch.int64, device="cuda")
+    kept_sum = torch.zeros(E, dtype=torch.int64, device="cuda")
+    nd = 0
+    for i in range(shards):
+        rows = slice(i * Tl, (i + 1) * Tl)
+        out = moe.moe_capacity_sharded(cfg_one, C, shard_counts, i, topk[rows].contiguous())
+        torch.cuda.synchronize()
+        assert torch.equal(out.keep, whole.keep[rows])
+        assert torch.equal(out.dropped, whole.dropped[rows])
+        e = topk[rows].long()
+        assert torch.equal(out.pos.long() + base[e], whole.pos[rows].long())
+        assert torch.equal(out.counts, local[i].counts)
+        kept_sum += out.kept.long()
+        nd += int(out.n_dropped.item())
+        base += out.counts.long()
+    assert torch.equal(kept_sum, whole.kept.long())
+    assert nd == int(whole.n_dropped.item())
+    if cf == 1.0:
+        assert nd > 0
+    # losses: counts summed, loss rows concatenated in shard order
+    part_l = [moe.moe_route(cfg_one, inp.x[i * Tl:(i + 1) * Tl].contiguous(), inp.W_r,
+                            inp.logit_bias, inp.select_bias)[2] for i in range(shards)]
+    aux_s, z_s = moe.moe_losses(cfg_all, shard_counts.sum(0).to(torch.int32), torch.cat(part_l))
+    aux_w, z_w = moe.moe_losses(cfg_all, whole.counts, part)
+    torch.cuda.synchronize()
+    assert aux_s.item() == pytest.approx(aux_w.item(), rel=LOSS_RTOL)
+    assert z_s.item() == pytest.approx(z_w.item(), rel=LOSS_RTOL)
