@@ -46,10 +46,10 @@ from moe_inputs import CONFIGS, generate, seed_for  # noqa: E402
 METRIC = "MoE layer fwd tokens/s on 1 B200; grouped-GEMM % BF16 peak; dispatch % HBM BW"
 UNIT = "tokens/s"
 def kernels_per_step(shape) -> int:
-    """Kernels of ours one forward launches: route (bf16: weight split, logits,
-    select; fp32: one), capacity 3, dispatch 1, expert FFN (bf16: the two
-    grouped GEMMs; fp32: two, plus two for shared experts), combine 1, losses 1."""
-    route = 3 if shape.dtype == 1 else 1
+    """Kernels of ours one forward launches: route 1, capacity 3, dispatch 1,
+    expert FFN (bf16: the two grouped GEMMs; fp32: two, plus two for shared
+    experts), combine 1, losses 1."""
+    route = 1
     ffn = 2 if shape.dtype == 1 else (4 if shape.n_shared else 2)
     return route + 3 + 1 + ffn + 1 + 1
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -82,6 +82,9 @@ def parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", choices=["route"], default=None,
+                    help="time one stage alone on the workload's tensors (profiling aid; "
+                         "prints its own JSON line, not the benchmark line)")
     return ap.parse_args(argv)
 
 
@@ -539,8 +542,45 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+def run_stage(args):
+    """The router alone on the workload's tokens and router weights: the same
+    seeded draw with the experts narrowed to 64 columns, so the expert weights
+    take no room.  W warm-up calls, then K calls between CUDA events."""
+    import mixture_experts_layer_54_b200 as moe
+    from moe_inputs import shrink
+    device = torch.device("cuda", 0)
+    shape = CONFIGS[args.config]
+    small = shrink(shape, d_ff=64, d_ff_shared=64 if shape.n_shared else shape.d_ff_shared)
+    inp = generate(small, device)
+    cfg = moe.moe_config(small)
+    ws = moe.workspace(moe.moe_stage_workspace_size(cfg), device)
+    call = lambda: moe.moe_route(cfg, inp.x, inp.W_r, inp.logit_bias, inp.select_bias, ws=ws)
+    for _ in range(max(args.warmup, 1)):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    if moe.moe_device_status(ws) != 0:
+        raise SystemExit("device status set: a bounded wait expired")
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    x_bytes = inp.x.numel() * inp.x.element_size()
+    peaks, _ = load_peaks()
+    print(json.dumps({"stage": "route", "workload": workload_name(shape), "calls": args.steps,
+                      "us_per_call": round(us, 2), "x_bytes": x_bytes,
+                      "GB/s": round(x_bytes / us / 1e3, 1),
+                      "hbm_frac": round(x_bytes / us / 1e3 / peaks["hbm_gbs"], 3),
+                      "timing": "back-to-back calls, CUDA events (launch gaps included)"}))
+
+
 def main(argv=None):
     args = parse(argv)
+    if args.stage:
+        run_stage(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

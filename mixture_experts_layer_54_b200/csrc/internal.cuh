@@ -29,11 +29,13 @@ int route_blocks(const moe_config &c);   // blocks of the tiled route kernel
 int partial_rows(const moe_config &c);   // rows of the loss partials, ceil(T / 32)
 int cap_blocks(const moe_config &c);
 
-// Tensor-core router layout (bf16 layers): experts padded to E_pad, split in
-// chunks of n_chunk per block, K split in k_parts.
+// Tensor-core router layout (bf16 layers).  Fused (E <= 16): one kernel, the
+// k_parts blocks of a 128-token tile form one cluster.  Otherwise three
+// launches: experts padded to E_pad in n_chunks chunks of n_chunk, K
+// (k_blocks of 64) split in k_parts of kb_per_part, through scratch.
 struct RoutePlan {
-    bool tensor_cores;
-    int E_pad, n_chunk, k_parts, kb_per_part;
+    bool tensor_cores, fused;
+    int E_pad, n_chunk, n_chunks, k_blocks, k_parts, kb_per_part, cluster, blocks;
 };
 RoutePlan route_plan(const moe_config &c);
 size_t route_scratch_bytes(const moe_config &c);
@@ -43,7 +45,7 @@ size_t route_scratch_bytes(const moe_config &c);
 // while it runs, and calls on one stream do not overlap).
 struct StageScratch {
     int32_t *status;      // device status word (timeouts)
-    void *route;          // tensor-core router: split weights and partial logits
+    void *route;          // tensor-core router (three launches): split weights, partial logits
     int32_t *hist;        // [cap_blocks][k][E]
     int32_t *base;        // [cap_blocks][k][E]
     int32_t *count_base;  // [E] sharded capacity: earlier shards' assignments

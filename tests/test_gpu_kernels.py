@@ -301,15 +301,8 @@ def test_gathered_expert_ffn_equals_dispatch_then_ffn(case):
         assert torch.equal(Ysh, Ysh_ref)
 
 
-@pytest.mark.parametrize("E,k", [(9, 2), (16, 4), (32, 8), (33, 3), (64, 6), (96, 8), (128, 1),
-                                 (129, 5), (200, 8), (256, 8)])
-@pytest.mark.parametrize("score", [0, 1], ids=["softmax", "sigmoid"])
-def test_route_selection_every_width(E, k, score):
-    """The selection kernel at every lane width (1, 2, 4 or 8 experts per
-    lane), ragged expert counts included: top-k of the kernel's own fp32 keys
-    with ties to the lower index, gates, and the loss partials."""
-    T, d = 1000, 256
-    g = torch.Generator(device=DEV).manual_seed(E * 10 + k + score)
+def _check_route(T, d, E, k, score, seed):
+    g = torch.Generator(device=DEV).manual_seed(seed)
     x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
     W_r = torch.randn((d, E), generator=g, device=DEV) * 0.05
     sb = ((torch.rand(E, generator=g, device=DEV) - 0.5) * 0.2) if score == 1 else None
@@ -317,6 +310,10 @@ def test_route_selection_every_width(E, k, score):
     topk, gates, part, logits, scores = moe.moe_route(cfg, x, W_r, None, sb, want_logits=True,
                                                       want_scores=True)
     torch.cuda.synchronize()
+    # the logits are the fp32 router: within the recursive-summation bound of x W_r
+    z = x.double() @ W_r.double()
+    bound = d * 2.0 ** -24 * (x.double().abs() @ W_r.double().abs())
+    assert torch.all((logits.double() - z).abs() <= bound + 1e-7)
     key = logits if score == 0 else scores + sb   # fp32, as the kernel ranks
     ref = np.argsort(-key.double().cpu().numpy(), axis=1, kind="stable")[:, :k]
     np.testing.assert_array_equal(topk.cpu().numpy(), ref)
@@ -325,8 +322,39 @@ def test_route_selection_every_width(E, k, score):
     assert (gates.double() - want).abs().max().item() < 1e-6
     # loss partials: the probability mass per expert and lse^2, summed over the batch
     rows = part.view(-1, E + 1).double()
+    assert rows.shape[0] == (T + 31) // 32
     p = scores.double() if score == 0 else scores.double() / scores.double().sum(1, keepdim=True)
     np.testing.assert_allclose(rows[:, :E].sum(0).cpu().numpy(), p.sum(0).cpu().numpy(),
                                rtol=1e-5, atol=1e-4)
     lse = torch.logsumexp(logits.double(), dim=1)
     assert rows[:, E].sum().item() == pytest.approx((lse ** 2).sum().item(), rel=1e-5)
+    # each row holds its own 32 tokens
+    r0 = rows[0].cpu()
+    assert r0[:E].numpy() == pytest.approx(p[:32].sum(0).cpu().numpy(), rel=1e-5, abs=1e-5)
+
+
+@pytest.mark.parametrize("E,k", [(9, 2), (16, 4), (32, 8), (33, 3), (64, 6), (96, 8), (128, 1),
+                                 (129, 5), (200, 8), (256, 8)])
+@pytest.mark.parametrize("score", [0, 1], ids=["softmax", "sigmoid"])
+def test_route_selection_every_width(E, k, score):
+    """The selection at every lane width (1, 2, 4 or 8 experts per lane),
+    ragged expert counts included: top-k of the kernel's own fp32 keys with
+    ties to the lower index, gates, and the loss partials."""
+    _check_route(1000, 256, E, k, score, E * 10 + k + score)
+
+
+@pytest.mark.parametrize("T,d,E,k", [
+    (1000, 1024, 4, 1),    # 4 experts per token group, K in 4 parts (cluster of 4)
+    (777, 512, 8, 2),      # 8 experts per token group, K in 2 parts
+    (1000, 1024, 16, 4),   # a warp per token, K in 4 parts
+    (600, 512, 40, 3),     # 48-wide expert chunk, K in 2 parts
+    (333, 1024, 64, 6),    # 64-wide chunk, K in 4 parts, ragged last tile
+    (500, 512, 100, 8),    # 2 expert chunks x 2 K parts
+    (64, 256, 8, 2),       # less than one 128-token tile
+    (40, 256, 200, 8),     # 4 expert chunks, two rows of the loss partials
+])
+@pytest.mark.parametrize("score", [0, 1], ids=["softmax", "sigmoid"])
+def test_route_cluster_shapes(T, d, E, k, score):
+    """Every way the blocks of a token tile split the work (K parts, expert
+    chunks, clusters of 1, 2 or 4 blocks): the same checks as above."""
+    _check_route(T, d, E, k, score, T + d + E + k + score)
