@@ -295,7 +295,8 @@ __device__ __forceinline__ void select_token(const RouteParams &a, bool renorm, 
 
 // ---------------------------------------------------------------- kernel
 
-// N: experts per block (16, 32, 48 or 64).  Selection: E_T > 0 takes E <= E_T
+// N: experts per block (launched with 16; the kernel also takes 32, 48 or 64,
+// measured slower than three launches there).  Selection: E_T > 0 takes E <= E_T
 // experts with E_T lanes per token (32 / E_T tokens per warp at once); E_T == 0
 // takes a warp per token with PL experts per lane.
 template <int N, int E_T, int PL>
