@@ -930,17 +930,20 @@ typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, 
                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (a function-local static is
+// initialised once even when several host threads make their first call
+// together); null when the driver does not provide it.
 EncodeTiled encoder()
 {
-    static EncodeTiled fn = nullptr;
-    if (!fn) {
+    static const EncodeTiled fn = []() -> EncodeTiled {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(ptr);
-    }
+            return reinterpret_cast<EncodeTiled>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
