@@ -35,8 +35,13 @@ def moe_config(shape=None, **kw) -> MoeConfig:
 
 
 def _p(t):
+    """Device pointer of a tensor argument (None passes a null pointer).  The
+    library reads and writes dense row-major buffers, so a strided view is
+    refused rather than read as if it were dense."""
     if t is None:
         return None
+    if not t.is_contiguous():
+        raise ValueError("moe ops take contiguous tensors (call .contiguous() on views)")
     if not t.is_cuda:
         raise ValueError("moe ops take CUDA tensors")
     return ctypes.c_void_p(t.data_ptr())

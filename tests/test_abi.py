@@ -131,3 +131,17 @@ def test_sizes_cover_every_config():
         assert R >= min(shape.T * shape.k, shape.E * C) + shape.E * (_abi.MOE_ROW_ALIGN - 1)
         assert moe.moe_workspace_size(cfg) > moe.moe_stage_workspace_size(cfg) > 0
         assert moe.moe_loss_partials_count(cfg) == math.ceil(shape.T / 32) * (shape.E + 1)
+
+
+def test_binding_refuses_views_and_host_tensors_before_calling_the_library():
+    """The library reads dense row-major device buffers: the binding refuses a
+    strided view (whatever its device) and a host tensor."""
+    import torch
+    from mixture_experts_layer_54_b200 import ops
+    cfg = moe.moe_config(CONFIGS["tiny"])
+    W_r = torch.zeros((cfg.d, cfg.E))
+    with pytest.raises(ValueError, match="contiguous"):
+        moe.moe_route(cfg, torch.zeros((cfg.d, cfg.T)).t(), W_r, ws=torch.zeros(256))
+    with pytest.raises(ValueError, match="CUDA"):
+        ops._p(torch.zeros(4))
+    assert ops._p(None) is None
