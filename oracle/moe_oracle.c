@@ -143,9 +143,10 @@ int oracle_route(int T, int d, int E, int k, int score, int renorm,
 /* ------------------------------------------------------------------------ */
 
 /*
- * C = ceil(capacity_factor * T k / E)   ([Lab18 sec. 3] capacity formula)
- * A factor below 1 is an error ([Lab01] traps).  An infinite factor means no
- * limit; C = T then suffices because a token's k experts are distinct.
+ * C = ceil(capacity_factor * T k / E)   ([Lab18 sec. 3] capacity formula),
+ * held at T when it exceeds T.  A factor below 1 is an error ([Lab01] traps).
+ * An infinite factor means no limit; C = T then suffices because a token's k
+ * experts are distinct.
  */
 int oracle_capacity_value(int T, int E, int k, double cf, int64_t *C)
 {
@@ -157,7 +158,11 @@ int oracle_capacity_value(int T, int E, int k, double cf, int64_t *C)
         *C = T;
         return OR_OK;
     }
-    *C = (int64_t)ceil(cf * (double)((int64_t)T * k) / (double)E);
+    /* A token's k experts are distinct, so no expert receives more than T
+     * assignments and any C >= T keeps them all: C is held at T, which keeps
+     * the integer conversion defined for huge finite factors. */
+    const double c = ceil(cf * (double)((int64_t)T * k) / (double)E);
+    *C = c >= (double)T ? (int64_t)T : (int64_t)c;
     return OR_OK;
 }
 

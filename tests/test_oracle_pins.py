@@ -233,6 +233,20 @@ def test_capacity_ceil_formula_values():
     assert oracle.capacity(10, 3, 1, 1.0) == 4          # ceil(10/3)
 
 
+def test_capacity_above_T_is_held_at_T_and_changes_no_decision():
+    # a token's k experts are distinct ("Lab 18" section 1, top-k), so an
+    # expert receives at most T assignments: any C >= T keeps everything
+    assert oracle.capacity(64, 4, 2, 1e20) == 64
+    assert oracle.capacity(10, 2, 2, 1.25) == 10        # ceil(12.5) = 13 > T
+    rng = np.random.default_rng(5)
+    topk = np.stack([rng.choice(2, size=2, replace=False) for _ in range(10)]).astype(np.int32)
+    held = oracle.capacity_walk(topk, 2, 1.25)
+    unclamped = oracle.capacity_walk(topk, 2, C=13)
+    assert held.keep.all() and unclamped.keep.all() and held.n_dropped == 0
+    big = oracle.capacity_walk(np.zeros((64, 1), np.int32), 4, 1e20)
+    assert big.keep.all() and big.n_dropped == 0
+
+
 def test_token_order_fcfs_keeps_the_earliest_tokens():
     # "Lab 01" step 4: first come first served in token order
     T, E, k = 16, 4, 1
