@@ -45,17 +45,44 @@ from moe_inputs import CONFIGS, generate, seed_for  # noqa: E402
 
 METRIC = "MoE layer fwd tokens/s on 1 B200; grouped-GEMM % BF16 peak; dispatch % HBM BW"
 UNIT = "tokens/s"
+def route_kernels(shape) -> int:
+    """Kernels of the router: bf16 layers with up to 64 experts whose split
+    router weights of a K part (3 x E padded x 64 x 2 bytes per K block) fit
+    in shared memory run one kernel, wider ones three (split, logits,
+    select); the fp32 layer one."""
+    if shape.dtype != 1:
+        return 1
+    if shape.E <= 64:
+        ne = 16 if shape.E <= 16 else (shape.E + 15) // 16 * 16
+        kb = shape.d // 64
+        p = 4
+        while p > 1 and (kb % p or kb // p < 4):
+            p //= 2
+        kbp = kb // p
+        for stages in (4, 3, 2):
+            x = (kbp * 3 * ne * 128 + 1023) // 1024 * 1024
+            total = x + stages * 16384 + 2 * 128 * (ne + 4) * 4 + \
+                max(8 * (ne + 1), 32 * 9) * 4 + 1024
+            if total <= 227 * 1024:
+                break
+        if kbp * 3 * ne * 128 <= 112 * 1024 and total <= 227 * 1024:
+            return 1
+    return 3
+
+
 def kernels_per_step(shape) -> int:
-    """Kernels of ours one forward launches: route 1, capacity 3, dispatch 1,
-    expert FFN (bf16: the two grouped GEMMs; fp32: two, plus two for shared
-    experts), combine 1, losses 1."""
-    route = 1
+    """Kernels of ours one moe_forward launches: the router (route_kernels),
+    capacity 2 (histograms; placement with the totals and the losses),
+    dispatch 1, expert FFN (bf16: the two grouped GEMMs; fp32: two, plus two
+    for shared experts), combine 1; the score-ordered capacity adds three
+    launches and a losses launch."""
     ffn = 2 if shape.dtype == 1 else (4 if shape.n_shared else 2)
-    return route + 3 + 1 + ffn + 1 + 1
+    extra = 4 if shape.priority == 2 else 0
+    return route_kernels(shape) + 2 + 1 + ffn + 1 + extra
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) of the expert-FFN stage (GEMM1 + GEMM2) per launch, from one ncu
-# capture (profiles/gemm_2sm_mixtral.md), valid only for the GEMM source it was taken on.
+# capture of the same workload, valid only for the GEMM source it was taken on.
 GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_54_b200", "csrc", "ffn_tcgen05.cu")
 MEASURED_TRAFFIC = {
     ("mixtral", "872c0a36b644350c28d3aa0b8c0abd44d4e57e623453bff990cab6d72699abde"): 4.964e9,
@@ -82,9 +109,15 @@ def parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=["route"], default=None,
+    ap.add_argument("--no-per-layer", action="store_true",
+                    help="skip the Switch, DeepSeekMoE and DeepSeek-V3 shaped layers that the "
+                         "default (Mixtral-shaped) run also times")
+    ap.add_argument("--stage", choices=["route", "ffn"], default=None,
                     help="time one stage alone on the workload's tensors (profiling aid; "
                          "prints its own JSON line, not the benchmark line)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="with --stage ffn: this many experts, tokens scaled so that each "
+                         "expert keeps its rows (a smaller device footprint, same GEMM shapes)")
     return ap.parse_args(argv)
 
 
@@ -184,7 +217,8 @@ class ClockSampler:
 
 def perm_rows(shape) -> int:
     """Rows of the permuted buffers: kept slots plus per-expert padding to 128."""
-    C = shape.T if math.isinf(shape.cf) else math.ceil(shape.cf * shape.T * shape.k / shape.E)
+    C = shape.T if math.isinf(shape.cf) else min(shape.T, math.ceil(shape.cf * shape.T * shape.k
+                                                                    / shape.E))
     kept = min(shape.T * shape.k, C * shape.E)
     return (kept + shape.E * 127 + 127) // 128 * 128
 
@@ -249,9 +283,12 @@ def time_oracle(shape, h, n_tokens):
 
 
 def size_oracle_sample(shape, h, seconds):
-    """Tokens whose FFNs take about `seconds` on the host cores."""
-    _, t4 = time_oracle(shape, h, 4)
-    per = max(t4 / 4, 1e-6)
+    """Tokens whose FFNs take about `seconds` on the host cores (probed on one
+    token per host thread, so the probe itself keeps every core busy)."""
+    import oracle
+    probe = min(shape.T, max(4, oracle.num_threads()))
+    _, tp = time_oracle(shape, h, probe)
+    per = max(tp / probe, 1e-6)
     return int(max(4, min(shape.T, seconds / per)))
 
 
@@ -302,29 +339,64 @@ def next_rows(moe, shape, inp, staged, seq_len):
 
 
 def fused_dispatch(moe, cfg, inp, staged):
-    """The dispatch fused into GEMM1 (row table + gathered expert FFN) against
-    the permuted copy + expert FFN that the step runs, same batch, same box."""
+    """The dispatch fused into GEMM1 (row table + rows gathered from x) and the
+    combine's gate fused into GEMM2 (gated rows to a [T k, d] buffer, then an
+    ordered sum), against the permuted copy + expert FFN + combine that the
+    step runs; same batch, same box, each from a captured graph."""
     R = moe.moe_perm_rows(cfg)
     dev = inp.x.device
     rows = torch.empty((R,), dtype=torch.int32, device=dev)
     Y = torch.empty_like(staged.Y_perm)
     Ysh = None if staged.Y_sh is None else torch.empty_like(staged.Y_sh)
+    Yslot = torch.empty((cfg.T * cfg.k, cfg.d), dtype=staged.y.dtype, device=dev)
+    y = torch.empty_like(staged.y)
+    w = (inp.W1, inp.W3, inp.W2)
+    ws = (inp.Ws1, inp.Ws3, inp.Ws2)
 
-    def fused():
+    def dispatch_fused():
         moe.moe_dispatch_rows(cfg, staged.topk, staged.pos, staged.keep, staged.offsets, rows)
-        moe.moe_expert_ffn_gather(cfg, inp.x, rows, staged.offsets, inp.W1, inp.W3, inp.W2,
-                                  inp.Ws1, inp.Ws3, inp.Ws2, ws=staged.ws, Y_perm=Y, Y_shared=Ysh)
+        moe.moe_expert_ffn_gather(cfg, inp.x, rows, staged.offsets, *w, *ws, ws=staged.ws,
+                                  Y_perm=Y, Y_shared=Ysh)
 
-    def unfused():
+    def dispatch_unfused():
         moe.moe_dispatch(cfg, inp.x, staged.topk, staged.pos, staged.keep, staged.offsets,
                          staged.x_perm)
-        moe.moe_expert_ffn(cfg, staged.x_perm, staged.offsets, inp.W1, inp.W3, inp.W2, inp.x,
-                           inp.Ws1, inp.Ws3, inp.Ws2, ws=staged.ws, Y_perm=Y, Y_shared=Ysh)
-    t_fused = graph_time_us(fused, n=5)
-    t_unfused = graph_time_us(unfused, n=5)
-    return {"us": round(t_fused, 1), "unfused_us": round(t_unfused, 1), "launches": 3,
-            "note": "moe_dispatch_rows + moe_expert_ffn_gather (TMA gather4 rows) vs "
-                    "moe_dispatch + moe_expert_ffn"}
+        moe.moe_expert_ffn(cfg, staged.x_perm, staged.offsets, *w, inp.x, *ws, ws=staged.ws,
+                           Y_perm=Y, Y_shared=Ysh)
+
+    def unfused():
+        dispatch_unfused()
+        moe.moe_combine(cfg, Y, Ysh, staged.gates, staged.topk, staged.pos, staged.keep,
+                        staged.offsets, y=y)
+
+    def combine_fused():
+        moe.moe_dispatch(cfg, inp.x, staged.topk, staged.pos, staged.keep, staged.offsets,
+                         staged.x_perm, src_slot=rows)
+        moe.moe_expert_ffn_slots(cfg, staged.x_perm, inp.x, rows, staged.offsets, staged.kept,
+                                 staged.gates, *w, *ws, ws=staged.ws, Y_slot=Yslot, Y_shared=Ysh)
+        moe.moe_combine_slots(cfg, Yslot, Ysh, staged.keep, y=y)
+
+    def both_fused():
+        moe.moe_dispatch_rows(cfg, staged.topk, staged.pos, staged.keep, staged.offsets, rows)
+        moe.moe_expert_ffn_slots(cfg, None, inp.x, rows, staged.offsets, staged.kept,
+                                 staged.gates, *w, *ws, ws=staged.ws, Y_slot=Yslot, Y_shared=Ysh)
+        moe.moe_combine_slots(cfg, Yslot, Ysh, staged.keep, y=y)
+
+    t = {name: graph_time_us(fn, n=5) for name, fn in
+         [("dispatch_fused", dispatch_fused), ("dispatch_unfused", dispatch_unfused),
+          ("unfused", unfused), ("combine_fused", combine_fused), ("both_fused", both_fused)]}
+    if moe.moe_device_status(staged.ws) != 0:
+        raise SystemExit("device status set by a fused variant")
+    return {"us": round(t["dispatch_fused"], 1), "unfused_us": round(t["dispatch_unfused"], 1),
+            "launches": 3,
+            "dispatch_and_ffn": {"fused_us": round(t["dispatch_fused"], 1),
+                                 "unfused_us": round(t["dispatch_unfused"], 1)},
+            "dispatch_ffn_combine": {"unfused_us": round(t["unfused"], 1),
+                                     "combine_fused_us": round(t["combine_fused"], 1),
+                                     "both_fused_us": round(t["both_fused"], 1)},
+            "note": "dispatch fused: moe_dispatch_rows + moe_expert_ffn_gather (cp.async row "
+                    "gathers) vs moe_dispatch + moe_expert_ffn; combine fused: "
+                    "moe_expert_ffn_slots (gate in GEMM2's epilogue) + moe_combine_slots"}
 
 
 def cpu_baseline(shape, inp, seconds):
@@ -358,7 +430,9 @@ def run_reference(args):
     shape = CONFIGS[args.config]
     inp = generate(shape, device="cpu")
     h = oracle_inputs(inp)
-    n = size_oracle_sample(shape, h, 1.0)
+    # at least four tokens per host thread (the oracle's FFN loop runs OpenMP
+    # over tokens), else too few tokens leave cores idle and understate it
+    n = max(size_oracle_sample(shape, h, 1.0), min(shape.T, 4 * oracle.num_threads()))
     for _ in range(args.warmup):
         time_oracle(shape, h, n)
     tr = tf = 0.0
@@ -385,6 +459,161 @@ def run_reference(args):
 
 # ------------------------------------------------------------ our arm
 
+def time_layer_graph(moe, shape, inp, dev, steps, warmup, local):
+    """Graph-timed forwards of one layer (inputs resident).
+
+    value: `steps` calls of moe_forward (the public one-call API) captured
+    once in a CUDA graph with events only before the first and after the last,
+    replayed once between synchronises while clocks are sampled.
+    stages: the same number of forwards as the six per-stage calls (route,
+    capacity, dispatch, expert FFN, combine, losses) with events between the
+    stages, captured and replayed separately; events between kernels keep the
+    next kernel from starting early, so the stages add up to a little more
+    than the forward."""
+    cfg = moe.moe_config(shape)
+    fwd = moe.MoEForward(cfg, dev)
+    w = moe.weights_struct(inp.W_r, inp.W1, inp.W2, inp.W3, inp.logit_bias, inp.select_bias,
+                           inp.Ws1, inp.Ws3, inp.Ws2)
+    staged = moe.StagedForward(cfg, dev)
+    wargs = (inp.x, inp.W_r, inp.W1, inp.W2, inp.W3, inp.logit_bias, inp.select_bias, inp.Ws1,
+             inp.Ws3, inp.Ws2)
+    nst = len(moe.StagedForward.STAGES)
+    for _ in range(max(warmup, 3)):
+        fwd(inp.x, w)
+        staged(*wargs)
+    torch.cuda.synchronize()
+    for ws in (fwd.ws, staged.ws):
+        status = moe.moe_device_status(ws)
+        if status != 0:
+            raise SystemExit(f"device status {status} after warm-up ({shape.name}): a bounded "
+                             "wait gave up; not timing a failing kernel")
+    if steps is None:   # enough steps for about a quarter of a second
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            fwd(inp.x, w)
+        e1.record()
+        torch.cuda.synchronize()
+        per = e0.elapsed_time(e1) / 3 / 1e3
+        steps = int(min(max(0.25 / max(per, 1e-6), 20), 2000))
+
+    # ---- the forward, K calls in one graph ----
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        ev[0].record()
+        for _ in range(steps):
+            fwd(inp.x, w)
+        ev[1].record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        graph.replay()
+        torch.cuda.synchronize()
+    barrier(dev)
+    status = moe.moe_device_status(fwd.ws)
+    if status != 0:
+        raise SystemExit(f"device status {status} in the timed region ({shape.name})")
+    total_ms = ev[0].elapsed_time(ev[1])
+    del graph
+
+    # ---- the per-stage calls, with events between the stages ----
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nst + 1)]
+              for _ in range(steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        for i in range(steps):
+            staged(*wargs, events=events[i])
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    if moe.moe_device_status(staged.ws) != 0:
+        raise SystemExit(f"device status set in the per-stage replay ({shape.name})")
+    stage_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in events) / steps for i in range(nst)]
+    staged_total = events[0][0].elapsed_time(events[-1][-1]) / steps
+    del graph
+    if not torch.equal(fwd.y, staged.y):
+        raise SystemExit(f"the forward and the per-stage calls disagree ({shape.name})")
+    return {"staged": staged, "fwd": fwd, "steps": steps, "ms_per_step": total_ms / steps,
+            "staged_ms_per_step": staged_total,
+            "stage_ms": dict(zip(moe.StagedForward.STAGES, stage_ms)),
+            "kept": int(staged.kept.sum().item()),
+            "dropped_tokens": int(staged.dropped.sum().item()),
+            "status": status, "clocks": clk.summary()}
+
+
+def summarize_layer(shape, ms_per_step, stage_ms, kept, dropped_tokens, steps, peaks, world=1):
+    """Per-stage rates, the expert FFN against the bf16 peak, and the layer
+    roofline (slower of its FLOPs at the bf16 peak and its bytes at the HBM
+    copy bandwidth) for one graph-timed layer."""
+    work = layer_work(shape, None, kept, dropped_tokens)
+    stages = {}
+    for name, ms in stage_ms.items():
+        entry = {"us": round(ms * 1e3, 2)}
+        if "bytes" in work[name]:
+            entry["GB/s"] = round(work[name]["bytes"] / (ms / 1e3) / 1e9, 1)
+            entry["hbm_frac"] = round(entry["GB/s"] / peaks["hbm_gbs"], 3)
+        if "flops" in work[name]:
+            entry["TFLOP/s"] = round(work[name]["flops"] / (ms / 1e3) / 1e12, 1)
+        stages[name] = entry
+    ffn = work["expert_ffn"]
+    ach = ffn["flops"] / (stage_ms["expert_ffn"] / 1e3) / 1e12
+    # A timed region long enough for the 1 kW power cap to settle (>= 0.2 s)
+    # is compared with the sustained matmul figure, a shorter one with the
+    # burst figure; both fractions are reported.
+    region_s = ms_per_step * steps / 1e3
+    peak_kind = "sustained" if region_s >= 0.2 else "burst"
+    peak = peaks["bf16_tflops_sustained" if peak_kind == "sustained" else "bf16_tflops"]
+    t_flop = ffn["flops"] / (peak * 1e12)
+    all_bytes = sum(work[n].get("bytes", 0) for n in stage_ms)
+    t_byte = all_bytes / (peaks["hbm_gbs"] * 1e9)
+    ffn_t_byte = ffn["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    return {
+        "stages": stages,
+        "expert_ffn": {"TFLOP/s": round(ach, 1), "peak_TFLOP/s": peak, "peak_kind": peak_kind,
+                       "frac_of_peak": round(ach / peak, 4),
+                       "GB/s": round(ffn["bytes"] / (stage_ms["expert_ffn"] / 1e3) / 1e9, 1),
+                       "hbm_frac": round(ffn_t_byte / (stage_ms["expert_ffn"] / 1e3), 4),
+                       "bound": "tensor" if ffn["flops"] / (peak * 1e12) >= ffn_t_byte else "hbm",
+                       "flops": ffn["flops"], "algorithmic_bytes": ffn["bytes"]},
+        "layer_roofline": {"t_flop_us": round(t_flop * 1e6, 1), "t_byte_us": round(t_byte * 1e6, 1),
+                           "bound": "tensor" if t_flop >= t_byte else "hbm",
+                           "frac": round(max(t_flop, t_byte) / (ms_per_step / 1e3), 4)},
+        "timed_region_s": round(region_s, 3),
+        "roofline_peak": (peak, peak_kind, ach),
+    }
+
+
+def per_layer(moe, dev, local, peaks, names, warmup):
+    """The other model-shaped layers, graph-timed one after another in the
+    same run (each layer's tensors freed before the next is drawn)."""
+    out = {}
+    for name in names:
+        shape = CONFIGS[name]
+        inp = generate(shape, device=dev)
+        r = time_layer_graph(moe, shape, inp, dev, None, warmup, local)
+        sm = summarize_layer(shape, r["ms_per_step"], r["stage_ms"], r["kept"],
+                             r["dropped_tokens"], r["steps"], peaks)
+        sm.pop("roofline_peak")
+        clk = r["clocks"]
+        out[name] = {"workload": workload_name(shape),
+                     "value": round(shape.T / (r["ms_per_step"] / 1e3), 1), "unit": UNIT,
+                     "ms_per_step": round(r["ms_per_step"], 4), "steps": r["steps"],
+                     "staged_ms_per_step": round(r["staged_ms_per_step"], 4),
+                     "kept_assignments": r["kept"], "dropped_tokens": r["dropped_tokens"],
+                     "gpu_launches": kernels_per_step(shape) * r["steps"],
+                     "clocks": {"sm_mhz": clk["sm_mhz"], "reasons": clk["reasons"],
+                                "samples": clk["samples"]},
+                     "traffic": measured_traffic(name), **sm}
+        r.pop("staged")
+        r.pop("fwd")
+        del r, inp
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import mixture_experts_layer_54_b200 as moe
 
@@ -396,44 +625,13 @@ def run_ours(args):
     shape = CONFIGS[args.config]
     inp = generate(shape, device=dev, seed=seed_for(shape) + 1000 * rank)
     cfg = moe.moe_config(shape)
-    staged = moe.StagedForward(cfg, dev)
-    wargs = (inp.x, inp.W_r, inp.W1, inp.W2, inp.W3, inp.logit_bias, inp.select_bias, inp.Ws1,
-             inp.Ws3, inp.Ws2)
-    nst = len(moe.StagedForward.STAGES)
-
-    for _ in range(max(args.warmup, 3)):
-        staged(*wargs)
-    torch.cuda.synchronize()
-    kept_total = int(staged.kept.sum().item())
-    dropped_tokens = int(staged.dropped.sum().item())
-    status = moe.moe_device_status(staged.ws)
-    if status != 0:
-        raise SystemExit(f"device status {status} after warm-up: the expert GEMM gave up "
-                         "waiting; not timing a failing kernel")
 
     # ---- device-timed region: the K steps, captured once in a CUDA graph with
     # timing events between the stages, replayed once between barriers ----
-    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nst + 1)]
-              for _ in range(args.steps)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
-        for i in range(args.steps):
-            staged(*wargs, events=events[i])
-    torch.cuda.synchronize()
-    barrier(dev)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        graph.replay()
-        torch.cuda.synchronize()
-    barrier(dev)
-    status = moe.moe_device_status(staged.ws)
-    if status != 0:
-        raise SystemExit(f"device status {status} in the timed region")
-    total_ms = events[0][0].elapsed_time(events[-1][-1])
-    stage_ms = [sum(ev[s].elapsed_time(ev[s + 1]) for ev in events) / args.steps
-                for s in range(nst)]
-    del graph
-    ms_per_step = max_over_ranks(total_ms / args.steps, dev)
+    r = time_layer_graph(moe, shape, inp, dev, args.steps, args.warmup, local)
+    staged, status, clocks = r["staged"], r["status"], r["clocks"]
+    kept_total, dropped_tokens = r["kept"], r["dropped_tokens"]
+    ms_per_step = max_over_ranks(r["ms_per_step"], dev)
 
     # ---- end to end: pinned host input in, result out, inside the timed region.
     # Batches stream through HostStream (public API): each step copies its x
@@ -469,55 +667,41 @@ def run_ours(args):
         if shape.T % 32 == 0 and shape.T > 0 else None
     if extra is not None:
         extra["fused_dispatch"] = fused_dispatch(moe, cfg, inp, staged)
+    peaks, peak_src = load_peaks()
+    layers = None
+    if world == 1 and not args.no_per_layer and args.config == "mixtral":
+        del staged, inp, w
+        r.pop("staged")
+        r.pop("fwd")
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        layers = per_layer(moe, dev, local, peaks, ["switch", "deepseekmoe", "deepseek_v3"],
+                           args.warmup)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return
 
-    peaks, peak_src = load_peaks()
-    work = layer_work(shape, None, kept_total, dropped_tokens)
     tokens = shape.T * world
     value = tokens / (ms_per_step / 1e3)
-    st = dict(zip(moe.StagedForward.STAGES, stage_ms))
-    stages = {}
-    for name, ms in st.items():
-        entry = {"us": round(ms * 1e3, 2)}
-        if "bytes" in work[name]:
-            entry["GB/s"] = round(work[name]["bytes"] / (ms / 1e3) / 1e9, 1)
-            entry["hbm_frac"] = round(entry["GB/s"] / peaks["hbm_gbs"], 3)
-        if "flops" in work[name]:
-            entry["TFLOP/s"] = round(work[name]["flops"] / (ms / 1e3) / 1e12, 1)
-        stages[name] = entry
-    ffn = work["expert_ffn"]
-    ach = ffn["flops"] / (st["expert_ffn"] / 1e3) / 1e12
-    # The stage runs inside a step of one graph replay.  A timed region long
-    # enough for the 1 kW power cap to settle (>= 0.2 s) is compared with the
-    # sustained matmul figure, a shorter one with the burst figure; both
-    # fractions are reported.
-    region_s = ms_per_step * args.steps / 1e3
-    peak_kind = "sustained" if region_s >= 0.2 else "burst"
-    peak = peaks["bf16_tflops_sustained" if peak_kind == "sustained" else "bf16_tflops"]
+    sm = summarize_layer(shape, ms_per_step, r["stage_ms"], kept_total, dropped_tokens,
+                         args.steps, peaks, world)
+    peak, peak_kind, ach = sm["roofline_peak"]
+    ffn = sm["expert_ffn"]
     roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(ach / peak, 4),
                 "traffic": measured_traffic(args.config),
                 "traffic_unit": "bytes per launch (ncu dram read + write, GEMM1 + GEMM2)",
-                "algorithmic_bytes": ffn["bytes"],
+                "algorithmic_bytes": ffn["algorithmic_bytes"],
                 "kernel": "moe_expert_ffn: grouped tcgen05 GEMM1 (act fused) + GEMM2",
                 "flops_per_launch": ffn["flops"],
                 "peak_source": f"{peak_src} bf16 {peak_kind} (MEASURED_PEAKS.json)",
-                "timed_region_s": round(region_s, 3),
+                "timed_region_s": sm["timed_region_s"],
                 "frac_of_burst": round(ach / peaks["bf16_tflops"], 4),
                 "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4)}
-    t_flop = ffn["flops"] / (peak * 1e12)
-    all_bytes = sum(work[n].get("bytes", 0) for n in moe.StagedForward.STAGES)
-    t_byte = all_bytes / (peaks["hbm_gbs"] * 1e9)
-    layer_roof = {"t_flop_us": round(t_flop * 1e6, 1), "t_byte_us": round(t_byte * 1e6, 1),
-                  "bound": "tensor" if t_flop >= t_byte else "hbm",
-                  "frac": round(max(t_flop, t_byte) / (ms_per_step / 1e3), 4)}
     b = 2 if shape.dtype == 1 else 4
     h2d = shape.T * shape.d * b
     d2h = shape.T * shape.d * b + 8
-    clocks = clk.summary()
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -530,15 +714,19 @@ def run_ours(args):
             "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": kernels_per_step(shape) * args.steps,
-            "timing": "device: one CUDA graph of the K steps; e2e: HostStream (copies of step "
-                      "i +- 1 overlap step i's kernels)",
-            "roofline": roofline, "layer_roofline": layer_roof, "stages": stages,
+            "timing": "device: one CUDA graph of K moe_forward calls; stages: a second graph "
+                      "of the per-stage calls with events between them; e2e: HostStream "
+                      "(copies of step i +- 1 overlap step i's kernels)",
+            "roofline": roofline, "layer_roofline": sm["layer_roofline"], "stages": sm["stages"],
+            "staged_ms_per_step": round(r["staged_ms_per_step"], 4),
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
             "device_status": status,
             "next_rows": extra}
+    if layers is not None:
+        line["per_layer"] = layers
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(shape, inp, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(shape, generate(shape, device=dev), args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
@@ -576,8 +764,59 @@ def run_stage(args):
                       "timing": "back-to-back calls, CUDA events (launch gaps included)"}))
 
 
+def run_stage_ffn(args):
+    """The expert FFN (the two grouped GEMMs) alone: route, capacity and
+    dispatch once, then W warm-up calls and K calls of moe_expert_ffn between
+    CUDA events.  --experts E keeps the layer's per-expert GEMM shapes with E
+    experts (T scaled by E / E_layer)."""
+    import mixture_experts_layer_54_b200 as moe
+    from moe_inputs import shrink
+    device = torch.device("cuda", 0)
+    shape = CONFIGS[args.config]
+    if args.experts:
+        E = args.experts
+        shape = shrink(shape, E=E, T=max(shape.T * E // shape.E, 1), k=min(shape.k, E))
+    inp = generate(shape, device)
+    cfg = moe.moe_config(shape)
+    topk, gates, _, _, _ = moe.moe_route(cfg, inp.x, inp.W_r, inp.logit_bias, inp.select_bias)
+    cap = moe.moe_capacity(cfg, topk)
+    x_perm = moe.moe_dispatch(cfg, inp.x, topk, cap.pos, cap.keep, cap.offsets)
+    Y, Ysh, ws = moe.moe_expert_ffn(cfg, x_perm, cap.offsets, inp.W1, inp.W3, inp.W2, inp.x,
+                                    inp.Ws1, inp.Ws3, inp.Ws2)
+    call = lambda: moe.moe_expert_ffn(cfg, x_perm, cap.offsets, inp.W1, inp.W3, inp.W2, inp.x,
+                                      inp.Ws1, inp.Ws3, inp.Ws2, ws=ws, Y_perm=Y, Y_shared=Ysh)
+    for _ in range(max(args.warmup, 1)):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    if moe.moe_device_status(ws) != 0:
+        raise SystemExit("device status set: a bounded wait expired")
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    kept = int(cap.kept.sum().item())
+    work = layer_work(shape, None, kept, 0)["expert_ffn"]
+    peaks, _ = load_peaks()
+    w_bytes = sum(t.numel() * t.element_size() for t in
+                  (inp.W1, inp.W3, inp.W2, inp.Ws1, inp.Ws3, inp.Ws2) if t is not None)
+    print(json.dumps({"stage": "expert_ffn", "workload": workload_name(shape), "calls": args.steps,
+                      "us_per_call": round(us, 2), "kept_assignments": kept,
+                      "TFLOP/s": round(work["flops"] / us / 1e6, 1),
+                      "frac_of_burst": round(work["flops"] / us / 1e6 / peaks["bf16_tflops"], 3),
+                      "weight_bytes": w_bytes, "algorithmic_bytes": work["bytes"],
+                      "GB/s": round(work["bytes"] / us / 1e3, 1),
+                      "hbm_frac": round(work["bytes"] / us / 1e3 / peaks["hbm_gbs"], 3),
+                      "timing": "back-to-back calls, CUDA events (launch gaps included)"}))
+
+
 def main(argv=None):
     args = parse(argv)
+    if args.stage == "ffn":
+        run_stage_ffn(args)
+        return
     if args.stage:
         run_stage(args)
         return

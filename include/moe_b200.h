@@ -132,8 +132,9 @@ const char *moe_status_string(moe_status s);
 moe_status moe_validate(const moe_config *cfg);
 
 /* C = ceil(capacity_factor * T * k / E), computed in double on the host in
- * exactly that order of operations; T when the factor is +infinity
- * ("Lab 18" section 3).  Writes *C (host). */
+ * exactly that order of operations, held at T when it exceeds T (an expert
+ * receives at most T assignments, so that changes no decision); T when the
+ * factor is +infinity ("Lab 18" section 3).  Writes *C (host). */
 moe_status moe_capacity_value(const moe_config *cfg, int64_t *C);
 
 /* Rows the caller must allocate for the permuted buffers x_perm and Y_perm:
@@ -264,13 +265,15 @@ moe_status moe_capacity_scored(const moe_config *cfg, const int32_t *topk_idx,
  * another allocator that must not be bypassed).  The caller still allocates
  * and passes every input and output; the arguments mean what they mean for
  * moe_capacity, and the results are identical to it.
- *   - The scratch is a file-scope device array of 512 KiB (two tables of
+ *   - The scratch is a file-scope device array of 256 KiB (one table of
  *     65536 int32), held by every GPU that loads the library until the process
  *     exits.  Shapes that need more, ceil(T / 256) * k * E > 65536, return
  *     MOE_ERR_WORKSPACE and launch nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  The cached address is not
+ *     refreshed: cudaDeviceReset after the first call on a device is not
+ *     supported for this entry point.
  *   - No cudaMalloc, cudaFree or other allocating call is made.
  *   - All calls share the one array: calls whose work overlaps on the GPU
  *     (other streams, other threads) race and give wrong results.  Each call
@@ -288,22 +291,31 @@ moe_status moe_capacity_noalloc(const moe_config *cfg, const int32_t *topk_idx,
  *   x [T, d] dtype in; topk_idx, pos, keep, offsets from moe_capacity.
  *   x_perm [moe_perm_rows, d] dtype out: row offsets[e] + pos[t, j] = x[t] for
  *     every kept (t, j).  Padding rows are left untouched.
+ *   src_slot [moe_perm_rows] int32 out, nullable: entry offsets[e] + pos[t, j]
+ *     = t k + j (the assignment the row holds) for every kept (t, j); padding
+ *     entries are left untouched.  moe_expert_ffn_slots reads it.
+ *   zero_rows [T, d] dtype out, nullable: the row of every token with all its
+ *     slots dropped is set to zero (for a top-1 layer without shared experts
+ *     whose combine is moe_expert_ffn_slots writing y directly); other rows
+ *     are left untouched.
  */
 moe_status moe_dispatch(const moe_config *cfg, const void *x,
                         const int32_t *topk_idx, const int32_t *pos,
                         const uint8_t *keep, const int32_t *offsets,
-                        void *x_perm, moe_stream_t stream);
+                        void *x_perm, int32_t *src_slot, void *zero_rows,
+                        moe_stream_t stream);
 
 /*
- * moe_dispatch_rows - the dispatch as a row table, for moe_expert_ffn_gather
- * (the dispatch fused into the expert GEMM): src_rows[offsets[e] + pos[t, j]]
- * = t for every kept (t, j); every other row (segment padding) = 0.
- *   topk_idx, pos, keep, offsets from moe_capacity; src_rows [moe_perm_rows]
+ * moe_dispatch_rows - the dispatch as a row table only, for the expert GEMM
+ * that gathers its rows from x (moe_expert_ffn_gather, moe_expert_ffn_slots
+ * without x_perm): src_slot[offsets[e] + pos[t, j]] = t k + j for every kept
+ * (t, j) (the row is token t's); every other entry (segment padding) = -1.
+ *   topk_idx, pos, keep, offsets from moe_capacity; src_slot [moe_perm_rows]
  *   int32 out (device).  Moves T k small entries instead of the rows.
  */
 moe_status moe_dispatch_rows(const moe_config *cfg, const int32_t *topk_idx,
                              const int32_t *pos, const uint8_t *keep,
-                             const int32_t *offsets, int32_t *src_rows,
+                             const int32_t *offsets, int32_t *src_slot,
                              moe_stream_t stream);
 
 /*
@@ -329,19 +341,59 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm,
 
 /*
  * moe_expert_ffn_gather - moe_expert_ffn with the dispatch fused in: row r of
- * segment e is token src_rows[r] of x, read by GEMM1 straight from x (bf16:
- * TMA row gathers into each tile; fp32: indexed loads), so x_perm is never
- * written.  Results are those of moe_dispatch + moe_expert_ffn on the same
- * rows.
- *   x [T, d] dtype in; src_rows [moe_perm_rows] from moe_dispatch_rows;
+ * segment e is token src_slot[r] / k of x, read by GEMM1 straight from x
+ * (bf16: TMA row gathers into each tile; fp32: indexed loads), so x_perm is
+ * never written.  Results are those of moe_dispatch + moe_expert_ffn on the
+ * same rows.
+ *   x [T, d] dtype in; src_slot [moe_perm_rows] from moe_dispatch_rows;
  *   every other argument as for moe_expert_ffn.
  */
 moe_status moe_expert_ffn_gather(const moe_config *cfg, const void *x,
-                                 const int32_t *src_rows, const int32_t *offsets,
+                                 const int32_t *src_slot, const int32_t *offsets,
                                  const void *W1, const void *W3, const void *W2,
                                  const void *Ws1, const void *Ws3, const void *Ws2,
                                  void *Y_perm, void *Y_shared, void *ws,
                                  size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn_slots - moe_expert_ffn with the combine's gate fused into
+ * GEMM2's epilogue ("Lab 18" section 1, y = sum g_i FFN_i(x); section 3, a
+ * dropped slot contributes nothing): every kept row r of segment e, holding
+ * assignment a = src_slot[r] (token a / k, slot a % k), is written as
+ *     Y_slot[a] = gates[a] * FFN_e(row)      (rounded once to dtype)
+ * so the combine is left with a plain sum of a token's k contiguous rows
+ * (moe_combine_slots), or with nothing for k = 1 and no shared expert: there
+ * Y_slot may be y itself, and only the rows of tokens whose slot was dropped
+ * are left to fill (they are not written).
+ *   x_perm [moe_perm_rows, d]: the permuted rows (moe_dispatch), or NULL to
+ *     gather them from x through src_slot (moe_dispatch_rows) as
+ *     moe_expert_ffn_gather does.
+ *   x [T, d]: the tokens (required when x_perm is NULL or S > 0).
+ *   src_slot [moe_perm_rows] int32 (moe_dispatch or moe_dispatch_rows);
+ *   kept [E] int32 (moe_capacity): rows past kept[e] in segment e are padding.
+ *   gates [T, k] fp32 (moe_route).
+ *   Y_slot [T k, d] dtype out: rows of dropped assignments are not written.
+ *   Y_shared, ws and the weights as for moe_expert_ffn.
+ */
+moe_status moe_expert_ffn_slots(const moe_config *cfg, const void *x_perm, const void *x,
+                                const int32_t *src_slot, const int32_t *offsets,
+                                const int32_t *kept, const float *gates,
+                                const void *W1, const void *W3, const void *W2,
+                                const void *Ws1, const void *Ws3, const void *Ws2,
+                                void *Y_slot, void *Y_shared, void *ws, size_t ws_bytes,
+                                moe_stream_t stream);
+
+/*
+ * moe_combine_slots - the combine after moe_expert_ffn_slots ("Lab 18"
+ * section 1 and section 3):
+ *   y[t] = sum_{j = 0..k-1, keep[t, j]} Y_slot[t k + j] + Y_shared[t] (+ residual[t])
+ * summed in fp32 in that order and stored as dtype; the k rows of a token are
+ * contiguous.  A token with every slot dropped gets Y_shared[t] (or 0), plus
+ * the residual when given.  Y_shared: required when S > 0; residual nullable.
+ */
+moe_status moe_combine_slots(const moe_config *cfg, const void *Y_slot, const void *Y_shared,
+                             const uint8_t *keep, const void *residual, void *y,
+                             moe_stream_t stream);
 
 /*
  * moe_combine - gate-weighted sum plus shared experts ("Lab 18" section 1,
@@ -407,9 +459,17 @@ moe_status moe_bias_update(const moe_config *cfg, const int32_t *counts, float g
  * combine, losses ("Lab 18", MoE.forward row of "What to implement").
  *   x [T, d] dtype; weights; outputs as described at moe_outputs.
  *   ws: at least moe_workspace_size(cfg) bytes, 256-byte aligned.
- * Six kernel stages, no host synchronisation, safe to capture in a CUDA graph.
- * With MOE_PRIORITY_SCORE the router also writes its scores [T, E] to the
- * workspace and the capacity stage is moe_capacity_scored.
+ * The stages' kernels, no host synchronisation, safe to capture in a CUDA
+ * graph; each kernel is launched so that it may start while the previous one
+ * finishes (programmatic dependent launch) and waits for it on the device.
+ * The losses are computed inside the capacity launch, with the same
+ * fixed-order reduction as moe_losses (the same bits).  For k = 1 without
+ * shared experts the combine is fused into the expert GEMM (as
+ * moe_expert_ffn_slots writing y, the dispatch zeroing dropped tokens' rows),
+ * so y is g FFN(x) rounded once instead of twice.  With
+ * MOE_PRIORITY_SCORE the router also writes its scores [T, E] to the
+ * workspace, the capacity stage is moe_capacity_scored and the losses are a
+ * launch of their own.
  */
 moe_status moe_forward(const moe_config *cfg, const moe_weights *w,
                        const void *x, const moe_outputs *out, void *ws,

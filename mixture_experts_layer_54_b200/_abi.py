@@ -63,13 +63,16 @@ SIGNATURES = {
                                             _P, ctypes.c_size_t, _P]),
     "moe_seq_balance_loss": (ctypes.c_int, [_CFG, ctypes.c_int32, _P, _P, _P, _P, _P]),
     "moe_bias_update": (ctypes.c_int, [_CFG, _P, ctypes.c_float, _P, _P]),
-    "moe_dispatch": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_dispatch": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_rows": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn_gather": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                              _P, ctypes.c_size_t, _P]),
     "moe_expert_ffn": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]),
+    "moe_expert_ffn_slots": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                            _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_combine_slots": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
     "moe_losses": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_CFG, ctypes.POINTER(MoeWeights), _P,
                                    ctypes.POINTER(MoeOutputs), _P, ctypes.c_size_t, _P]),

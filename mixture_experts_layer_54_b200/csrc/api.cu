@@ -39,7 +39,11 @@ int64_t capacity_of(const moe_config &c)
 {
     if (isinf(c.capacity_factor))
         return c.T;
-    return (int64_t)ceil(c.capacity_factor * (double)((int64_t)c.T * c.k) / (double)c.E);
+    // A token's k experts are distinct, so an expert receives at most T
+    // assignments: any C >= T keeps them all.  Holding C at T changes no
+    // decision and keeps the conversion defined for huge finite factors.
+    const double C = ceil(c.capacity_factor * (double)((int64_t)c.T * c.k) / (double)c.E);
+    return C >= (double)c.T ? (int64_t)c.T : (int64_t)C;
 }
 
 int64_t perm_rows(const moe_config &c)
@@ -82,7 +86,6 @@ void carve_stage_into(const moe_config &c, Carver &cv, StageScratch &s)
     Carver route_cv{cv.base, off}, cap_cv{cv.base, off}, ffn_cv{cv.base, off};
     s.route = route_cv.take(route_scratch_bytes(c));
     s.hist = static_cast<int32_t *>(cap_cv.take(hk));
-    s.base = static_cast<int32_t *>(cap_cv.take(hk));
     s.count_base = static_cast<int32_t *>(cap_cv.take((size_t)c.E * 4));
     s.keys = static_cast<unsigned long long *>(
         cap_cv.take(c.priority == MOE_PRIORITY_SCORE ? (size_t)c.T * c.k * 8 : 0));
@@ -94,7 +97,7 @@ void carve_stage_into(const moe_config &c, Carver &cv, StageScratch &s)
 }
 
 struct ForwardBufs {
-    int32_t *topk, *counts, *kept, *offsets, *n_dropped, *pos;
+    int32_t *topk, *counts, *kept, *offsets, *n_dropped, *pos, *slot;
     float *gates, *partials, *scores;
     uint8_t *keep, *dropped;
     void *x_perm, *Y_perm, *Y_sh;
@@ -121,6 +124,7 @@ void carve_forward_into(const moe_config &c, Carver &cv, ForwardBufs &f)
     f.x_perm = cv.take((size_t)R * c.d * esz);
     f.Y_perm = cv.take((size_t)R * c.d * esz);
     f.Y_sh = c.n_shared > 0 ? cv.take((size_t)c.T * c.d * esz) : nullptr;
+    f.slot = static_cast<int32_t *>(cv.take((size_t)R * 4));   // row -> assignment
 }
 
 }  // namespace
@@ -237,17 +241,18 @@ moe_status route_impl(const moe_config *cfg, const void *x, const float *W_r,
     if (ws_bytes < stage_scratch_bytes(*cfg))
         return MOE_ERR_WORKSPACE;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    if (clear_status && cudaMemsetAsync(ws, 0, sizeof(int32_t), cs) != cudaSuccess)
-        return MOE_ERR_CUDA;
     const RoutePlan plan = route_plan(*cfg);
     if (plan.tensor_cores) {
         if (!aligned16(x))
             return MOE_ERR_ALIGN;
+        // the router's first kernel clears the status word itself
         StageScratch s = carve_stage(*cfg, ws);
         return cuda_status(launch_route_tc(*cfg, x, W_r, logit_bias, select_bias, topk_idx,
                                            gates, loss_partials, logits_out, scores_out, s.route,
-                                           s.status, cs));
+                                           s.status, clear_status, cs));
     }
+    if (clear_status && cudaMemsetAsync(ws, 0, sizeof(int32_t), cs) != cudaSuccess)
+        return MOE_ERR_CUDA;
     return cuda_status(launch_route(*cfg, x, W_r, logit_bias, select_bias, topk_idx, gates,
                                     loss_partials, logits_out, scores_out, cs));
 }
@@ -282,7 +287,7 @@ moe_status moe_capacity(const moe_config *cfg, const int32_t *topk_idx, int32_t 
         return MOE_ERR_WORKSPACE;
     StageScratch s = carve_stage(*cfg, ws);
     return cuda_status(launch_capacity(*cfg, capacity_of(*cfg), topk_idx, counts, pos, keep, kept,
-                                       offsets, dropped, n_dropped, s.hist, s.base,
+                                       offsets, dropped, n_dropped, s.hist,
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -313,7 +318,7 @@ moe_status moe_capacity_sharded(const moe_config *cfg, int64_t capacity,
     if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     return cuda_status(launch_capacity(*cfg, capacity, topk_idx, counts, pos, keep, kept, offsets,
-                                       dropped, n_dropped, s.hist, s.base, cs, s.count_base));
+                                       dropped, n_dropped, s.hist, cs, s.count_base));
 }
 
 moe_status moe_capacity_scored(const moe_config *cfg, const int32_t *topk_idx,
@@ -336,26 +341,26 @@ moe_status moe_capacity_scored(const moe_config *cfg, const int32_t *topk_idx,
     StageScratch s = carve_stage(*cfg, ws);
     return cuda_status(launch_capacity_scored(*cfg, capacity_of(*cfg), topk_idx, scores, counts,
                                               pos, keep, kept, offsets, dropped, n_dropped,
-                                              s.hist, s.base, s.keys,
+                                              s.hist, s.keys,
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_dispatch_rows(const moe_config *cfg, const int32_t *topk_idx, const int32_t *pos,
-                             const uint8_t *keep, const int32_t *offsets, int32_t *src_rows,
+                             const uint8_t *keep, const int32_t *offsets, int32_t *src_slot,
                              moe_stream_t stream)
 {
     moe_status st = check_cfg(cfg);
     if (st != MOE_OK)
         return st;
-    if (!offsets || !src_rows || (cfg->T > 0 && (!topk_idx || !pos || !keep)))
+    if (!offsets || !src_slot || (cfg->T > 0 && (!topk_idx || !pos || !keep)))
         return MOE_ERR_NULL;
-    return cuda_status(launch_dispatch_rows(*cfg, topk_idx, pos, keep, offsets, src_rows,
+    return cuda_status(launch_dispatch_rows(*cfg, topk_idx, pos, keep, offsets, src_slot,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_idx,
                         const int32_t *pos, const uint8_t *keep, const int32_t *offsets,
-                        void *x_perm, moe_stream_t stream)
+                        void *x_perm, int32_t *src_slot, void *zero_rows, moe_stream_t stream)
 {
     moe_status st = check_cfg(cfg);
     if (st != MOE_OK)
@@ -364,20 +369,25 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *top
         return MOE_OK;
     if (!x || !topk_idx || !pos || !keep || !offsets || !x_perm)
         return MOE_ERR_NULL;
-    if (!aligned16(x) || !aligned16(x_perm))
+    if (!aligned16(x) || !aligned16(x_perm) || (zero_rows && !aligned16(zero_rows)))
         return MOE_ERR_ALIGN;
     return cuda_status(launch_dispatch(*cfg, x, topk_idx, pos, keep, offsets, x_perm,
-                                       reinterpret_cast<cudaStream_t>(stream)));
+                                       reinterpret_cast<cudaStream_t>(stream), src_slot,
+                                       zero_rows));
 }
 
 namespace {
 
+// x_perm NULL: routed rows gathered from x through src_slot.  slot_out
+// non-NULL: GEMM2 writes gates[a] * FFN(row) to row a of slot_out (src_slot,
+// kept, gates required) instead of Y_perm.
 moe_status expert_ffn_impl(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
-                           const int32_t *src_rows, const void *W1, const void *W3,
+                           const int32_t *src_slot, const void *W1, const void *W3,
                            const void *W2, const void *x, const void *Ws1, const void *Ws3,
                            const void *Ws2, void *Y_perm,
                            void *Y_shared, void *ws, size_t ws_bytes, moe_stream_t stream,
-                           bool clear_status)
+                           bool clear_status, const int32_t *kept = nullptr,
+                           const float *gates = nullptr, void *slot_out = nullptr)
 {
     moe_status st = check_cfg(cfg);
     if (st != MOE_OK)
@@ -385,13 +395,15 @@ moe_status expert_ffn_impl(const moe_config *cfg, const void *x_perm, const int3
     const moe_config &c = *cfg;
     const bool swiglu = c.act == MOE_ACT_SWIGLU;
     const bool shared = c.n_shared > 0;
-    if (!offsets || !W1 || !W2 || !Y_perm || !ws || (swiglu && !W3))
+    if (!offsets || !W1 || !W2 || !ws || (swiglu && !W3) || (!slot_out && !Y_perm))
         return MOE_ERR_NULL;
-    if (src_rows ? (c.T > 0 && !x) : !x_perm)   // routed rows: gathered from x, or x_perm
+    if (!x_perm && (!src_slot || (c.T > 0 && !x)))   // routed rows: x_perm, or gathered from x
+        return MOE_ERR_NULL;
+    if (slot_out && (!src_slot || !kept || !gates))
         return MOE_ERR_NULL;
     if (shared && (!x || !Ws1 || !Ws2 || !Y_shared || (swiglu && !Ws3)))
         return MOE_ERR_NULL;
-    const void *ptrs[] = {x_perm, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm, Y_shared};
+    const void *ptrs[] = {x_perm, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm, Y_shared, slot_out};
     for (const void *p : ptrs)
         if (p && !aligned16(p))
             return MOE_ERR_ALIGN;
@@ -402,15 +414,17 @@ moe_status expert_ffn_impl(const moe_config *cfg, const void *x_perm, const int3
     StageScratch s = carve_stage(c, ws);
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (clear_status && cudaMemsetAsync(s.status, 0, sizeof(int32_t), cs) != cudaSuccess)
+    // bf16: GEMM1 clears the status word itself before any of its waits
+    if (clear_status && c.dtype != MOE_DTYPE_BF16 &&
+        cudaMemsetAsync(s.status, 0, sizeof(int32_t), cs) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (c.dtype == MOE_DTYPE_BF16)
-        e = launch_ffn_tcgen05(c, x_perm, offsets, src_rows, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
-                               Y_shared, s.H, s.H_sh, s.status, cs);
+        e = launch_ffn_tcgen05(c, x_perm, offsets, src_slot, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
+                               Y_shared, s.H, s.H_sh, s.status, clear_status, cs, kept, gates,
+                               slot_out);
     else
-        e = launch_ffn_simt(c, x_perm, offsets, src_rows, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
-                            Y_shared,
-                            s.H, s.H_sh, cs);
+        e = launch_ffn_simt(c, x_perm, offsets, src_slot, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
+                            Y_shared, s.H, s.H_sh, cs, kept, gates, slot_out);
     return cuda_status(e);
 }
 
@@ -425,16 +439,48 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32
                            Y_shared, ws, ws_bytes, stream, true);
 }
 
-moe_status moe_expert_ffn_gather(const moe_config *cfg, const void *x, const int32_t *src_rows,
+moe_status moe_expert_ffn_gather(const moe_config *cfg, const void *x, const int32_t *src_slot,
                                  const int32_t *offsets, const void *W1, const void *W3,
                                  const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
                                  void *Y_perm, void *Y_shared, void *ws, size_t ws_bytes,
                                  moe_stream_t stream)
 {
-    if (!src_rows)
+    if (!src_slot)
         return MOE_ERR_NULL;
-    return expert_ffn_impl(cfg, nullptr, offsets, src_rows, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
+    return expert_ffn_impl(cfg, nullptr, offsets, src_slot, W1, W3, W2, x, Ws1, Ws3, Ws2, Y_perm,
                            Y_shared, ws, ws_bytes, stream, true);
+}
+
+moe_status moe_expert_ffn_slots(const moe_config *cfg, const void *x_perm, const void *x,
+                                const int32_t *src_slot, const int32_t *offsets,
+                                const int32_t *kept, const float *gates, const void *W1,
+                                const void *W3, const void *W2, const void *Ws1, const void *Ws3,
+                                const void *Ws2, void *Y_slot, void *Y_shared, void *ws,
+                                size_t ws_bytes, moe_stream_t stream)
+{
+    if (!src_slot || !kept || !gates || !Y_slot)
+        return MOE_ERR_NULL;
+    return expert_ffn_impl(cfg, x_perm, offsets, src_slot, W1, W3, W2, x, Ws1, Ws3, Ws2, nullptr,
+                           Y_shared, ws, ws_bytes, stream, true, kept, gates, Y_slot);
+}
+
+moe_status moe_combine_slots(const moe_config *cfg, const void *Y_slot, const void *Y_shared,
+                             const uint8_t *keep, const void *residual, void *y,
+                             moe_stream_t stream)
+{
+    moe_status st = check_cfg(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (cfg->T == 0)
+        return MOE_OK;
+    if (!Y_slot || !keep || !y || (cfg->n_shared > 0 && !Y_shared))
+        return MOE_ERR_NULL;
+    const void *ptrs[] = {Y_slot, Y_shared, residual, y};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return MOE_ERR_ALIGN;
+    return cuda_status(launch_combine_slots(*cfg, Y_slot, Y_shared, keep, residual, y,
+                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine(const moe_config *cfg, const void *Y_perm, const void *Y_shared,
@@ -527,28 +573,49 @@ moe_status moe_forward(const moe_config *cfg, const moe_weights *w, const void *
     if (out->counts) f.counts = out->counts;
     if (out->n_dropped) f.n_dropped = out->n_dropped;
     const size_t ssz = stage_scratch_bytes(c);
-    if ((st = moe_clear_device_status(ws, stream)) != MOE_OK)
+    if (c.T == 0 && (st = moe_clear_device_status(ws, stream)) != MOE_OK)
         return st;
     const bool scored = c.priority == MOE_PRIORITY_SCORE;
+    // the router clears the status word once for the whole layer
     if ((st = route_impl(cfg, x, w->W_r, w->logit_bias, w->select_bias, f.topk, f.gates,
                          f.partials, nullptr, scored ? f.scores : nullptr, ws, ssz, stream,
-                         false)) != MOE_OK)
+                         true)) != MOE_OK)
         return st;
-    st = scored ? moe_capacity_scored(cfg, f.topk, f.scores, f.counts, f.pos, f.keep, f.kept,
-                                      f.offsets, f.dropped, f.n_dropped, ws, ssz, stream)
-                : moe_capacity(cfg, f.topk, f.counts, f.pos, f.keep, f.kept, f.offsets, f.dropped,
-                               f.n_dropped, ws, ssz, stream);
+    if (scored)
+        st = moe_capacity_scored(cfg, f.topk, f.scores, f.counts, f.pos, f.keep, f.kept,
+                                 f.offsets, f.dropped, f.n_dropped, ws, ssz, stream);
+    else   // token or rank order: the capacity launch also writes the two losses
+        st = cuda_status(launch_capacity(c, capacity_of(c), f.topk, f.counts, f.pos, f.keep,
+                                         f.kept, f.offsets, f.dropped, f.n_dropped, s.hist,
+                                         reinterpret_cast<cudaStream_t>(stream), nullptr,
+                                         f.partials, out->aux, out->zloss));
     if (st != MOE_OK)
         return st;
-    if ((st = moe_dispatch(cfg, x, f.topk, f.pos, f.keep, f.offsets, f.x_perm, stream)) != MOE_OK)
-        return st;
-    if ((st = expert_ffn_impl(cfg, f.x_perm, f.offsets, nullptr, w->W1, w->W3, w->W2, x, w->Ws1,
-                              w->Ws3, w->Ws2, f.Y_perm, f.Y_sh, ws, ssz, stream, false)) != MOE_OK)
-        return st;
-    if ((st = moe_combine(cfg, f.Y_perm, f.Y_sh, f.gates, f.topk, f.pos, f.keep, f.offsets,
-                          nullptr, out->y, stream)) != MOE_OK)
-        return st;
-    return moe_losses(cfg, f.counts, f.partials, out->aux, out->zloss, stream);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (c.k == 1 && c.n_shared == 0) {
+        // one slot per token and no shared expert: the combine is the gate,
+        // applied in GEMM2's epilogue, which writes y's rows directly; the
+        // dispatch records each row's assignment and zeroes dropped tokens' y
+        if ((st = cuda_status(launch_dispatch(c, x, f.topk, f.pos, f.keep, f.offsets, f.x_perm, cs,
+                                              f.slot, out->y))) != MOE_OK)
+            return st;
+        if ((st = expert_ffn_impl(cfg, f.x_perm, f.offsets, f.slot, w->W1, w->W3, w->W2, x,
+                                  w->Ws1, w->Ws3, w->Ws2, nullptr, nullptr, ws, ssz, stream,
+                                  false, f.kept, f.gates, out->y)) != MOE_OK)
+            return st;
+    } else {
+        if ((st = cuda_status(launch_dispatch(c, x, f.topk, f.pos, f.keep, f.offsets, f.x_perm,
+                                              cs))) != MOE_OK)
+            return st;
+        if ((st = expert_ffn_impl(cfg, f.x_perm, f.offsets, nullptr, w->W1, w->W3, w->W2, x,
+                                  w->Ws1, w->Ws3, w->Ws2, f.Y_perm, f.Y_sh, ws, ssz, stream,
+                                  false)) != MOE_OK)
+            return st;
+        if ((st = moe_combine(cfg, f.Y_perm, f.Y_sh, f.gates, f.topk, f.pos, f.keep, f.offsets,
+                              nullptr, out->y, stream)) != MOE_OK)
+            return st;
+    }
+    return scored ? moe_losses(cfg, f.counts, f.partials, out->aux, out->zloss, stream) : MOE_OK;
 }
 
 moe_status moe_device_status(const void *ws, int32_t *status, moe_stream_t stream)

@@ -7,16 +7,17 @@
 // where to start step 4 (first come first served in token order).
 //
 // The sequential definition is a walk over the T*k assignments in priority
-// order with one counter per expert.  It is computed here in three launches:
+// order with one counter per expert.  It is computed here in two launches:
 //   count  - each block of 256 tokens histograms its assignments per (rank j,
 //            expert e) in shared memory (integer atomics, order-free);
-//   scan   - one block turns the histograms into, for every block, the number
-//            of assignments to each expert that come before the block in
-//            priority order, plus counts, kept, offsets and the drop total;
-//   place  - each warp of a block walks its 32 tokens' assignments in
-//            priority order, 32 at a time, ranking equal experts with
-//            __match_any_sync; one scan over the block's warps gives each
-//            warp's start per expert.
+//   place  - each block sums the histograms of the blocks before it (and,
+//            rank-major, all blocks' lower ranks): the number of assignments
+//            to each expert that come before the block in priority order;
+//            then each warp walks its 32 tokens' assignments in priority
+//            order, 32 at a time, ranking equal experts with __match_any_sync,
+//            after one scan over the block's warps has given each warp its
+//            start per expert.  One more block computes counts, kept, offsets
+//            and the drop total (and, for the whole forward, the losses).
 // Integers only, so the result is bit-exact with the sequential walk.
 //
 // Batch-prioritized order ("Lab 18" section 3, V-MoE: assignments ranked by
@@ -33,6 +34,7 @@
 //            memory in tiles;
 //   drop   - a token is dropped when none of its k slots was kept.
 #include "internal.cuh"
+#include "losses_common.cuh"
 
 namespace moe {
 namespace {
@@ -45,6 +47,8 @@ __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int 
     extern __shared__ int32_t h[];   // [k][E]
     for (int i = threadIdx.x; i < k * E; i += CT)
         h[i] = 0;
+    pdl_wait();   // topk comes from the router
+    pdl_trigger();
     __syncthreads();
     const int t = blockIdx.x * CT + threadIdx.x;
     if (t < T) {
@@ -59,40 +63,53 @@ __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int 
         hist[(int64_t)blockIdx.x * k * E + i] = h[i];
 }
 
-__global__ void __launch_bounds__(1024)
-cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int priority,
-                long long C, const int32_t *__restrict__ count_base, int32_t *__restrict__ base,
-                int32_t *__restrict__ counts, int32_t *__restrict__ kept,
-                int32_t *__restrict__ offsets, int32_t *__restrict__ n_dropped)
+// Column sums of the per-block histograms [nblk][cols]: before[col] = blocks
+// [0, upto), and (total != nullptr) total[col] = all blocks; BATCH loads of a
+// column in flight per thread.
+__device__ __forceinline__ void hist_sums(const int32_t *__restrict__ hist, int nblk, int cols,
+                                          int upto, int32_t *before, int32_t *total)
 {
-    constexpr int BATCH = 32;   // blocks' histogram entries in flight per column
-    __shared__ int32_t total[kMaxK * kMaxE];   // per (j, e), all blocks
-    __shared__ int32_t cnt[kMaxE];
-    __shared__ int32_t kept_s[kMaxE];
-    __shared__ long long drop_w[32];
-    const int cols = k * E;
-    // exclusive scan over blocks of each (j, e) column, BATCH loads at a time
+    constexpr int BATCH = 16;
+    const int end = total ? nblk : upto;
     for (int col = threadIdx.x; col < cols; col += blockDim.x) {
-        int run = 0;
-        for (int b0 = 0; b0 < nblk; b0 += BATCH) {
+        int bsum = 0, tsum = 0;
+        for (int b0 = 0; b0 < end; b0 += BATCH) {
             int v[BATCH];
 #pragma unroll
             for (int i = 0; i < BATCH; ++i)
-                v[i] = b0 + i < nblk ? hist[(int64_t)(b0 + i) * cols + col] : 0;
+                v[i] = b0 + i < end ? hist[(int64_t)(b0 + i) * cols + col] : 0;
 #pragma unroll
             for (int i = 0; i < BATCH; ++i) {
-                if (b0 + i < nblk)
-                    base[(int64_t)(b0 + i) * cols + col] = run;
-                run += v[i];
+                bsum += b0 + i < upto ? v[i] : 0;
+                tsum += v[i];
             }
         }
-        total[col] = run;
+        before[col] = bsum;
+        if (total)
+            total[col] = tsum;
     }
+}
+
+// The block after the placement blocks: counts, kept, the padded segment
+// offsets and the drop total from the histograms of all blocks; with
+// partials, also the two balancing losses (the forward's losses stage, in the
+// same fixed order as moe_losses).
+__device__ void capacity_totals(const int32_t *__restrict__ hist, int nblk, int k, int E,
+                                long long C, const int32_t *__restrict__ count_base, int T,
+                                int32_t *__restrict__ counts, int32_t *__restrict__ kept,
+                                int32_t *__restrict__ offsets, int32_t *__restrict__ n_dropped,
+                                const float *partials, int prows, float *aux, float *zloss,
+                                int32_t *colsum)
+{
+    __shared__ int32_t cnt[kMaxE];
+    __shared__ int32_t kept_s[kMaxE];
+    __shared__ double term[kMaxE + 1];
+    hist_sums(hist, nblk, k * E, nblk, colsum, nullptr);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int s = 0;
         for (int j = 0; j < k; ++j)
-            s += total[j * E + e];
+            s += colsum[j * E + e];
         // slots left for this batch: C, less what earlier shards of the same
         // global batch already took (count_base, sharded capacity only)
         long long room = C - (count_base ? (long long)count_base[e] : 0LL);
@@ -104,32 +121,6 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
         kept[e] = kv;
     }
     __syncthreads();
-    if (priority == MOE_PRIORITY_TOKEN) {
-        // assignments to e in earlier blocks, any rank: stored in the j = 0
-        // slot (every slot of the item read before it is written)
-        for (int i = threadIdx.x; i < nblk * E; i += blockDim.x) {
-            const int b = i / E, e = i % E;
-            int v[kMaxK];
-#pragma unroll
-            for (int j = 0; j < kMaxK; ++j)
-                v[j] = j < k ? base[(int64_t)b * cols + j * E + e] : 0;
-            int s = 0;
-#pragma unroll
-            for (int j = 0; j < kMaxK; ++j)
-                s += v[j];
-            base[(int64_t)b * cols + e] = s;
-        }
-    } else {
-        // rank-major: every rank j' < j of all tokens comes first
-        for (int i = threadIdx.x; i < nblk * cols; i += blockDim.x) {
-            int col = i % cols;
-            int j = col / E, e = col % E;
-            int s = 0;
-            for (int jj = 0; jj < j; ++jj)
-                s += total[jj * E + e];
-            base[i] += s;
-        }
-    }
     // segment offsets: kept counts rounded up to MOE_ROW_ALIGN, exclusive scan
     // by one warp; the drop total summed in a fixed order
     if (threadIdx.x < 32) {
@@ -155,16 +146,16 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
                 offsets[e] = carry + incl - padded;
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        drop_w[lane] = drop;
-        __syncwarp();
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            drop += __shfl_xor_sync(0xffffffffu, drop, o);
         if (lane == 0) {
-            long long d = 0;
-            for (int l = 0; l < 32; ++l)
-                d += drop_w[l];
             offsets[E] = carry;
-            *n_dropped = (int32_t)d;
+            *n_dropped = (int32_t)drop;
         }
     }
+    if (partials)
+        block_losses(cnt, partials, prows, T > 0 ? T : 1, k, E, aux, zloss, term);
 }
 
 // Each warp owns 32 consecutive tokens of the block.  Per pass (token order:
@@ -173,20 +164,56 @@ cap_scan_kernel(const int32_t *__restrict__ hist, int nblk, int k, int E, int pr
 // turns the counts into each warp's start inside the block; (C) the warp walks
 // its assignments in priority order, 32 at a time, ranking equal experts with
 // __match_any_sync and keeping its own running count per expert.
+//
+// Each block first takes its bases from the histograms: token order, the
+// assignments to e of earlier blocks (any rank); rank-major, those of rank j
+// in earlier blocks plus every assignment of a lower rank.  Block nblk
+// computes the totals instead (capacity_totals).
 __global__ void __launch_bounds__(CT)
-cap_place_kernel(const int32_t *topk, int T, int k, int E, int priority, long long C,
-                 const int32_t *count_base, const int32_t *base, int32_t *pos, uint8_t *keep,
-                 uint8_t *dropped)
+cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int priority, long long C,
+                 const int32_t *__restrict__ count_base, const int32_t *__restrict__ hist,
+                 int nblk, int32_t *__restrict__ pos, uint8_t *__restrict__ keep,
+                 uint8_t *__restrict__ dropped, int32_t *__restrict__ counts,
+                 int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
+                 int32_t *__restrict__ n_dropped, const float *partials, int prows, float *aux,
+                 float *zloss)
 {
     __shared__ int32_t wrun[CT / 32][kMaxE];
     __shared__ uint8_t keep_s[CT * kMaxK];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int32_t before[kMaxK * kMaxE], total[kMaxK * kMaxE];
+    pdl_wait();   // topk from the router, the histograms from cap_count
+    pdl_trigger();
     const int cols = k * E;
-    const int32_t *bb = base + (int64_t)blockIdx.x * cols;
+    if (blockIdx.x == nblk) {
+        capacity_totals(hist, nblk, k, E, C, count_base, T, counts, kept, offsets, n_dropped,
+                        partials, prows, aux, zloss, before);
+        return;
+    }
+    const bool token_order = priority == MOE_PRIORITY_TOKEN;
+    hist_sums(hist, nblk, cols, blockIdx.x, before, token_order ? nullptr : total);
+    __syncthreads();
+    if (token_order) {
+        for (int e = threadIdx.x; e < E; e += CT) {
+            int s = 0;
+            for (int j = 0; j < k; ++j)
+                s += before[j * E + e];
+            total[e] = s;   // base of expert e (any rank)
+        }
+    } else {
+        for (int col = threadIdx.x; col < cols; col += CT) {
+            const int j = col / E, e = col % E;
+            int s = 0;
+            for (int jj = 0; jj < j; ++jj)
+                s += total[jj * E + e];
+            before[col] += s;
+        }
+    }
+    __syncthreads();
+    const int32_t *bb = token_order ? total : before;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int tw = blockIdx.x * CT + warp * 32;   // this warp's first token
     const int nw = max(0, min(32, T - tw));       // its tokens
-    const bool token_order = priority == MOE_PRIORITY_TOKEN;
     const int passes = token_order ? 1 : k;
     for (int p = 0; p < passes; ++p) {
         const int len = token_order ? nw * k : nw;
@@ -363,14 +390,14 @@ cudaError_t launch_capacity_scored(const moe_config &c, int64_t C, const int32_t
                                    const float *scores, int32_t *counts, int32_t *pos,
                                    uint8_t *keep, int32_t *kept, int32_t *offsets,
                                    uint8_t *dropped, int32_t *n_dropped, int32_t *hist,
-                                   int32_t *base, unsigned long long *keys, cudaStream_t s)
+                                   unsigned long long *keys, cudaStream_t s)
 {
     // token order first: counts, kept, offsets, drop total, and each
     // assignment's place in its expert's list (written to pos, then replaced)
     moe_config tok = c;
     tok.priority = MOE_PRIORITY_TOKEN;
     cudaError_t err = launch_capacity(tok, C, topk, counts, pos, keep, kept, offsets, dropped,
-                                      n_dropped, hist, base, s);
+                                      n_dropped, hist, s);
     if (err != cudaSuccess || c.T == 0)
         return err;
     const int64_t A = (int64_t)c.T * c.k;
@@ -410,24 +437,21 @@ cudaError_t launch_shard_base(const moe_config &c, const int32_t *shard_counts, 
 cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep, int32_t *kept,
                             int32_t *offsets, uint8_t *dropped, int32_t *n_dropped,
-                            int32_t *hist, int32_t *base, cudaStream_t s,
-                            const int32_t *count_base)
+                            int32_t *hist, cudaStream_t s, const int32_t *count_base,
+                            const float *partials, float *aux, float *zloss)
 {
     const int nblk = cap_blocks(c);
     if (nblk > 0) {
-        cap_count_kernel<<<nblk, CT, sizeof(int32_t) * c.k * c.E, s>>>(topk, c.T, c.k, c.E, hist);
-        cudaError_t err = cudaGetLastError();
+        cudaError_t err = launch_pdl(cap_count_kernel, dim3(nblk), dim3(CT),
+                                     sizeof(int32_t) * c.k * c.E, s, topk, c.T, c.k, c.E, hist);
         if (err != cudaSuccess)
             return err;
     }
-    cap_scan_kernel<<<1, 1024, 0, s>>>(hist, nblk, c.k, c.E, c.priority, (long long)C, count_base,
-                                       base, counts, kept, offsets, n_dropped);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess || nblk == 0)
-        return err;
-    cap_place_kernel<<<nblk, CT, 0, s>>>(topk, c.T, c.k, c.E, c.priority, (long long)C, count_base,
-                                         base, pos, keep, dropped);
-    return cudaGetLastError();
+    // placement blocks, then the totals block (and the losses when asked)
+    return launch_pdl(cap_place_kernel, dim3(nblk + 1), dim3(CT), 0, s, topk, c.T, c.k, c.E,
+                      c.priority, (long long)C, count_base, (const int32_t *)hist, nblk, pos,
+                      keep, dropped, counts, kept, offsets, n_dropped, partials, partial_rows(c),
+                      aux, zloss);
 }
 
 }  // namespace moe

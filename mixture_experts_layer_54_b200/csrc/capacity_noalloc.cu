@@ -9,7 +9,7 @@
 // inputs and outputs; only the stage's scratch moves into the library.
 //
 // The scratch is a file-scope __device__ array, so every GPU that loads the
-// library holds it (512 KiB) until the process exits.  In host code the
+// library holds it (256 KiB) until the process exits.  In host code the
 // array's name is only a host-side stand-in for the symbol, never a device
 // address: the device address is looked up with cudaGetSymbolAddress once per
 // device, with that device current, and cached.
@@ -19,9 +19,10 @@
 
 namespace {
 
-// two int32 tables (per-block histograms and their scanned bases), back to back
+// one int32 table: the per-block histograms, one entry per (block of 256
+// tokens, rank, expert)
 constexpr int64_t kTableInts = 65536;
-static __device__ __align__(256) int32_t g_capacity_scratch[2 * kTableInts];
+static __device__ __align__(256) int32_t g_capacity_scratch[kTableInts];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
@@ -67,17 +68,16 @@ extern "C" moe_status moe_capacity_noalloc(const moe_config *cfg, const int32_t 
     if (!counts || !kept || !offsets || !n_dropped ||
         (c.T > 0 && (!topk_idx || !pos || !keep || !dropped)))
         return MOE_ERR_NULL;
-    // each table holds one int32 per (token block of 256, rank, expert)
+    // the table holds one int32 per (token block of 256, rank, expert)
     if ((int64_t)moe::cap_blocks(c) * c.k * c.E > kTableInts)
         return MOE_ERR_WORKSPACE;
     int32_t *scratch = nullptr;
     if (scratch_on_current_device(&scratch) != cudaSuccess)
         return MOE_ERR_CUDA;
-    // Both tables are written in full by this call before they are read, so
-    // whatever an earlier call left in them does not matter.
+    // The table is written in full by this call before it is read, so
+    // whatever an earlier call left in it does not matter.
     cudaError_t err = moe::launch_capacity(c, moe::capacity_of(c), topk_idx, counts, pos, keep,
                                            kept, offsets, dropped, n_dropped, scratch,
-                                           scratch + kTableInts,
                                            reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

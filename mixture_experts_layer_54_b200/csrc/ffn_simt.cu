@@ -37,7 +37,12 @@ struct SimtGemm {
     float *C;
     int64_t ldc;
     int64_t c_group_col;         // dense, blockIdx.z = group: C column offset per group
-    const int32_t *a_rows;       // non-null: row r of A is row a_rows[r] of the A tensor
+    const int32_t *a_slot;       // non-null: row r of A is row a_slot[r] / a_div of the A
+    int a_div;                   // tensor (a_slot[r] = assignment t k + j, -1 = none)
+    // non-null: the combine's gate fused (routed GEMM2): kept row r of group e
+    // (r - offsets[e] < kept[e]) goes, times gates[a], to row a = a_slot[r] of C
+    const int32_t *kept;
+    const float *gates;
 };
 
 __device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
@@ -82,7 +87,11 @@ __global__ void __launch_bounds__(THREADS) simt_gemm_kernel(SimtGemm p)
             for (int i = threadIdx.x; i < TILE * KC; i += THREADS) {
                 int r = i / KC, c = i % KC;
                 int row = m0 + r, kk = k0 + c, n = n0 + r;
-                const int64_t arow = (row < row_end && p.a_rows) ? p.a_rows[row] : row;
+                int64_t arow = row;
+                if (row < row_end && p.a_slot && !p.kept) {
+                    const int a = p.a_slot[row];
+                    arow = a >= 0 ? a / p.a_div : 0;
+                }
                 As[r][c] = (row < row_end && kk < p.Kg) ? p.A[arow * p.lda + a_col0 + kk] : 0.f;
                 Bs[r][c] = (n < p.N && kk < p.Kg) ? B[(int64_t)n * p.Kg + kk] : 0.f;
                 if (ACT == ACT_SWIGLU)
@@ -118,7 +127,14 @@ __global__ void __launch_bounds__(THREADS) simt_gemm_kernel(SimtGemm p)
             v = gelu_erf(v);
         else if (ACT == ACT_SWIGLU)
             v = v / (1.f + expf(-v)) * acc3[i];
-        p.C[(int64_t)row * p.ldc + col] = v;
+        if (p.kept) {   // gated: to the assignment's row, kept rows only
+            if (row - p.offsets[group] >= p.kept[group])
+                continue;
+            const int a = p.a_slot[row];
+            p.C[(int64_t)a * p.ldc + col] = p.gates[a] * v;
+        } else {
+            p.C[(int64_t)row * p.ldc + col] = v;
+        }
     }
 }
 
@@ -139,25 +155,28 @@ cudaError_t run(const SimtGemm &p, int act, int grid_m, int grid_z, cudaStream_t
 }  // namespace
 
 cudaError_t launch_ffn_simt(const moe_config &c, const void *x_perm, const int32_t *offsets,
-                            const int32_t *src_rows, const void *W1, const void *W3, const void *W2, const void *x,
-                            const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
-                            void *Y_sh, void *H, void *H_sh, cudaStream_t s)
+                            const int32_t *src_slot, const void *W1, const void *W3, const void *W2,
+                            const void *x, const void *Ws1, const void *Ws3, const void *Ws2,
+                            void *Y_perm, void *Y_sh, void *H, void *H_sh, cudaStream_t s,
+                            const int32_t *kept, const float *gates, void *slot_out)
 {
     const int act1 = c.act == MOE_ACT_SWIGLU ? ACT_SWIGLU : ACT_GELU;
     const int R = (int)perm_rows(c);
     const int gm = (int)ceil_div(R, TILE);
     cudaError_t err;
-    // routed GEMM1: H = act(x_perm W1^T), or with src_rows the rows of x
-    SimtGemm g1{static_cast<const float *>(src_rows ? x : x_perm), c.d, 0, offsets, c.E,
+    // routed GEMM1: H = act(x_perm W1^T), or without x_perm the rows of x
+    // through src_slot
+    SimtGemm g1{static_cast<const float *>(x_perm ? x_perm : x), c.d, 0, offsets, c.E,
                 static_cast<const float *>(W1), static_cast<const float *>(W3),
                 (int64_t)c.d_ff * c.d, c.d_ff, c.d, 1, static_cast<float *>(H), c.d_ff, 0,
-                src_rows};
+                x_perm ? nullptr : src_slot, c.k};
     if ((err = run(g1, act1, gm, 1, s)) != cudaSuccess)
         return err;
-    // routed GEMM2: Y_perm = H W2^T
+    // routed GEMM2: Y_perm = H W2^T, or gated rows to slot_out
     SimtGemm g2{static_cast<const float *>(H), c.d_ff, 0, offsets, c.E,
                 static_cast<const float *>(W2), nullptr, (int64_t)c.d * c.d_ff, c.d, c.d_ff, 1,
-                static_cast<float *>(Y_perm), c.d, 0};
+                static_cast<float *>(slot_out ? slot_out : Y_perm), c.d, 0,
+                slot_out ? src_slot : nullptr, c.k, slot_out ? kept : nullptr, gates};
     if ((err = run(g2, ACT_NONE, gm, 1, s)) != cudaSuccess)
         return err;
     if (c.n_shared > 0 && c.T > 0) {

@@ -9,10 +9,13 @@
 //
 // Two launches: GEMM1 (hidden = act(A W1^T), SwiGLU fuses W3) and GEMM2
 // (out = hidden W2^T).  GEMM1's routed A rows come either from the permuted
-// buffer x_perm or, with the dispatch fused in, straight from x: each tile's
-// 128 rows are gathered by TMA (tile::gather4, four rows per copy, one copy
-// per lane of the producer warp) through the per-row source table that
-// moe_dispatch_rows writes.  Each launch covers two tile sets:
+// buffer x_perm or, with the dispatch fused in, straight from x: four more
+// warps copy each stage's 128 rows with 16-byte cp.async through the per-row
+// assignment table that moe_dispatch_rows writes (a TMA row gather, 4 rows
+// per instruction, was bound by the TMA issue rate: 64 instructions per stage
+// instead of 2).  GEMM2 may take the combine's gate too: each kept
+// row, times its assignment's gate, goes straight to that assignment's row of
+// a [T k, d] output (EPI_GATED).  Each launch covers two tile sets:
 //   set 0, routed: for expert e the rows [offsets[e], offsets[e+1]) of the
 //          permuted buffer, read from device memory (no host sync); segments
 //          start on multiples of 128 rows, so a 128-row tile has one expert;
@@ -28,7 +31,8 @@
 //
 // Warps: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..9 = epilogue
 // (warp w reads TMEM lanes 32 (w mod 4) .. +31; warps 2..5 take the first half
-// of the tile's columns, warps 6..9 the second).  Every wait on an mbarrier is
+// of the tile's columns, warps 6..9 the second), 10..13 = gather warps (only
+// when GEMM1 reads its rows from x).  Every wait on an mbarrier is
 // bounded by a wall-clock limit; on expiry the CTA records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, every role leaves its loop, the
 // CTA drains what it issued (bounded as well), frees TMEM and returns.
@@ -55,7 +59,11 @@ constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BYTES;
 constexpr int OFF_TILES = OFF_BAR + 256;
 constexpr int SMEM_BYTES = OFF_TILES + 2 * 4 * (kMaxE + 1) + 1024;   // + alignment slack
 
-enum Epi { EPI_NONE = 0, EPI_GELU = 1, EPI_SWIGLU = 2 };
+// EPI_GATED: GEMM2 with the combine's gate fused (routed rows only): row r
+// of expert e's segment, when kept (r - offsets[e] < kept[e]), holds
+// assignment a = src_slot[r]; gates[a] * acc goes, rounded to bf16, to row a
+// of slot_out.  Shared-expert tiles store as EPI_NONE.
+enum Epi { EPI_NONE = 0, EPI_GELU = 1, EPI_SWIGLU = 2, EPI_GATED = 3 };
 
 struct SetDesc {
     int routed;     // 1: rows and B group from the segment table
@@ -69,15 +77,22 @@ struct SetDesc {
 
 struct __align__(64) Params {
     CUtensorMap tmA[2], tmB[2], tmB3[2], tmC[2];
-    CUtensorMap tmX;             // x as a 2-D [T][d] map with one-row boxes (gathered A)
     SetDesc set[2];
     int nsets;
     int E;
-    int gather;                  // 1: routed A rows gathered from x through src_rows
-    int n_rows;                  // rows of the permuted buffers (entries of src_rows)
-    const int32_t *src_rows;     // [n_rows] token of each permuted row
+    int gather;                  // 1: routed A rows gathered from x through src_slot
+    const __nv_bfloat16 *xg;     // x [T][x_ld] (gathered A rows)
+    int x_ld;
+    int n_rows;                  // rows of the permuted buffers (entries of src_slot)
+    int k;                       // experts per token: token of assignment a = a / k
+    const int32_t *src_slot;     // [n_rows] assignment t k + j of each permuted row (-1: none)
+    const int32_t *kept;         // [E] kept rows of each segment (EPI_GATED)
+    const float *gates;          // [T k] (EPI_GATED)
+    __nv_bfloat16 *slot_out;     // [T k][slot_ld] (EPI_GATED)
+    int slot_ld;
     const int32_t *offsets;
     int32_t *status;
+    int clear_status;            // 1: block 0 clears the status word before any wait
     unsigned long long timeout_ns;
 };
 
@@ -104,16 +119,28 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// CL: acquire at cluster scope (the barrier's arrivals include writes of the
+// other CTA of an SM pair made by its threads, not by TMA)
+template <bool CL = false>
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
+    if (CL)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 
@@ -134,14 +161,15 @@ struct Ctl {
 // (returns false) when the time limit passed or, if honor_abort, when another
 // role already gave up.  Drain waits pass honor_abort = false: they must see
 // their own copies land even after an abort, but stay bounded.
+template <bool CL = false>
 __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &c,
                                       bool honor_abort = true)
 {
-    if (mbar_try(bar, parity))
+    if (mbar_try<CL>(bar, parity))
         return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try(bar, parity))
+        if (mbar_try<CL>(bar, parity))
             return true;
         if ((i & 31u) == 0) {
             if (honor_abort && *c.abort)
@@ -165,25 +193,116 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// Four rows (r0..r3) of a 2-D map, one 64-element box each, into 512
-// consecutive bytes of shared memory (the same swizzled layout a 4-row box
-// would give at that offset).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int col, int r0, int r1, int r2, int r3)
+// ---- gathered A rows (the dispatch fused into GEMM1) ----
+// GATHER_WARPS extra warps copy the tile's 128 rows of each stage straight
+// from x with 16-byte cp.async, into the 128-byte swizzled layout a TMA box
+// would give (row r of a 64-wide box at r * 128 bytes, its 16-byte chunk j at
+// position j ^ (r & 7)).  A warp copies whole rows: with KS boxes per stage a
+// row is 8 KS chunks, so one instruction moves 32 / (8 KS) rows.
+constexpr int GATHER_WARPS = 4;
+
+// 16 bytes, or (src_bytes = 0) 16 zero bytes without reading src
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
 {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(bar)
-        : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// the source row of permuted row r (rows past the table read token 0; their
-// results are never used)
+template <int KS>
+struct GatherLanes {
+    static constexpr int CPR = 8 * KS;      // 16-byte chunks of a row per stage
+    static constexpr int RPI = 32 / CPR;    // rows per warp instruction
+    static constexpr int NI = 32 / RPI;     // instructions per warp per stage (32 rows)
+};
+
+// This lane's copies of one stage: gather warp gw owns rows [32 gw, 32 gw + 32)
+// of the CTA's 128; tok[i] is the token of its row in instruction i.  Columns
+// at or past the row length x_ld (the second box of a stage when d is an odd
+// multiple of 64) are zero-filled, as TMA fills a box past the tensor.
+template <int KS>
+__device__ __forceinline__ void gather_stage(uint32_t a_stage, uint32_t box_stride,
+                                             const __nv_bfloat16 *x, int x_ld, int kcol,
+                                             const int *tok, int gw, int lane)
+{
+    using G = GatherLanes<KS>;
+    const int c = lane % G::CPR, sub = lane / G::CPR;
+    const int box = c >> 3, j = c & 7;
+    const bool inside = kcol + c * 8 < x_ld;
+#pragma unroll
+    for (int i = 0; i < G::NI; ++i) {
+        const int row = 32 * gw + G::RPI * i + sub;
+        const __nv_bfloat16 *src = inside ? x + (int64_t)tok[i] * x_ld + kcol + c * 8 : x;
+        cp_async16(a_stage + box * box_stride + row * 128 + ((j ^ (row & 7)) << 4), src,
+                   inside ? 16u : 0u);
+    }
+}
+
+// A stage's copies by this lane have landed (cp.async.wait_group before this):
+// make them visible to the tensor core (async proxy), then one arrive per
+// warp on the stage's full barrier; PAIR: the leader CTA's barrier, releasing
+// at cluster scope.
+template <bool PAIR>
+__device__ __forceinline__ void gather_arrive(uint32_t full, int lane)
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) {
+        if (PAIR) {
+            uint32_t remote;
+            asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(full));
+            asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                             remote)
+                         : "memory");
+        } else {
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(full) : "memory");
+        }
+    }
+}
+
+// the token whose x row permuted row r holds (padding rows, and rows past the
+// table, read token 0; their results are never used)
 __device__ __forceinline__ int gather_row(const Params &p, int r)
 {
-    return r < p.n_rows ? p.src_rows[r] : 0;
+    const int a = r < p.n_rows ? p.src_slot[r] : -1;
+    return a >= 0 ? a / p.k : 0;
+}
+
+// EPI_GATED: the assignment a routed row `row` of expert e holds (-1 for a
+// padding row) and its gate.
+__device__ __forceinline__ int gated_slot(const Params &p, int e, int row, float *gate)
+{
+    const int a = row - p.offsets[e] < p.kept[e] ? p.src_slot[row] : -1;
+    *gate = a >= 0 ? p.gates[a] : 0.f;
+    return a;
+}
+
+// EPI_GATED: 32 accumulator columns of one row, times the gate, rounded to
+// bf16, to 64 bytes of the slot's output row.
+__device__ __forceinline__ void store_gated(const Params &p, int a, float gate, int col,
+                                            const float *v)
+{
+    uint4 *dst = reinterpret_cast<uint4 *>(p.slot_out + (int64_t)a * p.slot_ld + col);
+#pragma unroll
+    for (int q = 0; q < CHUNK / 8; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(gate * v[8 * q + 2 * i],
+                                                     gate * v[8 * q + 2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
 }
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
@@ -325,7 +444,8 @@ __device__ __forceinline__ void epilogue_chunk(const float *g, const float *u, u
 }
 
 template <int EPI, bool GATHER>
-__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p)
+__global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
+    grouped_gemm_kernel(const __grid_constant__ Params p)
 {
     constexpr int BN_B = EPI == EPI_SWIGLU ? BN / 2 : BN;     // B rows per tensor per tile
     constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;   // output columns per tile
@@ -354,7 +474,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     // ---- set-up: barriers, TMEM, tile table ----
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
+            // the producer's expect_tx arrive, and one arrive per gather warp
+            mbar_init(full_bar(s), 1 + (GATHER ? GATHER_WARPS : 0));
             mbar_init(empty_bar(s), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -372,9 +493,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // the segment table and the A rows come from the previous kernels
+    pdl_wait();
+    pdl_trigger();
+    if (p.clear_status && blockIdx.x == 0 && threadIdx.x == 0)
+        *p.status = 0;
     int routed_total = 0;
     if (p.set[0].routed && p.nsets > 0) {
-        for (int e = threadIdx.x; e < p.E; e += THREADS)
+        for (int e = threadIdx.x; e < p.E; e += blockDim.x)
             mtiles[e] = (p.offsets[e + 1] - p.offsets[e]) / BM;
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -401,10 +527,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
 
     if (warp == 0) {
         // ================= TMA producer =================
-        // Lane 0 owns the barrier waits and the box copies; with gathered A
-        // rows (GATHER) the whole warp runs and every lane copies four of the
-        // tile's 128 rows.  The other lanes of the warp stay in this branch.
-        if (GATHER || lane == 0) {
+        // Lane 0 owns the barrier waits and the box copies (with gathered A
+        // rows, the B boxes only: the gather warps copy A).
+        if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int issued[STAGES];
@@ -416,23 +541,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                 const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
                 const SetDesc &sd = p.set[t.set];
                 const bool gath = GATHER && t.set == 0;
-                int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
-                if (gath) {
-                    const int r = t.m0 + lane * 4;
-                    g0 = gather_row(p, r);
-                    g1 = gather_row(p, r + 1);
-                    g2 = gather_row(p, r + 2);
-                    g3 = gather_row(p, r + 3);
-                }
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
-                    int okw = 1;
-                    if (lane == 0)
-                        okw = wait_bar(empty_bar(stage), phase ^ 1u, ctl) ? 1 : 0;
-                    if (GATHER) {
-                        okw = __shfl_sync(0xffffffffu, okw, 0);
-                        __syncwarp();
-                    }
-                    if (!okw) {
+                    if (!wait_bar(empty_bar(stage), phase ^ 1u, ctl)) {
                         ok = false;
                         break;
                     }
@@ -442,20 +552,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                         kcol = (kb % sd.kbg) * BK;
                     }
                     const uint32_t fb = full_bar(stage);
-                    if (lane == 0)
-                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
-                    if (gath)
-                        tma_gather4(sA + stage * A_BYTES + lane * 512, &p.tmX, fb, kcol, g0, g1, g2, g3);
-                    if (lane == 0) {
-                        if (!gath)
-                            tma_load_3d(sA + stage * A_BYTES, &p.tmA[t.set], fb, kcol, t.m0, ga);
-                        if (EPI == EPI_SWIGLU) {
-                            tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
-                            tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &p.tmB3[t.set], fb, kcol,
-                                        t.b_row, gb);
-                        } else {
-                            tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
-                        }
+                    mbar_expect_tx(fb, (gath ? 0 : A_BYTES) + B_BYTES);
+                    if (!gath)
+                        tma_load_3d(sA + stage * A_BYTES, &p.tmA[t.set], fb, kcol, t.m0, ga);
+                    if (EPI == EPI_SWIGLU) {
+                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                        tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &p.tmB3[t.set], fb, kcol,
+                                    t.b_row, gb);
+                    } else {
+                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
                     }
                     issued[stage] = 1;
                     last_phase[stage] = phase;
@@ -465,13 +570,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                     }
                 }
             }
-            // drain: every load this warp issued has landed before the CTA exits
-            if (lane == 0)
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued[s])
-                        wait_bar(full_bar(s), last_phase[s], ctl, false);
-            if (GATHER)
-                __syncwarp();
+            // drain: every load this CTA issued has landed before it exits
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s])
+                    wait_bar(full_bar(s), last_phase[s], ctl, false);
         }
     } else if (warp == 1) {
         // ================= MMA issuer =================
@@ -522,6 +624,49 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                 wait_bar(drain_bar, 0, ctl, false);
             }
         }
+    } else if (GATHER && warp >= 2 + EPI_WARPS) {
+        // ================= gather warps: routed A rows from x =================
+        // A stage is signalled D issues after its copies were issued, so the
+        // copies of D + 1 stages are in flight while the MMA has a full stage
+        // to work on.
+        using G = GatherLanes<1>;
+        constexpr int D = STAGES - 2;
+        const int gw = warp - (2 + EPI_WARPS);
+        const int sub = lane / G::CPR;
+        int stage = 0, seq = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+            const SetDesc &sd = p.set[t.set];
+            const bool gath = t.set == 0;   // shared-expert tiles: TMA boxes of x
+            int tok[G::NI];
+#pragma unroll
+            for (int i = 0; i < G::NI; ++i)
+                tok[i] = gath ? gather_row(p, t.m0 + 32 * gw + G::RPI * i + sub) : 0;
+            for (int kb = 0; kb < sd.k_blocks; ++kb) {
+                int okw = lane == 0 ? (wait_bar(empty_bar(stage), phase ^ 1u, ctl) ? 1 : 0) : 1;
+                if (!__shfl_sync(0xffffffffu, okw, 0)) {
+                    ok = false;
+                    break;
+                }
+                if (gath)
+                    gather_stage<1>(sA + stage * A_BYTES, 0, p.xg, p.x_ld, kb * BK, tok, gw, lane);
+                cp_async_commit();
+                if (seq >= D) {
+                    cp_async_wait<D>();
+                    gather_arrive<false>(full_bar((stage + STAGES - D) % STAGES), lane);
+                }
+                ++seq;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        cp_async_wait<0>();   // the last stages' copies, then their arrivals
+        for (int q = seq < D ? seq : D; q > 0; --q)
+            gather_arrive<false>(full_bar((stage + STAGES - q) % STAGES), lane);
     } else {
         // ================= epilogue (warps 2..9) =================
         const int q = warp & 3;                      // TMEM lane quarter
@@ -538,6 +683,18 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const int c_end = min((half + 1) * (BN_OUT / 2), p.set[t.set].c_cols - t.c_col);
+            if (EPI == EPI_GATED && t.set == 0) {
+                // gate and scatter: this lane's row goes to its assignment's row
+                float gate;
+                const int a = gated_slot(p, t.b_group, t.m0 + q * 32 + lane, &gate);
+#pragma unroll 1
+                for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
+                    float g[CHUNK];
+                    tmem_ld32(tbase + c, g);
+                    if (a >= 0)
+                        store_gated(p, a, gate, t.c_col + c, g);
+                }
+            } else {
 #pragma unroll 1
             for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
                 float g[CHUNK], u[CHUNK];
@@ -568,6 +725,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                     tma_store_3d(&p.tmC[t.set], stg, t.c_col + c, t.m0 + q * 32, t.c_group);
                     bulk_commit();
                 }
+            }
             }
             // this warp's reads of the accumulator are done
             tc_fence_before();
@@ -657,19 +815,6 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
-// tma_gather4 with the completion reported to the leader CTA's barrier
-__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap *map,
-                                                 uint32_t bar_leader, int col, int r0, int r1,
-                                                 int r2, int r3)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
-        "complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(bar_leader)
-        : "memory");
-}
-
 __device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                               uint32_t accumulate)
 {
@@ -748,7 +893,8 @@ __device__ __forceinline__ Tile2 decode2(const Params &p, const int *tstart, con
 }
 
 template <int EPI, bool GATHER>
-__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __grid_constant__ Params p)
+__global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
+    grouped_gemm_2sm_kernel(const __grid_constant__ Params p)
 {
     constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;   // output columns per tile
     extern __shared__ uint8_t smem_raw[];
@@ -777,7 +923,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES2; ++s) {
-            mbar_init(full_bar(s), 1);
+            // the leader producer's expect_tx arrive, and (gathered A rows) one
+            // arrive per gather warp of both CTAs
+            mbar_init(full_bar(s), 1 + (GATHER ? 2 * GATHER_WARPS : 0));
             mbar_init(empty_bar(s), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -795,9 +943,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
+    // the segment table and the A rows come from the previous kernels
+    pdl_wait();
+    pdl_trigger();
+    if (p.clear_status && blockIdx.x == 0 && threadIdx.x == 0)
+        *p.status = 0;
     int routed_total = 0;
     if (p.set[0].routed && p.nsets > 0) {
-        for (int e = threadIdx.x; e < p.E; e += THREADS) {
+        for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
             const int mt = (p.offsets[e + 1] - p.offsets[e]) / BM;
             mpairs[e] = (mt + 1) / 2;
         }
@@ -826,10 +979,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
 
     if (warp == 0) {
         // ================= TMA producer (both CTAs) =================
-        // Lane 0 owns the barrier waits and the box copies; with gathered A
-        // rows (GATHER) the whole warp runs and every lane copies four of its
-        // CTA's 128 rows.  The other lanes of the warp stay in this branch.
-        if (GATHER || lane == 0) {
+        // Lane 0 owns the barrier waits and the box copies (with gathered A
+        // rows, the B boxes only: the gather warps copy A).
+        if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int issued[STAGES2];
@@ -845,23 +997,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                 const CUtensorMap *bmap =
                     (EPI == EPI_SWIGLU && rank == 1) ? &p.tmB3[t.set] : &p.tmB[t.set];
                 const bool gath = GATHER && t.set == 0;
-                int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
-                if (gath) {
-                    const int r = t.m0 + (int)rank * 128 + lane * 4;
-                    g0 = gather_row(p, r);
-                    g1 = gather_row(p, r + 1);
-                    g2 = gather_row(p, r + 2);
-                    g3 = gather_row(p, r + 3);
-                }
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
-                    int okw = 1;
-                    if (lane == 0)
-                        okw = wait_bar(empty_bar(stage), phase ^ 1u, ctl) ? 1 : 0;
-                    if (GATHER) {
-                        okw = __shfl_sync(0xffffffffu, okw, 0);
-                        __syncwarp();
-                    }
-                    if (!okw) {
+                    if (!wait_bar(empty_bar(stage), phase ^ 1u, ctl)) {
                         ok = false;
                         break;
                     }
@@ -870,21 +1007,16 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                         ga = gb = kb / sd.kbg;
                         kcol = (kb % sd.kbg) * BK * KSUB;
                     }
-                    if (leader && lane == 0)
-                        mbar_expect_tx(full_bar(stage), 4 * KSUB * HALF_BYTES);
+                    if (leader)   // both CTAs' B boxes (and A boxes unless gathered)
+                        mbar_expect_tx(full_bar(stage), (gath ? 2 : 4) * KSUB * HALF_BYTES);
                     const uint32_t fb = map_to_rank(full_bar(stage), 0);
                     for (int ks = 0; ks < KSUB; ++ks) {
                         const uint32_t a_dst = sA + (stage * KSUB + ks) * HALF_BYTES;
-                        if (gath)
-                            tma_gather4_pair(a_dst + lane * 512, &p.tmX, fb, kcol + ks * BK, g0, g1,
-                                             g2, g3);
-                        if (lane == 0) {
-                            if (!gath)
-                                tma_load_3d_pair(a_dst, &p.tmA[t.set], fb, kcol + ks * BK,
-                                                 t.m0 + (int)rank * 128, ga);
-                            tma_load_3d_pair(sB + (stage * KSUB + ks) * HALF_BYTES, bmap, fb,
-                                             kcol + ks * BK, brow, gb);
-                        }
+                        if (!gath)
+                            tma_load_3d_pair(a_dst, &p.tmA[t.set], fb, kcol + ks * BK,
+                                             t.m0 + (int)rank * 128, ga);
+                        tma_load_3d_pair(sB + (stage * KSUB + ks) * HALF_BYTES, bmap, fb,
+                                         kcol + ks * BK, brow, gb);
                     }
                     issued[stage] = 1;
                     last_phase[stage] = phase;
@@ -895,12 +1027,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                 }
             }
             // the leader's full barriers count both CTAs' bytes: drain there
-            if (leader && lane == 0)
+            if (leader)
                 for (int s = 0; s < STAGES2; ++s)
                     if (issued[s])
-                        wait_bar(full_bar(s), last_phase[s], ctl, false);
-            if (GATHER)
-                __syncwarp();
+                        wait_bar<GATHER>(full_bar(s), last_phase[s], ctl, false);
         }
     } else if (warp == 1) {
         // ================= MMA issuer (leader CTA only) =================
@@ -920,7 +1050,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                 tc_fence_after();
                 const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
-                    if (!wait_bar(full_bar(stage), phase, ctl)) {
+                    // gathered rows: arrivals of the other CTA's threads too
+                    if (!wait_bar<GATHER>(full_bar(stage), phase, ctl)) {
                         ok = false;
                         break;
                     }
@@ -955,6 +1086,51 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                 wait_bar(drain_bar, 0, ctl, false);
             }
         }
+    } else if (GATHER && warp >= 2 + EPI_WARPS) {
+        // ================= gather warps: routed A rows from x (both CTAs) =====
+        // Each CTA's four gather warps copy its 128 rows of the pair tile and
+        // arrive on the leader's full barrier; a stage is signalled one issue
+        // after its copies were issued (two stages' copies in flight).
+        using G = GatherLanes<KSUB>;
+        constexpr int D = STAGES2 - 2;
+        const int gw = warp - (2 + EPI_WARPS);
+        const int sub = lane / G::CPR;
+        int stage = 0, seq = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = cluster_id; ok && tile < total; tile += nclusters) {
+            const Tile2 t = decode2(p, tstart, mpairs, routed_total, tile);
+            const SetDesc &sd = p.set[t.set];
+            const bool gath = t.set == 0;   // shared-expert tiles: TMA boxes of x
+            int tok[G::NI];
+#pragma unroll
+            for (int i = 0; i < G::NI; ++i)
+                tok[i] = gath ? gather_row(p, t.m0 + (int)rank * 128 + 32 * gw + G::RPI * i + sub)
+                              : 0;
+            for (int kb = 0; kb < sd.k_blocks; ++kb) {
+                int okw = lane == 0 ? (wait_bar(empty_bar(stage), phase ^ 1u, ctl) ? 1 : 0) : 1;
+                if (!__shfl_sync(0xffffffffu, okw, 0)) {
+                    ok = false;
+                    break;
+                }
+                if (gath)
+                    gather_stage<KSUB>(sA + stage * KSUB * HALF_BYTES, HALF_BYTES, p.xg, p.x_ld,
+                                       kb * BK * KSUB, tok, gw, lane);
+                cp_async_commit();
+                if (seq >= D) {
+                    cp_async_wait<D>();
+                    gather_arrive<true>(full_bar((stage + STAGES2 - D) % STAGES2), lane);
+                }
+                ++seq;
+                if (++stage == STAGES2) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        cp_async_wait<0>();   // the last stages' copies, then their arrivals
+        for (int q = seq < D ? seq : D; q > 0; --q)
+            gather_arrive<true>(full_bar((stage + STAGES2 - q) % STAGES2), lane);
     } else {
         // ================= epilogue (warps 2..9, both CTAs) =================
         const int q = warp & 3;
@@ -975,6 +1151,18 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                                   ? min((half + 1) * (BN_OUT / 2), p.set[t.set].c_cols - c_col)
                                   : 0;
             const int row = t.m0 + (int)rank * 128 + q * 32;
+            if (EPI == EPI_GATED && t.set == 0) {
+                // gate and scatter: this lane's row goes to its assignment's row
+                float gate;
+                const int a = gated_slot(p, t.b_group, row + lane, &gate);
+#pragma unroll 1
+                for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
+                    float g[CHUNK];
+                    tmem_ld32(tbase + c, g);
+                    if (a >= 0)
+                        store_gated(p, a, gate, c_col + c, g);
+                }
+            } else {
 #pragma unroll 1
             for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
                 float g[CHUNK], u[CHUNK];
@@ -1003,6 +1191,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_2sm_kernel(const __gr
                     tma_store_3d(&p.tmC[t.set], stg, c_col + c, row, t.c_group);
                     bulk_commit();
                 }
+            }
             }
             tc_fence_before();
             __syncwarp();
@@ -1068,23 +1257,6 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64
     return r == CUDA_SUCCESS;
 }
 
-// 2-D bf16 tensor (d0 contiguous x d1 rows, row pitch s1 bytes)
-bool make_map2d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t s1,
-                uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw)
-{
-    EncodeTiled enc = encoder();
-    if (!enc)
-        return false;
-    cuuint64_t dims[2] = {d0, d1 > 0 ? d1 : 1};
-    cuuint64_t strides[1] = {s1};
-    cuuint32_t box[2] = {b0, b1};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 int sm_count()
 {
     int dev = 0, n = 148;
@@ -1102,12 +1274,14 @@ cudaError_t launch_2sm(const Params &p, cudaStream_t s)
     if (err != cudaSuccess)
         return err;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(THREADS, 1, 1);
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1, 1);
     cfg.dynamicSmemBytes = SMEM2_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
@@ -1120,6 +1294,7 @@ cudaError_t launch_2sm(const Params &p, cudaStream_t s)
     if (clusters < 1)
         return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.numAttrs = 2;   // and programmatic dependent launch
     err = cudaLaunchKernelEx(&cfg, kern, p);
     if (err != cudaSuccess)
         return err;
@@ -1134,8 +1309,8 @@ cudaError_t launch(const Params &p, cudaStream_t s)
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess)
         return err;
-    kern<<<sm_count(), THREADS, SMEM_BYTES, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(sm_count()), dim3(THREADS + (GATHER ? 32 * GATHER_WARPS : 0)),
+                      SMEM_BYTES, s, p);
 }
 
 // Diagnostic for the timeout path: one thread waits, with the same bounded
@@ -1163,9 +1338,11 @@ cudaError_t launch_wait_probe(int32_t *status, unsigned long long timeout_ns, cu
 }
 
 cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const int32_t *offsets,
-                               const int32_t *src_rows, const void *W1, const void *W3, const void *W2, const void *x,
-                               const void *Ws1, const void *Ws3, const void *Ws2, void *Y_perm,
-                               void *Y_sh, void *H, void *H_sh, int32_t *status, cudaStream_t s)
+                               const int32_t *src_slot, const void *W1, const void *W3,
+                               const void *W2, const void *x, const void *Ws1, const void *Ws3,
+                               const void *Ws2, void *Y_perm, void *Y_sh, void *H, void *H_sh,
+                               int32_t *status, bool clear_status, cudaStream_t s,
+                               const int32_t *kept, const float *gates, void *slot_out)
 {
     using namespace tc;
     const uint64_t R = (uint64_t)perm_rows(c), d = c.d, F = c.d_ff, E = c.E;
@@ -1191,15 +1368,18 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     p1.E = c.E;
     p1.offsets = offsets;
     p1.status = status;
+    p1.clear_status = clear_status ? 1 : 0;
     p1.timeout_ns = 2000000000ull;
     p1.nsets = shared ? 2 : 1;
     bool ok = true;
-    if (src_rows) {
-        // dispatch fused in: tile rows gathered from x, one-row boxes (gather4)
+    if (!x_perm) {
+        // dispatch fused in: tile rows gathered from x by the gather warps
         p1.gather = 1;
-        p1.src_rows = src_rows;
+        p1.src_slot = src_slot;
         p1.n_rows = (int)R;
-        ok &= make_map2d(&p1.tmX, x, d, T, d * 2, BK, 1, SW128);
+        p1.k = c.k;
+        p1.xg = static_cast<const __nv_bfloat16 *>(x);
+        p1.x_ld = (int)d;
     } else {
         ok &= make_map(&p1.tmA[0], x_perm, d, R, 1, d * 2, 0, BK, BM, SW128);
     }
@@ -1242,7 +1422,18 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     ok = true;
     ok &= make_map(&p2.tmA[0], H, F, R, 1, F * 2, 0, BK, BM, SW128);
     ok &= make_map(&p2.tmB[0], W2, F, d, E, F * 2, d * F * 2, BK, bn2_b, SW128);
-    ok &= make_map(&p2.tmC[0], Y_perm, d, R, 1, d * 2, 0, CHUNK, 32, SW64);
+    if (slot_out) {
+        // the combine's gate fused: row r of expert e -> row src_slot[r] of slot_out
+        p2.src_slot = src_slot;
+        p2.n_rows = (int)R;
+        p2.k = c.k;
+        p2.kept = kept;
+        p2.gates = gates;
+        p2.slot_out = static_cast<__nv_bfloat16 *>(slot_out);
+        p2.slot_ld = (int)d;
+    } else {
+        ok &= make_map(&p2.tmC[0], Y_perm, d, R, 1, d * 2, 0, CHUNK, 32, SW64);
+    }
     p2.set[0] = SetDesc{1, 0, (int)ceil_div(d, BN), 1, (int)ceil_div(F, KB), 0, (int)d};
     if (shared) {
         ok &= make_map(&p2.tmA[1], H_sh, Fs, T, S, Fs * 2, T * Fs * 2, BK, BM, SW128);
@@ -1253,6 +1444,8 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     }
     if (!ok)
         return cudaErrorInvalidValue;
+    if (slot_out)
+        return pair ? launch_2sm<EPI_GATED>(p2, s) : launch<EPI_GATED>(p2, s);
     return pair ? launch_2sm<EPI_NONE>(p2, s) : launch<EPI_NONE>(p2, s);
 }
 

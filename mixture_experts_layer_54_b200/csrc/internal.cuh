@@ -21,6 +21,38 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline int dtype_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
 
+// ---- programmatic dependent launch ----
+// The forward's kernels are launched so that each may start while the
+// previous kernel in the stream is finishing: its blocks become resident and
+// run their set-up, then wait in pdl_wait() until the previous kernel has
+// completed and its writes are visible.  pdl_trigger() lets the next kernel
+// start launching; every kernel launched with launch_pdl calls pdl_wait()
+// before it reads anything an earlier kernel wrote (both are no-ops for a
+// kernel launched without the attribute).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
+
 // Shape limits and codes; also the capacity factor rule.
 moe_status validate(const moe_config &c);
 int64_t capacity_of(const moe_config &c);          // valid config only
@@ -29,13 +61,14 @@ int route_blocks(const moe_config &c);   // blocks of the tiled route kernel
 int partial_rows(const moe_config &c);   // rows of the loss partials, ceil(T / 32)
 int cap_blocks(const moe_config &c);
 
-// Tensor-core router layout (bf16 layers).  Fused (E <= 16): one kernel, the
-// k_parts blocks of a 128-token tile form one cluster.  Otherwise three
-// launches: experts padded to E_pad in n_chunks chunks of n_chunk, K
-// (k_blocks of 64) split in k_parts of kb_per_part, through scratch.
+// Tensor-core router layout (bf16 layers).  Fused (E <= 64 and the split
+// weights of a K part fit in shared memory): one persistent kernel, clusters
+// of k_parts blocks walking 128-token tiles.  Otherwise three launches:
+// experts padded to E_pad in n_chunks chunks of n_chunk, K (k_blocks of 64)
+// split in k_parts of kb_per_part, through scratch.
 struct RoutePlan {
     bool tensor_cores, fused;
-    int E_pad, n_chunk, n_chunks, k_blocks, k_parts, kb_per_part, cluster, blocks;
+    int E_pad, n_chunk, n_chunks, k_blocks, k_parts, kb_per_part, cluster, blocks, stages;
 };
 RoutePlan route_plan(const moe_config &c);
 size_t route_scratch_bytes(const moe_config &c);
@@ -47,7 +80,6 @@ struct StageScratch {
     int32_t *status;      // device status word (timeouts)
     void *route;          // tensor-core router (three launches): split weights, partial logits
     int32_t *hist;        // [cap_blocks][k][E]
-    int32_t *base;        // [cap_blocks][k][E]
     int32_t *count_base;  // [E] sharded capacity: earlier shards' assignments
     unsigned long long *keys;   // [T k] batch-prioritized capacity: per-expert lists
     void *H;              // [perm_rows][F] dtype
@@ -65,24 +97,28 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *W_r,
 cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r,
                             const float *logit_bias, const float *select_bias, int32_t *topk,
                             float *gates, float *partials, float *logits_out, float *scores_out,
-                            void *scratch, int32_t *status, cudaStream_t s);
+                            void *scratch, int32_t *status, bool clear_status, cudaStream_t s);
 
 cudaError_t launch_shard_base(const moe_config &c, const int32_t *shard_counts, int shard,
                               int32_t *count_base, cudaStream_t s);
 
-// count_base (nullable, [E]): assignments to each expert in earlier shards of
-// the same global batch (token order); C is then the global batch's capacity.
+// hist: scratch [cap_blocks][k][E] int32.  count_base (nullable, [E]):
+// assignments to each expert in earlier shards of the same global batch
+// (token order); C is then the global batch's capacity.  partials (nullable,
+// the router's loss partials): the same launch also writes aux and zloss.
 cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep,
                             int32_t *kept, int32_t *offsets, uint8_t *dropped,
-                            int32_t *n_dropped, int32_t *hist, int32_t *base,
-                            cudaStream_t s, const int32_t *count_base = nullptr);
+                            int32_t *n_dropped, int32_t *hist, cudaStream_t s,
+                            const int32_t *count_base = nullptr,
+                            const float *partials = nullptr, float *aux = nullptr,
+                            float *zloss = nullptr);
 
 cudaError_t launch_capacity_scored(const moe_config &c, int64_t C, const int32_t *topk,
                                    const float *scores, int32_t *counts, int32_t *pos,
                                    uint8_t *keep, int32_t *kept, int32_t *offsets,
                                    uint8_t *dropped, int32_t *n_dropped, int32_t *hist,
-                                   int32_t *base, unsigned long long *keys, cudaStream_t s);
+                                   unsigned long long *keys, cudaStream_t s);
 
 cudaError_t launch_seq_loss(const moe_config &c, int L, const int32_t *topk,
                             const float *partials, float *per_seq, float *loss, cudaStream_t s);
@@ -90,13 +126,25 @@ cudaError_t launch_seq_loss(const moe_config &c, int L, const int32_t *topk,
 cudaError_t launch_bias_update(const moe_config &c, const int32_t *counts, float gamma,
                                float *bias, cudaStream_t s);
 
+// src_slot[offsets[e] + pos[t, j]] = t k + j for every kept (t, j), -1 for
+// every other row.
 cudaError_t launch_dispatch_rows(const moe_config &c, const int32_t *topk, const int32_t *pos,
-                                 const uint8_t *keep, const int32_t *offsets, int32_t *src_rows,
+                                 const uint8_t *keep, const int32_t *offsets, int32_t *src_slot,
                                  cudaStream_t s);
 
+// x_perm nullable (only the table), src_slot nullable (no table; padding rows
+// are not written), zero_rows nullable: rows of tokens with every slot
+// dropped are set to 0 there (the fused combine of a top-1 layer).
 cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *topk,
                             const int32_t *pos, const uint8_t *keep,
-                            const int32_t *offsets, void *x_perm, cudaStream_t s);
+                            const int32_t *offsets, void *x_perm, cudaStream_t s,
+                            int32_t *src_slot = nullptr, void *zero_rows = nullptr);
+
+// y[t] = sum over kept slots j of Y_slot[t k + j] (+ Y_sh[t]) (+ residual[t]),
+// fp32 in slot order.
+cudaError_t launch_combine_slots(const moe_config &c, const void *Y_slot, const void *Y_sh,
+                                 const uint8_t *keep, const void *residual, void *y,
+                                 cudaStream_t s);
 
 cudaError_t launch_combine(const moe_config &c, const void *Y_perm, const void *Y_sh,
                            const float *gates, const int32_t *topk, const int32_t *pos,
@@ -110,20 +158,28 @@ cudaError_t launch_losses(const moe_config &c, const int32_t *counts,
 // one bounded wait on a barrier nobody arrives on (diagnostic)
 cudaError_t launch_wait_probe(int32_t *status, unsigned long long timeout_ns, cudaStream_t s);
 
-// fp32 expert FFNs on the CUDA cores
+// fp32 expert FFNs on the CUDA cores (x_perm, src_slot, kept, gates and
+// slot_out as for launch_ffn_tcgen05)
 cudaError_t launch_ffn_simt(const moe_config &c, const void *x_perm, const int32_t *offsets,
-                            const int32_t *src_rows, const void *W1, const void *W3, const void *W2,
+                            const int32_t *src_slot, const void *W1, const void *W3, const void *W2,
                             const void *x, const void *Ws1, const void *Ws3,
                             const void *Ws2, void *Y_perm, void *Y_sh, void *H,
-                            void *H_sh, cudaStream_t s);
+                            void *H_sh, cudaStream_t s, const int32_t *kept = nullptr,
+                            const float *gates = nullptr, void *slot_out = nullptr);
 
-// bf16 expert FFNs on the tensor cores (tcgen05 + TMEM + TMA)
+// bf16 expert FFNs on the tensor cores (tcgen05 + TMEM + TMA).  x_perm NULL:
+// GEMM1 gathers its routed rows from x through src_slot (row r holds
+// assignment src_slot[r], token src_slot[r] / k).  slot_out non-NULL: GEMM2
+// writes gates[a] * FFN(row) to row a = src_slot[r] of slot_out [T k, d] for
+// every kept row (r - offsets[e] < kept[e]) instead of Y_perm.
 cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm,
-                               const int32_t *offsets, const int32_t *src_rows,
+                               const int32_t *offsets, const int32_t *src_slot,
                                const void *W1, const void *W3,
                                const void *W2, const void *x, const void *Ws1,
                                const void *Ws3, const void *Ws2, void *Y_perm,
                                void *Y_sh, void *H, void *H_sh, int32_t *status,
-                               cudaStream_t s);
+                               bool clear_status, cudaStream_t s,
+                               const int32_t *kept = nullptr, const float *gates = nullptr,
+                               void *slot_out = nullptr);
 
 }  // namespace moe

@@ -6,44 +6,24 @@
 //   L_z   = (1/T) sum_t (logsumexp_i z_{t,i})^2
 // "Lab 01", where to start step 3: f divides by the T k slots.
 #include "internal.cuh"
+#include "losses_common.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int THREADS = 1024;
-constexpr int WARPS = THREADS / 32;
 
-// Column c of the partials (expert c < E, or the lse^2 column c = E) belongs
-// to warp c mod 32; lane l sums rows l, l + 32, ... in order (double), then
-// the 32 lane sums meet by xor shuffles in a fixed pattern: a fixed reduction
-// tree, so the result does not depend on timing.
+// One block: column c of the partials (expert c, or the lse^2 column c = E)
+// is summed by warp c mod 32 in the fixed order of loss_column_sum, then one
+// thread adds the E terms in expert order.
 __global__ void __launch_bounds__(THREADS)
 losses_kernel(const int32_t *__restrict__ counts, const float *__restrict__ partials, int rows,
               int T, int k, int E, float *aux, float *zloss)
 {
     __shared__ double term[kMaxE + 1];
-    const int C = E + 1;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int col = warp; col < C; col += WARPS) {
-        double s = 0.0;
-#pragma unroll 4
-        for (int r = lane; r < rows; r += 32)
-            s += (double)__ldg(partials + (int64_t)r * C + col);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0)
-            term[col] = col < E ? ((double)counts[col] / ((double)T * (double)k)) * (s / (double)T)
-                                : s / (double)T;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double a = 0.0;
-        for (int i = 0; i < E; ++i)
-            a += term[i];
-        *aux = (float)((double)E * a);
-        *zloss = (float)term[E];
-    }
+    pdl_wait();   // counts and partials come from the capacity and route stages
+    pdl_trigger();
+    block_losses(counts, partials, rows, T, k, E, aux, zloss, term);
 }
 
 }  // namespace
@@ -51,9 +31,8 @@ losses_kernel(const int32_t *__restrict__ counts, const float *__restrict__ part
 cudaError_t launch_losses(const moe_config &c, const int32_t *counts, const float *partials,
                           float *aux, float *zloss, cudaStream_t s)
 {
-    losses_kernel<<<1, THREADS, 0, s>>>(counts, partials, partial_rows(c), c.T > 0 ? c.T : 1,
-                                        c.k, c.E, aux, zloss);
-    return cudaGetLastError();
+    return launch_pdl(losses_kernel, dim3(1), dim3(THREADS), 0, s, counts, partials,
+                      partial_rows(c), c.T > 0 ? c.T : 1, c.k, c.E, aux, zloss);
 }
 
 }  // namespace moe

@@ -39,12 +39,18 @@ __device__ __forceinline__ void slot_rows(int t, int k, int E, const int32_t *to
         rows[j] = __shfl_sync(0xffffffffu, mine, j);
 }
 
+// x_perm nullable: only the slot table.  src_slot nullable: row r of a kept
+// slot gets its assignment t k + j.  zero_rows nullable: the row of a token
+// with every slot dropped is set to zero there.
 __global__ void __launch_bounds__(THREADS)
 dispatch_vec_kernel(const uint4 *__restrict__ x, int T, int k, int E, int nvec,
                     const int32_t *__restrict__ topk, const int32_t *__restrict__ pos,
                     const uint8_t *__restrict__ keep, const int32_t *__restrict__ offsets,
-                    uint4 *__restrict__ x_perm)
+                    uint4 *__restrict__ x_perm, int32_t *__restrict__ src_slot,
+                    uint4 *__restrict__ zero_rows)
 {
+    pdl_wait();   // the slots come from the capacity stage
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
     for (int t = gw; t < T; t += gridDim.x * WARPS) {
@@ -54,7 +60,19 @@ dispatch_vec_kernel(const uint4 *__restrict__ x, int T, int k, int E, int nvec,
 #pragma unroll
         for (int j = 0; j < kMaxK; ++j)
             any |= j < k && rows[j] >= 0;
-        if (!any)
+        if (src_slot) {   // lane j records slot j's row
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j)
+                if (j == lane && j < k && rows[j] >= 0)
+                    src_slot[rows[j]] = t * k + j;
+        }
+        if (!any) {
+            if (zero_rows)
+                for (int v = lane; v < nvec; v += 32)
+                    zero_rows[(int64_t)t * nvec + v] = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
+        if (!x_perm)
             continue;
         const uint4 *src = x + (int64_t)t * nvec;
         for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
@@ -82,19 +100,21 @@ dispatch_vec_kernel(const uint4 *__restrict__ x, int T, int k, int E, int nvec,
 }
 
 // Dispatch fused into the expert GEMM: instead of copying rows, record for
-// every kept assignment (t, j) that permuted row offsets[e] + pos[t, j] holds
-// token t.  Padding rows keep the 0 the table was cleared to.
+// every kept assignment a = (t, j) that permuted row offsets[e] + pos[t, j]
+// holds it (token a / k).  Padding rows keep the -1 the table was cleared to.
 __global__ void dispatch_rows_kernel(const int32_t *__restrict__ topk,
                                      const int32_t *__restrict__ pos,
                                      const uint8_t *__restrict__ keep,
-                                     const int32_t *__restrict__ offsets, int64_t A, int k, int E,
-                                     int32_t *__restrict__ src_rows)
+                                     const int32_t *__restrict__ offsets, int64_t A, int E,
+                                     int32_t *__restrict__ src_slot)
 {
+    pdl_wait();   // the slots come from the capacity stage
+    pdl_trigger();
     for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < A;
          a += (int64_t)gridDim.x * blockDim.x) {
         const int e = topk[a];
         if (keep[a] && e >= 0 && e < E)
-            src_rows[offsets[e] + pos[a]] = (int32_t)(a / k);
+            src_slot[offsets[e] + pos[a]] = (int32_t)a;
     }
 }
 
@@ -150,6 +170,8 @@ combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y
                    const int32_t *__restrict__ offsets, const uint4 *__restrict__ residual,
                    uint4 *__restrict__ y, int T, int E, int nvec)
 {
+    pdl_wait();   // the expert rows come from the expert GEMMs
+    pdl_trigger();
     constexpr int N = Vec<Elem>::N;
     constexpr int U = KS >= 4 ? 2 : 8 / KS;
     const int lane = threadIdx.x & 31;
@@ -220,6 +242,85 @@ combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y
     }
 }
 
+// The combine after the gate was applied in the expert GEMM: the k gated rows
+// of a token are contiguous (Y_slot row t k + j); their kept ones are summed
+// in fp32 in slot order, then the shared experts and the residual.
+template <typename Elem, int KS>
+__global__ void __launch_bounds__(THREADS)
+combine_slots_kernel(const uint4 *__restrict__ Y_slot, const uint4 *__restrict__ Y_sh,
+                     const uint8_t *__restrict__ keep, const uint4 *__restrict__ residual,
+                     uint4 *__restrict__ y, int T, int nvec)
+{
+    pdl_wait();   // the gated rows come from the expert GEMM
+    pdl_trigger();
+    constexpr int N = Vec<Elem>::N;
+    constexpr int U = KS >= 4 ? 2 : 8 / KS;
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
+    for (int t = gw; t < T; t += gridDim.x * WARPS) {
+        const int mk = lane < KS ? keep[(int64_t)t * KS + lane] : 0;
+        bool kp[KS];
+#pragma unroll
+        for (int j = 0; j < KS; ++j)
+            kp[j] = __shfl_sync(0xffffffffu, mk, j) != 0;
+        const uint4 *rows = Y_slot + (int64_t)t * KS * nvec;
+        for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
+            uint4 raw[KS][U];
+#pragma unroll
+            for (int j = 0; j < KS; ++j)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    raw[j][u] = (kp[j] && v < nvec) ? __ldcs(rows + (int64_t)j * nvec + v)
+                                                    : make_uint4(0u, 0u, 0u, 0u);
+                }
+            float acc[U][N];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+                    acc[u][i] = 0.f;
+#pragma unroll
+            for (int j = 0; j < KS; ++j) {
+                if (!kp[j])
+                    continue;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    float f[N];
+                    Vec<Elem>::load(raw[j][u], f);
+#pragma unroll
+                    for (int i = 0; i < N; ++i)
+                        acc[u][i] += f[i];
+                }
+            }
+            const uint4 *extra[2] = {Y_sh ? Y_sh + (int64_t)t * nvec : nullptr,
+                                     residual ? residual + (int64_t)t * nvec : nullptr};
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                if (!extra[q])
+                    continue;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) {
+                        float f[N];
+                        Vec<Elem>::load(__ldcs(extra[q] + v), f);
+#pragma unroll
+                        for (int i = 0; i < N; ++i)
+                            acc[u][i] += f[i];
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec)
+                    y[(int64_t)t * nvec + v] = Vec<Elem>::store(acc[u]);
+            }
+        }
+    }
+}
+
 // As many blocks of 8 token-warps as are resident at once, fewer for small T.
 template <typename K>
 int grid_for(K kernel, int T)
@@ -239,28 +340,63 @@ int grid_for(K kernel, int T)
 
 cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *topk,
                             const int32_t *pos, const uint8_t *keep, const int32_t *offsets,
-                            void *x_perm, cudaStream_t s)
+                            void *x_perm, cudaStream_t s, int32_t *src_slot, void *zero_rows)
 {
     if (c.T == 0)
         return cudaSuccess;
     const int nvec = (int)((int64_t)c.d * dtype_bytes(c.dtype) / 16);
-    dispatch_vec_kernel<<<grid_for(dispatch_vec_kernel, c.T), THREADS, 0, s>>>(
-        static_cast<const uint4 *>(x), c.T, c.k, c.E, nvec, topk, pos, keep, offsets,
-        static_cast<uint4 *>(x_perm));
-    return cudaGetLastError();
+    return launch_pdl(dispatch_vec_kernel, dim3(grid_for(dispatch_vec_kernel, c.T)), dim3(THREADS),
+                      0, s, static_cast<const uint4 *>(x), c.T, c.k, c.E, nvec, topk, pos, keep,
+                      offsets, static_cast<uint4 *>(x_perm), src_slot,
+                      static_cast<uint4 *>(zero_rows));
 }
 
 cudaError_t launch_dispatch_rows(const moe_config &c, const int32_t *topk, const int32_t *pos,
-                                 const uint8_t *keep, const int32_t *offsets, int32_t *src_rows,
+                                 const uint8_t *keep, const int32_t *offsets, int32_t *src_slot,
                                  cudaStream_t s)
 {
-    cudaError_t err = cudaMemsetAsync(src_rows, 0, sizeof(int32_t) * (size_t)perm_rows(c), s);
+    // every entry -1 (all bytes 0xFF), then the kept rows
+    cudaError_t err = cudaMemsetAsync(src_slot, 0xFF, sizeof(int32_t) * (size_t)perm_rows(c), s);
     if (err != cudaSuccess || c.T == 0)
         return err;
     const int64_t A = (int64_t)c.T * c.k;
     const int blocks = (int)(ceil_div(A, 256) < 1184 ? ceil_div(A, 256) : 1184);
-    dispatch_rows_kernel<<<blocks, 256, 0, s>>>(topk, pos, keep, offsets, A, c.k, c.E, src_rows);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_rows_kernel, dim3(blocks), dim3(256), 0, s, topk, pos, keep,
+                      offsets, A, c.E, src_slot);
+}
+
+cudaError_t launch_combine_slots(const moe_config &c, const void *Y_slot, const void *Y_sh,
+                                 const uint8_t *keep, const void *residual, void *y,
+                                 cudaStream_t s)
+{
+    if (c.T == 0)
+        return cudaSuccess;
+    const int nvec = (int)((int64_t)c.d * dtype_bytes(c.dtype) / 16);
+    cudaError_t err = cudaSuccess;
+    auto args = [&](auto kern) {
+        err = launch_pdl(kern, dim3(grid_for(kern, c.T)), dim3(THREADS), 0, s,
+                         static_cast<const uint4 *>(Y_slot), static_cast<const uint4 *>(Y_sh),
+                         keep, static_cast<const uint4 *>(residual), static_cast<uint4 *>(y),
+                         c.T, nvec);
+    };
+    auto by_k = [&](auto elem) {
+        using El = decltype(elem);
+        switch (c.k) {
+        case 1: args(combine_slots_kernel<El, 1>); break;
+        case 2: args(combine_slots_kernel<El, 2>); break;
+        case 3: args(combine_slots_kernel<El, 3>); break;
+        case 4: args(combine_slots_kernel<El, 4>); break;
+        case 5: args(combine_slots_kernel<El, 5>); break;
+        case 6: args(combine_slots_kernel<El, 6>); break;
+        case 7: args(combine_slots_kernel<El, 7>); break;
+        default: args(combine_slots_kernel<El, 8>); break;
+        }
+    };
+    if (c.dtype == MOE_DTYPE_BF16)
+        by_k(__nv_bfloat16());
+    else
+        by_k(float());
+    return err;
 }
 
 cudaError_t launch_combine(const moe_config &c, const void *Y_perm, const void *Y_sh,
@@ -271,11 +407,12 @@ cudaError_t launch_combine(const moe_config &c, const void *Y_perm, const void *
     if (c.T == 0)
         return cudaSuccess;
     const int nvec = (int)((int64_t)c.d * dtype_bytes(c.dtype) / 16);
+    cudaError_t err = cudaSuccess;
     auto args = [&](auto kern) {
-        kern<<<grid_for(kern, c.T), THREADS, 0, s>>>(
-            static_cast<const uint4 *>(Y_perm), static_cast<const uint4 *>(Y_sh), gates, topk,
-            pos, keep, offsets, static_cast<const uint4 *>(residual), static_cast<uint4 *>(y),
-            c.T, c.E, nvec);
+        err = launch_pdl(kern, dim3(grid_for(kern, c.T)), dim3(THREADS), 0, s,
+                         static_cast<const uint4 *>(Y_perm), static_cast<const uint4 *>(Y_sh),
+                         gates, topk, pos, keep, offsets, static_cast<const uint4 *>(residual),
+                         static_cast<uint4 *>(y), c.T, c.E, nvec);
     };
     auto by_k = [&](auto elem) {
         using El = decltype(elem);
@@ -294,7 +431,7 @@ cudaError_t launch_combine(const moe_config &c, const void *Y_perm, const void *
         by_k(__nv_bfloat16());
     else
         by_k(float());
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace moe

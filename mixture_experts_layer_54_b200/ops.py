@@ -44,6 +44,11 @@ def _p(t):
         raise ValueError("moe ops take contiguous tensors (call .contiguous() on views)")
     if not t.is_cuda:
         raise ValueError("moe ops take CUDA tensors")
+    if t.device.index != torch.cuda.current_device():
+        # the library launches on the current device (and the no-allocation
+        # capacity call uses that device's static scratch)
+        raise ValueError(f"tensor on {t.device} but the current device is "
+                         f"cuda:{torch.cuda.current_device()}: use torch.cuda.device(...)")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -254,28 +259,33 @@ def moe_capacity_noalloc(cfg: MoeConfig, topk) -> CapacityOut:
     return out
 
 
-def moe_dispatch(cfg: MoeConfig, x, topk, pos, keep, offsets, x_perm=None):
+def moe_dispatch(cfg: MoeConfig, x, topk, pos, keep, offsets, x_perm=None, src_slot=None,
+                 zero_rows=None):
+    """Permuted rows; with src_slot (an int32 [moe_perm_rows] tensor) also the
+    assignment t k + j each kept row holds; with zero_rows ([T, d]) the rows of
+    tokens whose every slot was dropped are zeroed there."""
     if x_perm is None:
         x_perm = torch.empty((moe_perm_rows(cfg), cfg.d), dtype=_tdtype(cfg), device=_dev(x))
     check(lib().moe_dispatch(ctypes.byref(cfg), _p(x), _p(topk), _p(pos), _p(keep), _p(offsets),
-                             _p(x_perm), _stream()), "moe_dispatch")
+                             _p(x_perm), _p(src_slot), _p(zero_rows), _stream()), "moe_dispatch")
     return x_perm
 
 
-def moe_dispatch_rows(cfg: MoeConfig, topk, pos, keep, offsets, src_rows=None):
-    """The dispatch as a row table: src_rows[r] = token whose row goes to
-    permuted row r (0 for padding rows), for moe_expert_ffn_gather."""
-    if src_rows is None:
-        src_rows = torch.empty((moe_perm_rows(cfg),), dtype=torch.int32, device=_dev(offsets))
+def moe_dispatch_rows(cfg: MoeConfig, topk, pos, keep, offsets, src_slot=None):
+    """The dispatch as a row table: src_slot[r] = t k + j, the assignment whose
+    token row goes to permuted row r (-1 for padding rows), for the GEMMs that
+    gather their rows from x."""
+    if src_slot is None:
+        src_slot = torch.empty((moe_perm_rows(cfg),), dtype=torch.int32, device=_dev(offsets))
     check(lib().moe_dispatch_rows(ctypes.byref(cfg), _p(topk), _p(pos), _p(keep), _p(offsets),
-                                  _p(src_rows), _stream()), "moe_dispatch_rows")
-    return src_rows
+                                  _p(src_slot), _stream()), "moe_dispatch_rows")
+    return src_slot
 
 
-def moe_expert_ffn_gather(cfg: MoeConfig, x, src_rows, offsets, W1, W3, W2, Ws1=None, Ws3=None,
+def moe_expert_ffn_gather(cfg: MoeConfig, x, src_slot, offsets, W1, W3, W2, Ws1=None, Ws3=None,
                           Ws2=None, ws=None, Y_perm=None, Y_shared=None):
     """moe_expert_ffn with the dispatch fused in: routed rows read from x
-    through src_rows."""
+    through src_slot."""
     dev = _dev(x)
     if Y_perm is None:
         Y_perm = torch.empty((moe_perm_rows(cfg), cfg.d), dtype=_tdtype(cfg), device=dev)
@@ -283,11 +293,40 @@ def moe_expert_ffn_gather(cfg: MoeConfig, x, src_rows, offsets, W1, W3, W2, Ws1=
         Y_shared = torch.empty((cfg.T, cfg.d), dtype=_tdtype(cfg), device=dev)
     if ws is None:
         ws = workspace(moe_stage_workspace_size(cfg), dev)
-    check(lib().moe_expert_ffn_gather(ctypes.byref(cfg), _p(x), _p(src_rows), _p(offsets),
+    check(lib().moe_expert_ffn_gather(ctypes.byref(cfg), _p(x), _p(src_slot), _p(offsets),
                                       _p(W1), _p(W3), _p(W2), _p(Ws1), _p(Ws3), _p(Ws2),
                                       _p(Y_perm), _p(Y_shared), _p(ws), ws.numel(), _stream()),
           "moe_expert_ffn_gather")
     return Y_perm, Y_shared, ws
+
+
+def moe_expert_ffn_slots(cfg: MoeConfig, x_perm, x, src_slot, offsets, kept, gates, W1, W3, W2,
+                         Ws1=None, Ws3=None, Ws2=None, ws=None, Y_slot=None, Y_shared=None):
+    """moe_expert_ffn with the combine's gate in GEMM2's epilogue: Y_slot
+    [T k, d], row t k + j = gates[t, j] * FFN(x_t) for kept slots (others not
+    written).  x_perm None: rows gathered from x through src_slot."""
+    dev = _dev(src_slot)
+    if Y_slot is None:
+        Y_slot = torch.empty((cfg.T * cfg.k, cfg.d), dtype=_tdtype(cfg), device=dev)
+    if cfg.n_shared > 0 and Y_shared is None:
+        Y_shared = torch.empty((cfg.T, cfg.d), dtype=_tdtype(cfg), device=dev)
+    if ws is None:
+        ws = workspace(moe_stage_workspace_size(cfg), dev)
+    check(lib().moe_expert_ffn_slots(ctypes.byref(cfg), _p(x_perm), _p(x), _p(src_slot),
+                                     _p(offsets), _p(kept), _p(gates), _p(W1), _p(W3), _p(W2),
+                                     _p(Ws1), _p(Ws3), _p(Ws2), _p(Y_slot), _p(Y_shared), _p(ws),
+                                     ws.numel(), _stream()), "moe_expert_ffn_slots")
+    return Y_slot, Y_shared, ws
+
+
+def moe_combine_slots(cfg: MoeConfig, Y_slot, Y_shared, keep, residual=None, y=None):
+    """y[t] = sum of the kept rows t k + j of Y_slot (+ Y_shared[t])
+    (+ residual[t]), fp32 in slot order."""
+    if y is None:
+        y = torch.empty((cfg.T, cfg.d), dtype=_tdtype(cfg), device=_dev(Y_slot))
+    check(lib().moe_combine_slots(ctypes.byref(cfg), _p(Y_slot), _p(Y_shared), _p(keep),
+                                  _p(residual), _p(y), _stream()), "moe_combine_slots")
+    return y
 
 
 def moe_expert_ffn(cfg: MoeConfig, x_perm, offsets, W1, W3, W2, x=None, Ws1=None, Ws3=None,
@@ -460,14 +499,18 @@ __all__ = ["moe_config", "moe_validate", "moe_capacity_value", "moe_perm_rows",
            "HostStream", "moe_forward", "CapacityOut", "StagedForward", "moe_capacity_scored",
            "moe_seq_balance_loss", "moe_bias_update", "moe_clear_device_status",
            "moe_probe_wait_timeout", "moe_dispatch_rows", "moe_expert_ffn_gather",
+           "moe_expert_ffn_slots", "moe_combine_slots",
            "moe_capacity_sharded", "gather_shard_counts", "shard_losses"]
 
 
 class StagedForward:
-    """The forward as its six stage calls on preallocated buffers.  Runs the
-    same kernels as moe_forward; `events`, when given, are seven CUDA events
-    recorded before, between and after the stages so each stage's device time
-    can be read (route, capacity, dispatch, expert_ffn, combine, losses)."""
+    """The forward as its stage calls on preallocated buffers: the kernels
+    moe_forward runs, except that the losses are a launch of their own (the
+    forward computes them in the capacity launch, with the same bits);
+    `events`, when given, are seven CUDA events recorded before, between and
+    after the stages so each stage's device time can be read (route, capacity,
+    dispatch, expert_ffn, combine, losses).  A top-1 layer without shared
+    experts has its combine in the expert GEMM (the combine stage is empty)."""
 
     STAGES = ("route", "capacity", "dispatch", "expert_ffn", "combine", "losses")
 
@@ -492,6 +535,10 @@ class StagedForward:
         # batch-prioritized capacity ranks by the router scores [T, E]
         self.scores = e((T, E), torch.float32) if cfg.priority == 2 else None
         self.ws = workspace(moe_stage_workspace_size(cfg), dev)
+        # one slot per token and no shared expert: the combine's gate runs in the
+        # expert GEMM, which writes y (as moe_forward does)
+        self.fused_combine = cfg.k == 1 and cfg.n_shared == 0
+        self.slot = e((R,), torch.int32) if self.fused_combine else None
 
     def __call__(self, x, W_r, W1, W2, W3=None, logit_bias=None, select_bias=None, Ws1=None,
                  Ws3=None, Ws2=None, events=None):
@@ -513,16 +560,26 @@ class StagedForward:
                                  _p(self.n_dropped), _p(self.ws), self.ws.numel(), s),
                   "moe_capacity")
         rec(2)
+        fused = self.fused_combine
         check(L.moe_dispatch(c, _p(x), _p(self.topk), _p(self.pos), _p(self.keep),
-                             _p(self.offsets), _p(self.x_perm), s), "moe_dispatch")
+                             _p(self.offsets), _p(self.x_perm), _p(self.slot),
+                             _p(self.y) if fused else None, s), "moe_dispatch")
         rec(3)
-        check(L.moe_expert_ffn(c, _p(self.x_perm), _p(self.offsets), _p(W1), _p(W3), _p(W2),
-                               _p(x), _p(Ws1), _p(Ws3), _p(Ws2), _p(self.Y_perm), _p(self.Y_sh),
-                               _p(self.ws), self.ws.numel(), s), "moe_expert_ffn")
+        if fused:
+            check(L.moe_expert_ffn_slots(c, _p(self.x_perm), _p(x), _p(self.slot),
+                                         _p(self.offsets), _p(self.kept), _p(self.gates), _p(W1),
+                                         _p(W3), _p(W2), None, None, None, _p(self.y), None,
+                                         _p(self.ws), self.ws.numel(), s), "moe_expert_ffn_slots")
+        else:
+            check(L.moe_expert_ffn(c, _p(self.x_perm), _p(self.offsets), _p(W1), _p(W3), _p(W2),
+                                   _p(x), _p(Ws1), _p(Ws3), _p(Ws2), _p(self.Y_perm),
+                                   _p(self.Y_sh), _p(self.ws), self.ws.numel(), s),
+                  "moe_expert_ffn")
         rec(4)
-        check(L.moe_combine(c, _p(self.Y_perm), _p(self.Y_sh), _p(self.gates), _p(self.topk),
-                            _p(self.pos), _p(self.keep), _p(self.offsets), None, _p(self.y), s),
-              "moe_combine")
+        if not fused:   # (fused: the combine ran in the expert GEMM)
+            check(L.moe_combine(c, _p(self.Y_perm), _p(self.Y_sh), _p(self.gates), _p(self.topk),
+                                _p(self.pos), _p(self.keep), _p(self.offsets), None, _p(self.y),
+                                s), "moe_combine")
         rec(5)
         check(L.moe_losses(c, _p(self.counts), _p(self.partials), _p(self.aux), _p(self.zloss),
                            s), "moe_losses")

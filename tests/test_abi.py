@@ -47,6 +47,15 @@ def test_capacity_value_worked_example():
     assert moe.moe_capacity_value(moe.moe_config(CONFIGS["deepseekmoe"])) == 2304
 
 
+def test_capacity_value_is_held_at_T_for_huge_factors():
+    # an expert receives at most T assignments; a huge finite factor must not
+    # overflow the integer conversion (it keeps everything, like +infinity)
+    cfg = moe.moe_config(T=4096, d=1024, E=8, k=2, d_ff=4096, dtype=1, cf=1e20)
+    assert moe.moe_capacity_value(cfg) == 4096
+    assert moe.moe_capacity_value(moe.moe_config(cfg, cf=1.25, T=10, E=2)) == 10
+    assert moe.moe_perm_rows(cfg) == moe.moe_perm_rows(moe.moe_config(cfg, cf=math.inf))
+
+
 @pytest.mark.parametrize("kw", [dict(k=9, E=8), dict(k=3, E=2), dict(E=300, k=2),
                                 dict(d=100), dict(d_ff=100), dict(T=-1)])
 def test_bad_shapes_are_rejected(kw):

@@ -82,3 +82,22 @@ def test_peaks_fall_back_when_the_file_is_missing(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     peaks, src = bench.load_peaks()
     assert src == "fallback" and peaks["hbm_gbs"] == 6650.0
+
+
+def test_layer_summary_rates_and_roofline():
+    peaks = dict(bench.FALLBACK_PEAKS)
+    s = CONFIGS["deepseek_v3"]
+    kept = s.T * s.k
+    stage_ms = {"route": 0.1, "capacity": 0.01, "dispatch": 0.1, "expert_ffn": 4.0,
+                "combine": 0.1, "losses": 0.01}
+    ms = sum(stage_ms.values())
+    out = bench.summarize_layer(s, ms, stage_ms, kept, 0, steps=100, peaks=peaks)
+    w = bench.layer_work(s, None, kept, 0)
+    ffn = out["expert_ffn"]
+    assert ffn["TFLOP/s"] == round(w["expert_ffn"]["flops"] / 4e-3 / 1e12, 1)
+    # 22.6 GB of expert weights: the layer is bound by its bytes, not its FLOPs
+    assert out["layer_roofline"]["bound"] == "hbm" and ffn["bound"] == "hbm"
+    assert 0 < out["layer_roofline"]["frac"] <= 1
+    assert out["stages"]["dispatch"]["GB/s"] == round(w["dispatch"]["bytes"] / 1e-4 / 1e9, 1)
+    assert bench.summarize_layer(CONFIGS["mixtral"], 4.3, {**stage_ms, "expert_ffn": 4.0}, 16384,
+                                 0, 200, peaks)["layer_roofline"]["bound"] == "tensor"

@@ -76,6 +76,55 @@ def test_expert_ffn_grouped_gemm_against_torch(act, dims, pair):
         _close_bf16(Y[rows], ref)
 
 
+@pytest.mark.parametrize("act", [0, 1])
+def test_pair_gemm_with_many_tiles_per_sm_pair(act):
+    """SM-pair tiles where every SM pair runs many tiles in turn (GEMM1: 16 N
+    tiles x ~70 row pairs over 74 pairs), so the TMEM double buffer and the
+    shared-memory ring wrap many times; ragged segments, every kept row
+    compared with its expert's FFN in float64."""
+    d, F = 1024, 2048
+    kept = [4000, 1, 2900, 0, 5000, 129, 2047, 3300]
+    E = len(kept)
+    cfg = moe.moe_config(T=16384, d=d, E=E, k=2, d_ff=F, act=act, dtype=1, cf=math.inf)
+    R = moe.moe_perm_rows(cfg)
+    offsets = _segments(kept)
+    assert offsets[-1] <= R
+    g = torch.Generator(device=DEV).manual_seed(17 + act)
+    x_perm = torch.randn((R, d), generator=g, device=DEV).to(torch.bfloat16)
+    W1 = (torch.randn((E, F, d), generator=g, device=DEV) / math.sqrt(d)).to(torch.bfloat16)
+    W3 = (torch.randn((E, F, d), generator=g, device=DEV) / math.sqrt(d)).to(torch.bfloat16) \
+        if act == 1 else None
+    W2 = (torch.randn((E, d, F), generator=g, device=DEV) / math.sqrt(F)).to(torch.bfloat16)
+    off_t = torch.tensor(offsets, dtype=torch.int32, device=DEV)
+    Y, _, ws = moe.moe_expert_ffn(cfg, x_perm, off_t, W1, W3, W2)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status(ws) == 0
+    for e in range(E):
+        if kept[e] == 0:
+            continue
+        rows = slice(offsets[e], offsets[e] + kept[e])
+        ref = _ffn_ref(x_perm[rows], W1[e], None if W3 is None else W3[e], W2[e], act)
+        _close_bf16(Y[rows], ref)
+        # and row by row: no row may be wrong while the segment's norm is fine
+        err = (Y[rows].double() - ref).abs().amax(dim=1)
+        assert err.max().item() <= BF16_MAX_ABS * ref.abs().max().item()
+
+
+def test_capacity_with_a_huge_factor_keeps_everything():
+    """A finite factor far above T k / E holds C at T: nothing is dropped
+    (the integer conversion of ceil(cf T k / E) would overflow otherwise)."""
+    T, E, k = 1000, 8, 2
+    rng = np.random.default_rng(3)
+    topk = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    cfg = moe.moe_config(T=T, d=64, E=E, k=k, d_ff=64, dtype=1, cf=1e20)
+    assert moe.moe_capacity_value(cfg) == T
+    cap = moe.moe_capacity(cfg, torch.tensor(topk, device=DEV))
+    torch.cuda.synchronize()
+    assert int(cap.n_dropped.item()) == 0
+    assert bool(cap.keep.bool().all().item())
+    np.testing.assert_array_equal(cap.counts.cpu().numpy(), np.bincount(topk.ravel(), minlength=E))
+
+
 @pytest.mark.parametrize("act,S,T", [(1, 2, 333), (0, 1, 333), (1, 1, 333), (1, 2, 2100),
                                      (0, 1, 2100)])
 def test_shared_experts_against_torch(act, S, T):
@@ -276,7 +325,8 @@ def test_gathered_expert_ffn_equals_dispatch_then_ffn(case):
     pick = torch.rand((T, E), generator=g, device=DEV) + torch.linspace(0.5, 0, E, device=DEV)
     topk = pick.argsort(dim=1, descending=True)[:, :k].to(torch.int32).contiguous()
     cap = moe.moe_capacity(cfg, topk)
-    x_perm = moe.moe_dispatch(cfg, x, topk, cap.pos, cap.keep, cap.offsets)
+    slot_copy = torch.full((moe.moe_perm_rows(cfg),), -7, dtype=torch.int32, device=DEV)
+    x_perm = moe.moe_dispatch(cfg, x, topk, cap.pos, cap.keep, cap.offsets, src_slot=slot_copy)
     Y_ref, Ysh_ref, ws1 = moe.moe_expert_ffn(cfg, x_perm, cap.offsets, W1, W3, W2, x, Ws1, Ws3,
                                              Ws2)
     rows = moe.moe_dispatch_rows(cfg, topk, cap.pos, cap.keep, cap.offsets)
@@ -286,15 +336,20 @@ def test_gathered_expert_ffn_equals_dispatch_then_ffn(case):
     tk, pos, keep = topk.cpu().numpy(), cap.pos.cpu().numpy(), cap.keep.cpu().numpy()
     off = cap.offsets.cpu().numpy()
     assert keep.sum() < T * k   # something was dropped
-    want = np.zeros(moe.moe_perm_rows(cfg), np.int32)
+    # the table: row offsets[e] + pos[t, j] holds assignment t k + j, padding -1
+    want = np.full(moe.moe_perm_rows(cfg), -1, np.int32)
     kept_rows = []
     for t in range(T):
         for j in range(k):
             if keep[t, j]:
                 r = off[tk[t, j]] + pos[t, j]
-                want[r] = t
+                want[r] = t * k + j
                 kept_rows.append(r)
     np.testing.assert_array_equal(rows.cpu().numpy(), want)
+    # the copying dispatch writes the same entries for kept rows, no others
+    sc = slot_copy.cpu().numpy()
+    np.testing.assert_array_equal(sc[kept_rows], want[kept_rows])
+    assert np.all(np.delete(sc, kept_rows) == -7)
     kr = torch.as_tensor(kept_rows, device=DEV, dtype=torch.long)
     assert torch.equal(Y[kr], Y_ref[kr])
     if S:
@@ -344,17 +399,22 @@ def test_route_selection_every_width(E, k, score):
 
 
 @pytest.mark.parametrize("T,d,E,k", [
-    (1000, 1024, 4, 1),    # 4 experts per token group, K in 4 parts (cluster of 4)
+    (1000, 1024, 4, 1),    # one kernel: 4 experts per token group, K in 4 parts (cluster of 4)
     (777, 512, 8, 2),      # 8 experts per token group, K in 2 parts
     (1000, 1024, 16, 4),   # a warp per token, K in 4 parts
-    (600, 512, 40, 3),     # 48-wide expert chunk, K in 2 parts
-    (333, 1024, 64, 6),    # 64-wide chunk, K in 4 parts, ragged last tile
-    (500, 512, 100, 8),    # 2 expert chunks x 2 K parts
-    (64, 256, 8, 2),       # less than one 128-token tile
-    (40, 256, 200, 8),     # 4 expert chunks, two rows of the loss partials
+    (600, 512, 40, 3),     # 48 padded experts, two per lane, K in 2 parts
+    (333, 1024, 64, 6),    # 64 experts (3 x 64 = 192-wide MMA), 3 x stages, ragged last tile
+    (16384, 1024, 8, 2),   # 128 tiles: every cluster walks several (both accumulators and
+                           # logit buffers reused many times)
+    (16384, 1024, 64, 6),  # DeepSeekMoE-shaped: 4 tiles per cluster of 4
+    (20000, 512, 32, 4),   # 157 tiles on clusters of 2, ragged last tile
+    (500, 512, 100, 8),    # three launches: 2 expert chunks x 2 K parts
+    (64, 256, 8, 2),       # less than one 128-token tile (one block, K whole)
+    (40, 256, 200, 8),     # three launches: 4 expert chunks, two rows of the loss partials
 ])
 @pytest.mark.parametrize("score", [0, 1], ids=["softmax", "sigmoid"])
 def test_route_cluster_shapes(T, d, E, k, score):
-    """Every way the blocks of a token tile split the work (K parts, expert
-    chunks, clusters of 1, 2 or 4 blocks): the same checks as above."""
+    """Every way the router splits the work (one kernel: K parts over a
+    cluster of 1, 2 or 4 blocks, one or many 128-token tiles per cluster;
+    three launches: expert chunks and K parts): the same checks as above."""
     _check_route(T, d, E, k, score, T + d + E + k + score)

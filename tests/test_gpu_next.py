@@ -136,9 +136,16 @@ def test_forward_with_score_priority_matches_the_oracle(name):
     sure = ~np.isin(topk, list(unsure)) if unsure else np.ones_like(topk, dtype=bool)
     keep = fwd.keep.cpu().numpy()
     np.testing.assert_array_equal(keep[sure], ref.cap.keep[sure])
+    sel = oracle.selected_scores(ref.route.scores, ref.route.topk).astype(np.float64)
     for e in unsure:   # valid: the kept ones of e are its highest-scored, C of them
         m = topk == e
         assert keep[m].sum() == min(m.sum(), ref.cap.C)
+        kept_s, dropped_s = sel[m & (keep == 1)], sel[m & (keep == 0)]
+        if kept_s.size and dropped_s.size:
+            # every kept score is at least every dropped score of the expert,
+            # up to the fp32 near-tie window
+            lo, hi = kept_s.min(), dropped_s.max()
+            assert lo >= hi - 1e-5 * max(abs(hi), 1e-30), (e, lo, hi)
     tokens = np.nonzero(sure.all(axis=1))[0]
     assert tokens.size >= 0.9 * shape.T
     got = fwd.y[torch.as_tensor(tokens, device="cuda")].double().cpu().numpy()

@@ -94,6 +94,32 @@ def check_capacity(counts, keep, dropped, ref, pos=None, n_dropped=None):
         assert int(n_dropped.item()) == ref.cap.n_dropped
 
 
+def tile_stratified_tokens(topk, pos, keep, E, seed=54, tile=128):
+    """Tokens that reach every tile of every expert segment: for each expert,
+    one kept row drawn at random inside each 128-row tile of its segment (so
+    both 128-row halves of every 256-row SM-pair tile, and a varying TMEM lane
+    and epilogue warp), plus the segment's first and last kept rows; mapped
+    back to the token that owns the row."""
+    rng = np.random.default_rng(seed)
+    kept_rows = {}
+    t_idx, j_idx = np.nonzero(keep)
+    for t, j in zip(t_idx, j_idx):
+        kept_rows.setdefault(int(topk[t, j]), {})[int(pos[t, j])] = int(t)
+    tokens = set()
+    for e in range(E):
+        rows = kept_rows.get(e)
+        if not rows:
+            continue
+        n = len(rows)
+        assert sorted(rows) == list(range(n)), "kept positions of an expert are 0..kept-1"
+        tokens.add(rows[0])
+        tokens.add(rows[n - 1])
+        for lo in range(0, n, tile):
+            hi = min(lo + tile, n)
+            tokens.add(rows[int(rng.integers(lo, hi))])
+    return tokens
+
+
 SMALL = {
     "tiny": CONFIGS["tiny"],
     "switch_small": shrink(CONFIGS["switch"], T=1000, d=256, d_ff=512),
@@ -106,6 +132,10 @@ SMALL = {
                                 d_ff_shared=192),
     "k_equals_E": shrink(CONFIGS["mixtral"], T=200, d=128, d_ff=128, E=4, k=4, cf=math.inf),
     "single_expert": shrink(CONFIGS["mixtral"], T=130, d=64, d_ff=64, E=1, k=1, cf=1.0),
+    # T k = 512 E: the expert GEMMs run SM-pair (256-row) tiles over the full
+    # Mixtral-shaped K (d = 4096, d_ff = 14336), many tiles per SM pair, odd
+    # trailing 128-row halves; every token compared
+    "mixtral_full_k_pair": shrink(CONFIGS["mixtral"], T=2048),
 }
 
 
@@ -124,8 +154,66 @@ def test_every_token_matches_the_oracle(name):
     np.testing.assert_allclose(out["logits"].double().cpu().numpy(), ref.route.z, rtol=1e-4,
                                atol=1e-4)
     fwd = run_forward(inp)
-    assert torch.equal(fwd.y, out["y"])
     assert torch.equal(fwd.topk, out["topk"])
+    check_losses(fwd.aux, fwd.zloss, ref)
+    if inp.shape.k == 1 and inp.shape.n_shared == 0:
+        # the forward fuses this layer's combine into the expert GEMM (y rounded
+        # once, not twice): its own comparison with the oracle
+        check_y(inp.shape, fwd.y, ref.y)
+    else:   # the same kernels as the stage calls
+        assert torch.equal(fwd.y, out["y"])
+        assert torch.equal(fwd.aux, out["aux"]) and torch.equal(fwd.zloss, out["zloss"])
+
+
+def run_fused_combine(inp, gather, direct=False):
+    """The combine's gate fused into GEMM2 (moe_expert_ffn_slots), then the
+    ordered slot sum (moe_combine_slots); gather: the dispatch fused into GEMM1
+    too (moe_dispatch_rows).  direct (k = 1, no shared expert): GEMM2 writes y
+    itself, the dispatch zeroes the rows of dropped tokens."""
+    s = inp.shape
+    cfg = moe.moe_config(s)
+    topk, gates, _, _, _ = moe.moe_route(cfg, inp.x, inp.W_r, inp.logit_bias, inp.select_bias)
+    cap = moe.moe_capacity(cfg, topk)
+    R = moe.moe_perm_rows(cfg)
+    y = torch.full((s.T, s.d), float("nan"), dtype=inp.x.dtype, device="cuda")
+    if gather:
+        slot = moe.moe_dispatch_rows(cfg, topk, cap.pos, cap.keep, cap.offsets)
+        x_perm = None
+    else:
+        slot = torch.empty((R,), dtype=torch.int32, device="cuda")
+        x_perm = moe.moe_dispatch(cfg, inp.x, topk, cap.pos, cap.keep, cap.offsets,
+                                  src_slot=slot, zero_rows=y if direct else None)
+    Y_slot, Ysh, ws = moe.moe_expert_ffn_slots(cfg, x_perm, inp.x, slot, cap.offsets, cap.kept,
+                                               gates, inp.W1, inp.W3, inp.W2, inp.Ws1, inp.Ws3,
+                                               inp.Ws2, Y_slot=y if direct else None)
+    if not direct:
+        moe.moe_combine_slots(cfg, Y_slot, Ysh, cap.keep, y=y)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status(ws) == 0
+    return y, topk, cap
+
+
+FUSED = [n for n in SMALL if n != "mixtral_full_k_pair"]
+
+
+@pytest.mark.parametrize("gather", [False, True], ids=["copy", "gather"])
+@pytest.mark.parametrize("name", FUSED)
+def test_fused_combine_matches_the_oracle(name, gather):
+    """NEXT-2: the gate applied in GEMM2's epilogue, each kept row written to
+    its assignment's row, then a plain ordered sum of a token's contiguous
+    rows; with and without the dispatch fused into GEMM1.  Every token
+    compared with the oracle (dropped slots contribute nothing, fully dropped
+    tokens get the shared experts or 0)."""
+    inp = remove_near_ties(generate(SMALL[name], device="cuda"))
+    ref = oracle_forward(inp)
+    y, topk, cap = run_fused_combine(inp, gather)
+    np.testing.assert_array_equal(topk.cpu().numpy(), ref.route.topk)
+    np.testing.assert_array_equal(cap.keep.cpu().numpy(), ref.cap.keep)
+    check_y(inp.shape, y, ref.y)
+    if inp.shape.k == 1 and inp.shape.n_shared == 0 and not gather:
+        y2, _, _ = run_fused_combine(inp, gather, direct=True)
+        check_y(inp.shape, y2, ref.y)
+        assert not torch.isnan(y2.float()).any()   # dropped tokens' rows were zeroed
 
 
 def test_drops_happen_and_dropped_tokens_get_zero():
@@ -144,8 +232,10 @@ def test_drops_happen_and_dropped_tokens_get_zero():
 @pytest.mark.parametrize("name", ["tiny", "switch", "mixtral", "deepseekmoe", "deepseek_v3"])
 def test_full_size_config(name):
     """Full sizes, launched as the benchmark launches them: routing, capacity
-    and drops bit-exact on every token, losses on every token, y on a sample
-    of tokens the oracle computes one by one."""
+    and drops bit-exact on every token, losses on every token, y on a
+    tile-stratified sample of tokens the oracle computes one by one (a row in
+    every 128-row tile of every expert segment, each segment's first and last
+    kept rows, the first and last token and a dropped token)."""
     shape = CONFIGS[name]
     inp = remove_near_ties(generate(shape, device="cuda"))
     fwd = run_forward(inp)
@@ -160,8 +250,9 @@ def test_full_size_config(name):
     assert int(fwd.n_dropped.item()) == cap.n_dropped
     assert float(fwd.aux.item()) == pytest.approx(aux, rel=LOSS_RTOL)
     assert float(fwd.zloss.item()) == pytest.approx(zl, rel=LOSS_RTOL)
-    rng = np.random.default_rng(54)
-    tokens = set(rng.choice(shape.T, size=min(10, shape.T), replace=False).tolist())
+    # y on a tile-stratified sample: every 128-row tile of every expert
+    # segment (both halves of each SM-pair tile) holds a compared row
+    tokens = tile_stratified_tokens(r.topk, cap.pos, cap.keep, shape.E)
     tokens |= {0, shape.T - 1}
     dropped = np.nonzero(cap.dropped)[0]
     if dropped.size:

@@ -42,7 +42,7 @@ def test_noalloc_capacity_matches_the_workspace_version_on_two_calls(priority):
 
 
 def test_noalloc_capacity_rejects_shapes_beyond_its_static_scratch():
-    # ceil(T/256) * k * E > 65536 entries per table
+    # ceil(T/256) * k * E > 65536 entries of the histogram table
     cfg = moe.moe_config(T=256 * 40, d=64, E=256, k=8, d_ff=64, dtype=1, cf=1.0)
     topk = torch.zeros((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
     with pytest.raises(moe.MoEError) as ei:
