@@ -112,7 +112,7 @@ def parse(argv=None):
     ap.add_argument("--no-per-layer", action="store_true",
                     help="skip the Switch, DeepSeekMoE and DeepSeek-V3 shaped layers that the "
                          "default (Mixtral-shaped) run also times")
-    ap.add_argument("--stage", choices=["route", "ffn"], default=None,
+    ap.add_argument("--stage", choices=["route", "ffn", "forward"], default=None,
                     help="time one stage alone on the workload's tensors (profiling aid; "
                          "prints its own JSON line, not the benchmark line)")
     ap.add_argument("--experts", type=int, default=None,
@@ -812,10 +812,43 @@ def run_stage_ffn(args):
                       "timing": "back-to-back calls, CUDA events (launch gaps included)"}))
 
 
+def run_stage_forward(args):
+    """The whole layer through moe_forward, eagerly: W warm-up calls, then K
+    calls between CUDA events (launch gaps included).  The small command the
+    kernel launch list is taken from."""
+    import mixture_experts_layer_54_b200 as moe
+    device = torch.device("cuda", 0)
+    shape = CONFIGS[args.config]
+    inp = generate(shape, device)
+    cfg = moe.moe_config(shape)
+    fwd = moe.MoEForward(cfg, device)
+    w = moe.weights_struct(inp.W_r, inp.W1, inp.W2, inp.W3, inp.logit_bias, inp.select_bias,
+                           inp.Ws1, inp.Ws3, inp.Ws2)
+    for _ in range(max(args.warmup, 1)):
+        fwd(inp.x, w)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fwd(inp.x, w)
+    e1.record()
+    torch.cuda.synchronize()
+    if moe.moe_device_status(fwd.ws) != 0:
+        raise SystemExit("device status set: a bounded wait expired")
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"stage": "forward", "workload": workload_name(shape), "calls": args.steps,
+                      "ms_per_call": round(ms, 4), "tokens/s": round(shape.T / ms * 1e3, 1),
+                      "kernels_per_call": kernels_per_step(shape),
+                      "timing": "back-to-back eager calls, CUDA events (launch gaps included)"}))
+
+
 def main(argv=None):
     args = parse(argv)
     if args.stage == "ffn":
         run_stage_ffn(args)
+        return
+    if args.stage == "forward":
+        run_stage_forward(args)
         return
     if args.stage:
         run_stage(args)

@@ -52,12 +52,21 @@ constexpr int CHUNK = 32;                            // epilogue columns per ste
 constexpr int STG_BYTES = 32 * CHUNK * 2;            // 32 rows x 32 bf16 = 2 KB
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BYTES;
-constexpr int OFF_TILES = OFF_BAR + 256;
-constexpr int SMEM_BYTES = OFF_TILES + 2 * 4 * (kMaxE + 1) + 1024;   // + alignment slack
+// Shared-memory plan of the single-SM kernel for MT row tiles per tile: MT = 1,
+// four stages of A (16 KB) + B (32 KB); MT = 2, three stages of two A boxes
+// (the tile's two 128-row halves, 32 KB) + one B box that both halves share.
+template <int MT>
+struct Smem1 {
+    static constexpr int ST = MT == 1 ? STAGES : 3;
+    static constexpr int A_ST = MT * A_BYTES;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + ST * A_ST;
+    static constexpr int OFF_STG = OFF_B + ST * B_BYTES;
+    static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BYTES;
+    static constexpr int OFF_TILES = OFF_BAR + 256;
+    static constexpr int BYTES = OFF_TILES + 2 * 4 * (kMaxE + 1) + 1024;   // + alignment slack
+    static_assert(BYTES <= 227 * 1024, "shared memory");
+};
 
 // EPI_GATED: GEMM2 with the combine's gate fused (routed rows only): row r
 // of expert e's segment, when kept (r - offsets[e] < kept[e]), holds
@@ -93,6 +102,7 @@ struct __align__(64) Params {
     const int32_t *offsets;
     int32_t *status;
     int clear_status;            // 1: block 0 clears the status word before any wait
+    int b_stream;                // 1: routed B (weights) boxes loaded evict-first in L2
     unsigned long long timeout_ns;
 };
 
@@ -305,6 +315,26 @@ __device__ __forceinline__ void store_gated(const Params &p, int a, float gate, 
     }
 }
 
+// As tma_load_3d, with an L2 cache policy (createpolicy) for the box.
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                                 int c0, int c1, int c2, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+// L2 policy for data read once: evicted first, so it does not push out data
+// that is read again (the token rows every N tile of an expert re-reads).
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
                                              int c2)
 {
@@ -379,15 +409,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
 struct Tile {
     int set;
     int m0;       // first row of A and C
+    int halves;   // 128-row halves of the tile holding rows of its segment (1 or 2)
     int b_group;  // group of the B tensor (K not split)
     int b_row;    // first B row inside the group
     int c_col;    // first C column
     int c_group;  // group of the C tensor
 };
 
+// Tile `tile` of MT x 128 rows: routed tiles expert by expert, N outer and
+// row tiles inner; then the shared set over its dense rows.
+template <int MT>
 __device__ __forceinline__ Tile decode(const Params &p, const int *tstart, const int *mtiles,
                                        int routed_total, int tile, int bn_b, int bn_out)
 {
+    constexpr int TM = MT * BM;
     Tile t;
     if (tile < routed_total) {
         int lo = 0, hi = p.E;   // last e with tstart[e] <= tile
@@ -401,7 +436,8 @@ __device__ __forceinline__ Tile decode(const Params &p, const int *tstart, const
         const int e = lo, i = tile - tstart[e], mt = mtiles[e];
         const int n = i / mt, m = i % mt;
         t.set = 0;
-        t.m0 = p.offsets[e] + m * BM;
+        t.m0 = p.offsets[e] + m * TM;
+        t.halves = MT == 2 && t.m0 + BM < p.offsets[e + 1] ? 2 : 1;
         t.b_group = e;
         t.b_row = n * bn_b;
         t.c_col = n * bn_out;
@@ -409,11 +445,12 @@ __device__ __forceinline__ Tile decode(const Params &p, const int *tstart, const
     } else {
         const SetDesc &s = p.set[1];
         const int i = tile - routed_total;
-        const int mt = (s.rows + BM - 1) / BM;
+        const int mt = (s.rows + TM - 1) / TM;
         const int n = i / mt, m = i % mt;
         const int g = n / s.n_tiles, nn = n % s.n_tiles;
         t.set = 1;
-        t.m0 = m * BM;
+        t.m0 = m * TM;
+        t.halves = MT == 2 && t.m0 + BM < s.rows ? 2 : 1;
         t.b_group = g;
         t.b_row = nn * bn_b;
         t.c_col = nn * bn_out;
@@ -443,19 +480,29 @@ __device__ __forceinline__ void epilogue_chunk(const float *g, const float *u, u
     }
 }
 
-template <int EPI, bool GATHER>
+// MT = 2: a tile covers up to 256 rows of one segment as two 128-row halves
+// with their own accumulators (TMEM columns 0 and 256) and one shared B box
+// per K step, so a weight tile is read once for up to 256 rows; a half past
+// the segment's end is neither loaded nor computed.  The two accumulators take
+// all of TMEM, so MT = 2 tiles are not double buffered.
+template <int EPI, bool GATHER, int MT>
 __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     grouped_gemm_kernel(const __grid_constant__ Params p)
 {
+    static_assert(MT == 1 || (MT == 2 && !GATHER), "row tiles per tile");
+    using L = Smem1<MT>;
+    constexpr int STAGES = L::ST;                              // (shadows the 4-stage default)
+    constexpr int A_ST = L::A_ST;
+    constexpr int NBUF = MT == 1 ? 2 : 1;                      // accumulator sets in TMEM
     constexpr int BN_B = EPI == EPI_SWIGLU ? BN / 2 : BN;     // B rows per tensor per tile
     constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;   // output columns per tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    const uint32_t sA = smem_u32(smem + OFF_A);
-    const uint32_t sB = smem_u32(smem + OFF_B);
-    const uint32_t sStg = smem_u32(smem + OFF_STG);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    const uint32_t sA = smem_u32(smem + L::OFF_A);
+    const uint32_t sB = smem_u32(smem + L::OFF_B);
+    const uint32_t sStg = smem_u32(smem + L::OFF_STG);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
     // full[0..S), empty[S..2S), tfull[2S, 2S+2), tempty[2S+2, 2S+4), drain 2S+4
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -463,10 +510,10 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8 * (2 * STAGES + 5));
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_BAR + 8 * (2 * STAGES + 5));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *tstart = reinterpret_cast<int *>(smem + OFF_TILES);    // [E + 1]
-    int *mtiles = tstart + (kMaxE + 1);                         // [E]
+    int *tstart = reinterpret_cast<int *>(smem + L::OFF_TILES);   // [E + 1]
+    int *mtiles = tstart + (kMaxE + 1);                          // [E]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Ctl ctl{abort_flag, p.status, p.timeout_ns};
@@ -501,7 +548,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     int routed_total = 0;
     if (p.set[0].routed && p.nsets > 0) {
         for (int e = threadIdx.x; e < p.E; e += blockDim.x)
-            mtiles[e] = (p.offsets[e + 1] - p.offsets[e]) / BM;
+            mtiles[e] = ((p.offsets[e + 1] - p.offsets[e]) / BM + MT - 1) / MT;
         __syncthreads();
         if (threadIdx.x == 0) {
             int acc = 0;
@@ -520,7 +567,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     int shared_total = 0;
     if (p.nsets > 1) {
         const SetDesc &s = p.set[1];
-        shared_total = (s.rows + BM - 1) / BM * s.n_tiles * s.n_groups;
+        shared_total = (s.rows + MT * BM - 1) / (MT * BM) * s.n_tiles * s.n_groups;
     }
     const int total = routed_total + shared_total;
     const uint32_t tmem_base = *tmem_slot;
@@ -530,6 +577,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
         // Lane 0 owns the barrier waits and the box copies (with gathered A
         // rows, the B boxes only: the gather warps copy A).
         if (lane == 0) {
+            const uint64_t b_policy = l2_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             int issued[STAGES];
@@ -538,7 +586,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                 issued[s] = 0, last_phase[s] = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+                const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
                 const SetDesc &sd = p.set[t.set];
                 const bool gath = GATHER && t.set == 0;
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
@@ -552,15 +600,23 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                         kcol = (kb % sd.kbg) * BK;
                     }
                     const uint32_t fb = full_bar(stage);
-                    mbar_expect_tx(fb, (gath ? 0 : A_BYTES) + B_BYTES);
+                    mbar_expect_tx(fb, (gath ? 0 : t.halves * A_BYTES) + B_BYTES);
                     if (!gath)
-                        tma_load_3d(sA + stage * A_BYTES, &p.tmA[t.set], fb, kcol, t.m0, ga);
-                    if (EPI == EPI_SWIGLU) {
-                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
-                        tma_load_3d(sB + stage * B_BYTES + B_BYTES / 2, &p.tmB3[t.set], fb, kcol,
-                                    t.b_row, gb);
+                        for (int h = 0; h < t.halves; ++h)
+                            tma_load_3d(sA + stage * A_ST + h * A_BYTES, &p.tmA[t.set], fb, kcol,
+                                        t.m0 + h * BM, ga);
+                    const uint32_t b0 = sB + stage * B_BYTES;
+                    const bool stream = p.b_stream && t.set == 0;
+                    if (stream) {
+                        tma_load_3d_hint(b0, &p.tmB[t.set], fb, kcol, t.b_row, gb, b_policy);
+                        if (EPI == EPI_SWIGLU)
+                            tma_load_3d_hint(b0 + B_BYTES / 2, &p.tmB3[t.set], fb, kcol, t.b_row,
+                                             gb, b_policy);
+                    } else if (EPI == EPI_SWIGLU) {
+                        tma_load_3d(b0, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                        tma_load_3d(b0 + B_BYTES / 2, &p.tmB3[t.set], fb, kcol, t.b_row, gb);
                     } else {
-                        tma_load_3d(sB + stage * B_BYTES, &p.tmB[t.set], fb, kcol, t.b_row, gb);
+                        tma_load_3d(b0, &p.tmB[t.set], fb, kcol, t.b_row, gb);
                     }
                     issued[stage] = 1;
                     last_phase[stage] = phase;
@@ -584,13 +640,15 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
             uint32_t acc_phase = 0;
             bool ok = true, any = false;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+                const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
                 const SetDesc &sd = p.set[t.set];
                 if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, ctl)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                // MT = 1: accumulator set acc at columns acc * 256; MT = 2: the
+                // halves at columns 0 and 256
                 const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
                     if (!wait_bar(full_bar(stage), phase, ctl)) {
@@ -598,11 +656,13 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_base = sA + stage * A_BYTES, b_base = sB + stage * B_BYTES;
+                    const uint32_t b_base = sB + stage * B_BYTES;
+                    for (int h = 0; h < t.halves; ++h) {
+                        const uint32_t a_base = sA + stage * A_ST + h * A_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        mma_bf16(tmem_d, sdesc_sw128(a_base + kk * 32), sdesc_sw128(b_base + kk * 32),
-                                 (kb | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_bf16(tmem_d + (uint32_t)(h * BN), sdesc_sw128(a_base + kk * 32),
+                                     sdesc_sw128(b_base + kk * 32), (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit(empty_bar(stage));
                     any = true;
@@ -614,7 +674,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                 if (!ok)
                     break;
                 mma_commit(tfull_bar(acc));
-                if (++acc == 2) {
+                if (++acc == NBUF) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
@@ -637,7 +697,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
         uint32_t phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+            const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
             const SetDesc &sd = p.set[t.set];
             const bool gath = t.set == 0;   // shared-expert tiles: TMA boxes of x
             int tok[G::NI];
@@ -651,7 +711,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                     break;
                 }
                 if (gath)
-                    gather_stage<1>(sA + stage * A_BYTES, 0, p.xg, p.x_ld, kb * BK, tok, gw, lane);
+                    gather_stage<1>(sA + stage * A_ST, 0, p.xg, p.x_ld, kb * BK, tok, gw, lane);
                 cp_async_commit();
                 if (seq >= D) {
                     cp_async_wait<D>();
@@ -673,20 +733,23 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
         const int ew = warp - 2;                     // staging buffer owner
         const int half = ew >> 2;                    // which half of the columns
         const uint32_t stg = sStg + ew * STG_BYTES;
-        uint8_t *stg_ptr = smem + OFF_STG + ew * STG_BYTES;
+        uint8_t *stg_ptr = smem + L::OFF_STG + ew * STG_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+            const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
             if (!wait_bar(tfull_bar(acc), acc_phase, ctl))
                 break;
             tc_fence_after();
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const int c_end = min((half + 1) * (BN_OUT / 2), p.set[t.set].c_cols - t.c_col);
+            for (int h = 0; h < t.halves; ++h) {
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) +
+                                   (uint32_t)((acc + h) * BN);
+            const int row0 = t.m0 + h * BM + q * 32;   // this warp's 32 rows
             if (EPI == EPI_GATED && t.set == 0) {
                 // gate and scatter: this lane's row goes to its assignment's row
                 float gate;
-                const int a = gated_slot(p, t.b_group, t.m0 + q * 32 + lane, &gate);
+                const int a = gated_slot(p, t.b_group, row0 + lane, &gate);
 #pragma unroll 1
                 for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
                     float g[CHUNK];
@@ -722,9 +785,10 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&p.tmC[t.set], stg, t.c_col + c, t.m0 + q * 32, t.c_group);
+                    tma_store_3d(&p.tmC[t.set], stg, t.c_col + c, row0, t.c_group);
                     bulk_commit();
                 }
+            }
             }
             }
             // this warp's reads of the accumulator are done
@@ -732,7 +796,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(tempty_bar(acc));
-            if (++acc == 2) {
+            if (++acc == NBUF) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
@@ -1301,16 +1365,26 @@ cudaError_t launch_2sm(const Params &p, cudaStream_t s)
     return cudaGetLastError();
 }
 
-template <int EPI, bool GATHER = false>
+template <int EPI, bool GATHER = false, int MT = 1>
 cudaError_t launch(const Params &p, cudaStream_t s)
 {
-    auto kern = grouped_gemm_kernel<EPI, GATHER>;
-    cudaError_t err =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    auto kern = grouped_gemm_kernel<EPI, GATHER, MT>;
+    constexpr int smem = Smem1<MT>::BYTES;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
     return launch_pdl(kern, dim3(sm_count()), dim3(THREADS + (GATHER ? 32 * GATHER_WARPS : 0)),
-                      SMEM_BYTES, s, p);
+                      smem, s, p);
+}
+
+// Single-SM tiles: two 128-row halves per tile (MT = 2, each weight tile
+// read once for up to 256 rows) unless rows are gathered from x.
+template <int EPI>
+cudaError_t launch_1sm(const Params &p, bool two_halves, cudaStream_t s)
+{
+    if (p.gather)
+        return launch<EPI, true, 1>(p, s);
+    return two_halves ? launch<EPI, false, 2>(p, s) : launch<EPI, false, 1>(p, s);
 }
 
 // Diagnostic for the timeout path: one thread waits, with the same bounded
@@ -1352,6 +1426,10 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     // tiles (128 rows) for small segments, where a 256-row tile would mostly
     // compute padding.
     const bool pair = (int64_t)c.T * c.k >= (int64_t)512 * c.E;
+    // single-SM tiles of 256 rows in two halves once experts average more than
+    // 96 rows (many segments then span two 128-row tiles, whose weight tiles
+    // would otherwise be streamed twice)
+    const bool two_halves = !pair && (int64_t)c.T * c.k > (int64_t)96 * c.E;
     // B rows one TMA box brings into one CTA: half the 256-column accumulator
     // for SwiGLU (W1 and W3 halves) and for every SM-pair tile (one half per
     // CTA), the whole 256 otherwise.  The box must match what the kernel
@@ -1388,6 +1466,9 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
         ok &= make_map(&p1.tmB3[0], W3, d, F, E, d * 2, F * d * 2, BK, bn_b, SW128);
     ok &= make_map(&p1.tmC[0], H, F, R, 1, F * 2, 0, CHUNK, 32, SW64);
     const int KB = pair ? KSUB * BK : BK;   // K per stage: the pair kernel takes 128
+    // single-SM tiles serve small segments, whose weight tiles are read by one
+    // or two row tiles: stream them through L2 evict-first
+    p1.b_stream = pair ? 0 : 1;
     p1.set[0] = SetDesc{1, 0, (int)ceil_div(F, bn_out), 1, (int)ceil_div(d, KB), 0, (int)F};
     if (shared) {
         ok &= make_map(&p1.tmA[1], x, d, T, 1, d * 2, 0, BK, BM, SW128);
@@ -1402,12 +1483,13 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     if (!ok)
         return cudaErrorInvalidValue;
     cudaError_t err;
-    if (p1.gather)
-        err = pair ? (swiglu ? launch_2sm<EPI_SWIGLU, true>(p1, s) : launch_2sm<EPI_GELU, true>(p1, s))
-                   : (swiglu ? launch<EPI_SWIGLU, true>(p1, s) : launch<EPI_GELU, true>(p1, s));
+    if (pair)
+        err = p1.gather ? (swiglu ? launch_2sm<EPI_SWIGLU, true>(p1, s)
+                                  : launch_2sm<EPI_GELU, true>(p1, s))
+                        : (swiglu ? launch_2sm<EPI_SWIGLU>(p1, s) : launch_2sm<EPI_GELU>(p1, s));
     else
-        err = pair ? (swiglu ? launch_2sm<EPI_SWIGLU>(p1, s) : launch_2sm<EPI_GELU>(p1, s))
-                   : (swiglu ? launch<EPI_SWIGLU>(p1, s) : launch<EPI_GELU>(p1, s));
+        err = swiglu ? launch_1sm<EPI_SWIGLU>(p1, two_halves, s)
+                     : launch_1sm<EPI_GELU>(p1, two_halves, s);
     if (err != cudaSuccess)
         return err;
 
@@ -1417,6 +1499,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     p2.E = c.E;
     p2.offsets = offsets;
     p2.status = status;
+    p2.b_stream = pair ? 0 : 1;
     p2.timeout_ns = 2000000000ull;
     p2.nsets = shared ? 2 : 1;
     ok = true;
@@ -1445,8 +1528,8 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     if (!ok)
         return cudaErrorInvalidValue;
     if (slot_out)
-        return pair ? launch_2sm<EPI_GATED>(p2, s) : launch<EPI_GATED>(p2, s);
-    return pair ? launch_2sm<EPI_NONE>(p2, s) : launch<EPI_NONE>(p2, s);
+        return pair ? launch_2sm<EPI_GATED>(p2, s) : launch_1sm<EPI_GATED>(p2, two_halves, s);
+    return pair ? launch_2sm<EPI_NONE>(p2, s) : launch_1sm<EPI_NONE>(p2, two_halves, s);
 }
 
 }  // namespace moe
