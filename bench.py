@@ -74,11 +74,13 @@ def kernels_per_step(shape) -> int:
     """Kernels of ours one moe_forward launches: the router (route_kernels),
     capacity 2 (histograms; placement with the totals and the losses),
     dispatch 1, expert FFN (bf16: the two grouped GEMMs; fp32: two, plus two
-    for shared experts), combine 1; the score-ordered capacity adds three
-    launches and a losses launch."""
+    for shared experts), combine 1 (0 for a top-1 layer without shared
+    experts: GEMM2 writes y); the score-ordered capacity adds three launches
+    and a losses launch."""
     ffn = 2 if shape.dtype == 1 else (4 if shape.n_shared else 2)
     extra = 4 if shape.priority == 2 else 0
-    return route_kernels(shape) + 2 + 1 + ffn + 1 + extra
+    combine = 0 if shape.k == 1 and shape.n_shared == 0 else 1   # top-1: in GEMM2's epilogue
+    return route_kernels(shape) + 2 + 1 + ffn + combine + extra
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) of the expert-FFN stage (GEMM1 + GEMM2) per launch, from one ncu

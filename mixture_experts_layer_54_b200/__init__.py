@@ -6,9 +6,10 @@ raises ImportError when the library has not been built.
 """
 from ._abi import (MOE_ROW_ALIGN, CapacityFactorError, MoEError, MoeConfig, MoeOutputs,
                    MoeWeights, LIB_PATH, lib)
-from .ops import (HostStream, MoEForward, moe_bias_update, moe_capacity, moe_capacity_scored,
+from .ops import (CapacityOut, HostStream, MoEForward, moe_bias_update, moe_capacity, moe_capacity_scored,
                   moe_seq_balance_loss, moe_clear_device_status, moe_probe_wait_timeout,
-                  moe_dispatch_rows, moe_expert_ffn_gather, moe_capacity_sharded,
+                  moe_dispatch_rows, moe_expert_ffn_gather, moe_expert_ffn_slots,
+                  moe_combine_slots, moe_capacity_sharded,
                   gather_shard_counts, shard_losses, moe_capacity_noalloc, moe_capacity_value, moe_combine, moe_config,
                   moe_device_status, moe_dispatch, moe_expert_ffn, moe_forward,
                   moe_loss_partials_count, moe_losses, moe_perm_rows, moe_route,
@@ -17,9 +18,10 @@ from .ops import (HostStream, MoEForward, moe_bias_update, moe_capacity, moe_cap
                   workspace)
 
 __all__ = ["MOE_ROW_ALIGN", "CapacityFactorError", "MoEError", "MoeConfig", "MoeOutputs",
-           "MoeWeights", "LIB_PATH", "lib", "HostStream", "MoEForward", "moe_bias_update",
+           "MoeWeights", "LIB_PATH", "lib", "CapacityOut", "HostStream", "MoEForward", "moe_bias_update",
            "moe_capacity_scored", "moe_seq_balance_loss", "moe_clear_device_status",
            "moe_probe_wait_timeout", "moe_dispatch_rows", "moe_expert_ffn_gather",
+           "moe_expert_ffn_slots", "moe_combine_slots",
            "moe_capacity_sharded", "gather_shard_counts", "shard_losses", "moe_capacity", "moe_capacity_noalloc", "moe_capacity_value",
            "moe_combine", "moe_config", "moe_device_status", "moe_dispatch", "moe_expert_ffn",
            "moe_forward", "moe_loss_partials_count", "moe_losses", "moe_perm_rows", "moe_route",

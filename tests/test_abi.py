@@ -154,3 +154,10 @@ def test_binding_refuses_views_and_host_tensors_before_calling_the_library():
     with pytest.raises(ValueError, match="CUDA"):
         ops._p(torch.zeros(4))
     assert ops._p(None) is None
+
+
+def test_package_exports_every_binding():
+    from mixture_experts_layer_54_b200 import ops
+    missing = [n for n in ops.__all__ if not hasattr(moe, n)]
+    assert not missing, missing
+    assert set(ops.__all__) <= set(moe.__all__), set(ops.__all__) - set(moe.__all__)

@@ -101,3 +101,12 @@ def test_layer_summary_rates_and_roofline():
     assert out["stages"]["dispatch"]["GB/s"] == round(w["dispatch"]["bytes"] / 1e-4 / 1e9, 1)
     assert bench.summarize_layer(CONFIGS["mixtral"], 4.3, {**stage_ms, "expert_ffn": 4.0}, 16384,
                                  0, 200, peaks)["layer_roofline"]["bound"] == "tensor"
+
+
+def test_launch_count_follows_the_forward():
+    # router 1 (<= 64 experts, split weights fit) or 3, capacity 2, dispatch 1,
+    # two GEMMs, combine 1 unless top-1 without shared experts
+    assert bench.kernels_per_step(CONFIGS["mixtral"]) == 1 + 2 + 1 + 2 + 1
+    assert bench.kernels_per_step(CONFIGS["switch"]) == 1 + 2 + 1 + 2
+    assert bench.kernels_per_step(CONFIGS["deepseekmoe"]) == 1 + 2 + 1 + 2 + 1
+    assert bench.kernels_per_step(CONFIGS["deepseek_v3"]) == 3 + 2 + 1 + 2 + 1
