@@ -48,25 +48,24 @@ constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
 constexpr int EPI_WARPS = 8;                          // two per TMEM lane quarter
 constexpr int THREADS = 64 + 32 * EPI_WARPS;         // 320
-constexpr int CHUNK = 32;                            // epilogue columns per step
-constexpr int STG_BYTES = 32 * CHUNK * 2;            // 32 rows x 32 bf16 = 2 KB
+// Epilogue: a warp moves CHUNK accumulator columns of its 32 rows per step,
+// through STG_BUFS staging buffers of its own (a buffer is written again only
+// once the TMA store issued from it STG_BUFS steps earlier has read it), as
+// 32 rows of 2 CHUNK bytes in the swizzle of the store map (16-byte chunk c of
+// row r at c ^ ((r >> (3 - SWZ_BITS)) & (2^SWZ_BITS - 1))).
+constexpr int CHUNK = 16;                            // epilogue columns per step
+constexpr int STG_BUFS = 2;
+constexpr int STG_BYTES = 32 * CHUNK * 2;            // one buffer: 32 rows x CHUNK bf16
+constexpr int STG_WARP = STG_BUFS * STG_BYTES;       // a warp's buffers
+constexpr int SWZ_BITS = CHUNK == 16 ? 1 : (CHUNK == 32 ? 2 : 3);   // 32, 64 or 128 B rows
 constexpr uint32_t TMEM_COLS = 512;
 
-// Shared-memory plan of the single-SM kernel for MT row tiles per tile: MT = 1,
-// four stages of A (16 KB) + B (32 KB); MT = 2, three stages of two A boxes
-// (the tile's two 128-row halves, 32 KB) + one B box that both halves share.
-template <int MT>
-struct Smem1 {
-    static constexpr int ST = MT == 1 ? STAGES : 3;
-    static constexpr int A_ST = MT * A_BYTES;
-    static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + ST * A_ST;
-    static constexpr int OFF_STG = OFF_B + ST * B_BYTES;
-    static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BYTES;
-    static constexpr int OFF_TILES = OFF_BAR + 256;
-    static constexpr int BYTES = OFF_TILES + 2 * 4 * (kMaxE + 1) + 1024;   // + alignment slack
-    static_assert(BYTES <= 227 * 1024, "shared memory");
-};
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP;
+constexpr int OFF_TILES = OFF_BAR + 256;
+constexpr int SMEM_BYTES = OFF_TILES + 2 * 4 * (kMaxE + 1) + 1024;   // + alignment slack
 
 // EPI_GATED: GEMM2 with the combine's gate fused (routed rows only): row r
 // of expert e's segment, when kept (r - offsets[e] < kept[e]), holds
@@ -102,7 +101,6 @@ struct __align__(64) Params {
     const int32_t *offsets;
     int32_t *status;
     int clear_status;            // 1: block 0 clears the status word before any wait
-    int b_stream;                // 1: routed B (weights) boxes loaded evict-first in L2
     unsigned long long timeout_ns;
 };
 
@@ -296,8 +294,8 @@ __device__ __forceinline__ int gated_slot(const Params &p, int e, int row, float
     return a;
 }
 
-// EPI_GATED: 32 accumulator columns of one row, times the gate, rounded to
-// bf16, to 64 bytes of the slot's output row.
+// EPI_GATED: CHUNK accumulator columns of one row, times the gate, rounded to
+// bf16, to 2 CHUNK bytes of the slot's output row.
 __device__ __forceinline__ void store_gated(const Params &p, int a, float gate, int col,
                                             const float *v)
 {
@@ -315,26 +313,6 @@ __device__ __forceinline__ void store_gated(const Params &p, int a, float gate, 
     }
 }
 
-// As tma_load_3d, with an L2 cache policy (createpolicy) for the box.
-__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                                 int c0, int c1, int c2, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
-        : "memory");
-}
-
-// L2 policy for data read once: evicted first, so it does not push out data
-// that is read again (the token rows every N tile of an expert re-reads).
-__device__ __forceinline__ uint64_t l2_evict_first()
-{
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
                                              int c2)
 {
@@ -345,7 +323,9 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the TMA stores issued from this thread, all but the last n, have read their source
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -383,6 +363,23 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
                  : "memory");
 }
 
+// 32 lanes x 16 consecutive fp32 columns: thread i gets lane (base + i)
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v)
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
 // 32 lanes x 32 consecutive fp32 columns: thread i gets lane (base + i)
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
 {
@@ -409,20 +406,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
 struct Tile {
     int set;
     int m0;       // first row of A and C
-    int halves;   // 128-row halves of the tile holding rows of its segment (1 or 2)
     int b_group;  // group of the B tensor (K not split)
     int b_row;    // first B row inside the group
     int c_col;    // first C column
     int c_group;  // group of the C tensor
 };
 
-// Tile `tile` of MT x 128 rows: routed tiles expert by expert, N outer and
-// row tiles inner; then the shared set over its dense rows.
-template <int MT>
+// Tile `tile` of 128 rows: routed tiles expert by expert, N outer and row
+// tiles inner; then the shared set over its dense rows.
 __device__ __forceinline__ Tile decode(const Params &p, const int *tstart, const int *mtiles,
                                        int routed_total, int tile, int bn_b, int bn_out)
 {
-    constexpr int TM = MT * BM;
     Tile t;
     if (tile < routed_total) {
         int lo = 0, hi = p.E;   // last e with tstart[e] <= tile
@@ -436,8 +430,7 @@ __device__ __forceinline__ Tile decode(const Params &p, const int *tstart, const
         const int e = lo, i = tile - tstart[e], mt = mtiles[e];
         const int n = i / mt, m = i % mt;
         t.set = 0;
-        t.m0 = p.offsets[e] + m * TM;
-        t.halves = MT == 2 && t.m0 + BM < p.offsets[e + 1] ? 2 : 1;
+        t.m0 = p.offsets[e] + m * BM;
         t.b_group = e;
         t.b_row = n * bn_b;
         t.c_col = n * bn_out;
@@ -445,18 +438,39 @@ __device__ __forceinline__ Tile decode(const Params &p, const int *tstart, const
     } else {
         const SetDesc &s = p.set[1];
         const int i = tile - routed_total;
-        const int mt = (s.rows + TM - 1) / TM;
+        const int mt = (s.rows + BM - 1) / BM;
         const int n = i / mt, m = i % mt;
         const int g = n / s.n_tiles, nn = n % s.n_tiles;
         t.set = 1;
-        t.m0 = m * TM;
-        t.halves = MT == 2 && t.m0 + BM < s.rows ? 2 : 1;
+        t.m0 = m * BM;
         t.b_group = g;
         t.b_row = nn * bn_b;
         t.c_col = nn * bn_out;
         t.c_group = g;
     }
     return t;
+}
+
+// CHUNK columns of this thread's accumulator row
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, float *v)
+{
+    if (CHUNK == 16)
+        tmem_ld16(taddr, v);
+    else
+        tmem_ld32(taddr, v);
+}
+
+// Stage this thread's row of packed bf16 (2 CHUNK bytes) into a staging buffer
+// in the store map's swizzle.
+__device__ __forceinline__ void stage_row(uint8_t *buf, int lane, const uint32_t *packed)
+{
+    uint8_t *row = buf + lane * (CHUNK * 2);
+#pragma unroll
+    for (int ch = 0; ch < CHUNK / 8; ++ch) {
+        const int phys = ch ^ ((lane >> (3 - SWZ_BITS)) & ((1 << SWZ_BITS) - 1));
+        *reinterpret_cast<uint4 *>(row + phys * 16) =
+            make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
+    }
 }
 
 template <int EPI>
@@ -480,29 +494,19 @@ __device__ __forceinline__ void epilogue_chunk(const float *g, const float *u, u
     }
 }
 
-// MT = 2: a tile covers up to 256 rows of one segment as two 128-row halves
-// with their own accumulators (TMEM columns 0 and 256) and one shared B box
-// per K step, so a weight tile is read once for up to 256 rows; a half past
-// the segment's end is neither loaded nor computed.  The two accumulators take
-// all of TMEM, so MT = 2 tiles are not double buffered.
-template <int EPI, bool GATHER, int MT>
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     grouped_gemm_kernel(const __grid_constant__ Params p)
 {
-    static_assert(MT == 1 || (MT == 2 && !GATHER), "row tiles per tile");
-    using L = Smem1<MT>;
-    constexpr int STAGES = L::ST;                              // (shadows the 4-stage default)
-    constexpr int A_ST = L::A_ST;
-    constexpr int NBUF = MT == 1 ? 2 : 1;                      // accumulator sets in TMEM
     constexpr int BN_B = EPI == EPI_SWIGLU ? BN / 2 : BN;     // B rows per tensor per tile
     constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;   // output columns per tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    const uint32_t sA = smem_u32(smem + L::OFF_A);
-    const uint32_t sB = smem_u32(smem + L::OFF_B);
-    const uint32_t sStg = smem_u32(smem + L::OFF_STG);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
+    const uint32_t sA = smem_u32(smem + OFF_A);
+    const uint32_t sB = smem_u32(smem + OFF_B);
+    const uint32_t sStg = smem_u32(smem + OFF_STG);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     // full[0..S), empty[S..2S), tfull[2S, 2S+2), tempty[2S+2, 2S+4), drain 2S+4
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -510,10 +514,10 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_BAR + 8 * (2 * STAGES + 5));
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8 * (2 * STAGES + 5));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *tstart = reinterpret_cast<int *>(smem + L::OFF_TILES);   // [E + 1]
-    int *mtiles = tstart + (kMaxE + 1);                          // [E]
+    int *tstart = reinterpret_cast<int *>(smem + OFF_TILES);    // [E + 1]
+    int *mtiles = tstart + (kMaxE + 1);                         // [E]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Ctl ctl{abort_flag, p.status, p.timeout_ns};
@@ -548,7 +552,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     int routed_total = 0;
     if (p.set[0].routed && p.nsets > 0) {
         for (int e = threadIdx.x; e < p.E; e += blockDim.x)
-            mtiles[e] = ((p.offsets[e + 1] - p.offsets[e]) / BM + MT - 1) / MT;
+            mtiles[e] = (p.offsets[e + 1] - p.offsets[e]) / BM;
         __syncthreads();
         if (threadIdx.x == 0) {
             int acc = 0;
@@ -567,7 +571,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
     int shared_total = 0;
     if (p.nsets > 1) {
         const SetDesc &s = p.set[1];
-        shared_total = (s.rows + MT * BM - 1) / (MT * BM) * s.n_tiles * s.n_groups;
+        shared_total = (s.rows + BM - 1) / BM * s.n_tiles * s.n_groups;
     }
     const int total = routed_total + shared_total;
     const uint32_t tmem_base = *tmem_slot;
@@ -577,7 +581,6 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
         // Lane 0 owns the barrier waits and the box copies (with gathered A
         // rows, the B boxes only: the gather warps copy A).
         if (lane == 0) {
-            const uint64_t b_policy = l2_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             int issued[STAGES];
@@ -586,7 +589,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                 issued[s] = 0, last_phase[s] = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+                const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
                 const SetDesc &sd = p.set[t.set];
                 const bool gath = GATHER && t.set == 0;
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
@@ -600,19 +603,11 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                         kcol = (kb % sd.kbg) * BK;
                     }
                     const uint32_t fb = full_bar(stage);
-                    mbar_expect_tx(fb, (gath ? 0 : t.halves * A_BYTES) + B_BYTES);
+                    mbar_expect_tx(fb, (gath ? 0 : A_BYTES) + B_BYTES);
                     if (!gath)
-                        for (int h = 0; h < t.halves; ++h)
-                            tma_load_3d(sA + stage * A_ST + h * A_BYTES, &p.tmA[t.set], fb, kcol,
-                                        t.m0 + h * BM, ga);
+                        tma_load_3d(sA + stage * A_BYTES, &p.tmA[t.set], fb, kcol, t.m0, ga);
                     const uint32_t b0 = sB + stage * B_BYTES;
-                    const bool stream = p.b_stream && t.set == 0;
-                    if (stream) {
-                        tma_load_3d_hint(b0, &p.tmB[t.set], fb, kcol, t.b_row, gb, b_policy);
-                        if (EPI == EPI_SWIGLU)
-                            tma_load_3d_hint(b0 + B_BYTES / 2, &p.tmB3[t.set], fb, kcol, t.b_row,
-                                             gb, b_policy);
-                    } else if (EPI == EPI_SWIGLU) {
+                    if (EPI == EPI_SWIGLU) {
                         tma_load_3d(b0, &p.tmB[t.set], fb, kcol, t.b_row, gb);
                         tma_load_3d(b0 + B_BYTES / 2, &p.tmB3[t.set], fb, kcol, t.b_row, gb);
                     } else {
@@ -640,15 +635,13 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
             uint32_t acc_phase = 0;
             bool ok = true, any = false;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+                const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
                 const SetDesc &sd = p.set[t.set];
                 if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, ctl)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                // MT = 1: accumulator set acc at columns acc * 256; MT = 2: the
-                // halves at columns 0 and 256
                 const uint32_t tmem_d = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < sd.k_blocks; ++kb) {
                     if (!wait_bar(full_bar(stage), phase, ctl)) {
@@ -656,14 +649,11 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t b_base = sB + stage * B_BYTES;
-                    for (int h = 0; h < t.halves; ++h) {
-                        const uint32_t a_base = sA + stage * A_ST + h * A_BYTES;
+                    const uint32_t a_base = sA + stage * A_BYTES, b_base = sB + stage * B_BYTES;
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_bf16(tmem_d + (uint32_t)(h * BN), sdesc_sw128(a_base + kk * 32),
-                                     sdesc_sw128(b_base + kk * 32), (kb | kk) != 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16(tmem_d, sdesc_sw128(a_base + kk * 32), sdesc_sw128(b_base + kk * 32),
+                                 (kb | kk) != 0 ? 1u : 0u);
                     mma_commit(empty_bar(stage));
                     any = true;
                     if (++stage == STAGES) {
@@ -674,7 +664,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                 if (!ok)
                     break;
                 mma_commit(tfull_bar(acc));
-                if (++acc == NBUF) {
+                if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
@@ -697,7 +687,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
         uint32_t phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+            const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
             const SetDesc &sd = p.set[t.set];
             const bool gath = t.set == 0;   // shared-expert tiles: TMA boxes of x
             int tok[G::NI];
@@ -711,7 +701,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
                     break;
                 }
                 if (gath)
-                    gather_stage<1>(sA + stage * A_ST, 0, p.xg, p.x_ld, kb * BK, tok, gw, lane);
+                    gather_stage<1>(sA + stage * A_BYTES, 0, p.xg, p.x_ld, kb * BK, tok, gw, lane);
                 cp_async_commit();
                 if (seq >= D) {
                     cp_async_wait<D>();
@@ -732,20 +722,18 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
         const int q = warp & 3;                      // TMEM lane quarter
         const int ew = warp - 2;                     // staging buffer owner
         const int half = ew >> 2;                    // which half of the columns
-        const uint32_t stg = sStg + ew * STG_BYTES;
-        uint8_t *stg_ptr = smem + L::OFF_STG + ew * STG_BYTES;
-        int acc = 0;
+        const uint32_t stg = sStg + ew * STG_WARP;
+        uint8_t *stg_ptr = smem + OFF_STG + ew * STG_WARP;
+        int acc = 0, nchunk = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode<MT>(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
+            const Tile t = decode(p, tstart, mtiles, routed_total, tile, BN_B, BN_OUT);
             if (!wait_bar(tfull_bar(acc), acc_phase, ctl))
                 break;
             tc_fence_after();
             const int c_end = min((half + 1) * (BN_OUT / 2), p.set[t.set].c_cols - t.c_col);
-            for (int h = 0; h < t.halves; ++h) {
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) +
-                                   (uint32_t)((acc + h) * BN);
-            const int row0 = t.m0 + h * BM + q * 32;   // this warp's 32 rows
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            const int row0 = t.m0 + q * 32;   // this warp's 32 rows
             if (EPI == EPI_GATED && t.set == 0) {
                 // gate and scatter: this lane's row goes to its assignment's row
                 float gate;
@@ -753,42 +741,34 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
 #pragma unroll 1
                 for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
                     float g[CHUNK];
-                    tmem_ld32(tbase + c, g);
+                    tmem_ld_chunk(tbase + c, g);
                     if (a >= 0)
                         store_gated(p, a, gate, t.c_col + c, g);
                 }
             } else {
 #pragma unroll 1
-            for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
+            for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK, ++nchunk) {
                 float g[CHUNK], u[CHUNK];
                 uint32_t packed[CHUNK / 2];
-                tmem_ld32(tbase + c, g);
+                tmem_ld_chunk(tbase + c, g);
                 if (EPI == EPI_SWIGLU) {
-                    tmem_ld32(tbase + BN / 2 + c, u);
+                    tmem_ld_chunk(tbase + BN / 2 + c, u);
                     epilogue_chunk<EPI>(g, u, packed);
                 } else {
                     epilogue_chunk<EPI>(g, g, packed);
                 }
-                // staging tile: 32 rows x 64 bytes, 64-byte swizzle (16-byte
-                // chunk index XOR bits 1-2 of the row), as the store map expects
+                const int b = nchunk % STG_BUFS;   // this chunk's staging buffer
                 if (lane == 0)
-                    bulk_wait_read0();
+                    bulk_wait_read<STG_BUFS - 1>();
                 __syncwarp();
-                uint8_t *row = stg_ptr + lane * 64;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int phys = ch ^ ((lane >> 1) & 3);
-                    *reinterpret_cast<uint4 *>(row + phys * 16) =
-                        make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2],
-                                   packed[4 * ch + 3]);
-                }
+                stage_row(stg_ptr + b * STG_BYTES, lane, packed);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&p.tmC[t.set], stg, t.c_col + c, row0, t.c_group);
+                    tma_store_3d(&p.tmC[t.set], stg + b * STG_BYTES, t.c_col + c, row0,
+                                 t.c_group);
                     bulk_commit();
                 }
-            }
             }
             }
             // this warp's reads of the accumulator are done
@@ -796,7 +776,7 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(tempty_bar(acc));
-            if (++acc == NBUF) {
+            if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
@@ -840,7 +820,7 @@ constexpr int HALF_BYTES = 128 * BK * 2;             // 16 KB: 128 rows x 64 bf1
 constexpr int OFF2_A = 0;
 constexpr int OFF2_B = OFF2_A + STAGES2 * KSUB * HALF_BYTES;
 constexpr int OFF2_STG = OFF2_B + STAGES2 * KSUB * HALF_BYTES;
-constexpr int OFF2_BAR = OFF2_STG + EPI_WARPS * STG_BYTES;
+constexpr int OFF2_BAR = OFF2_STG + EPI_WARPS * STG_WARP;
 constexpr int OFF2_TILES = OFF2_BAR + 256;
 constexpr int SMEM2_BYTES = OFF2_TILES + 2 * 4 * (kMaxE + 1) + 1024;
 
@@ -1200,9 +1180,9 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
         const int q = warp & 3;
         const int ew = warp - 2;
         const int half = ew >> 2;
-        const uint32_t stg = sStg + ew * STG_BYTES;
-        uint8_t *stg_ptr = smem + OFF2_STG + ew * STG_BYTES;
-        int acc = 0;
+        const uint32_t stg = sStg + ew * STG_WARP;
+        uint8_t *stg_ptr = smem + OFF2_STG + ew * STG_WARP;
+        int acc = 0, nchunk = 0;
         uint32_t acc_phase = 0;
         for (int tile = cluster_id; tile < total; tile += nclusters) {
             const Tile2 t = decode2(p, tstart, mpairs, routed_total, tile);
@@ -1222,37 +1202,31 @@ __global__ void __launch_bounds__(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1)
 #pragma unroll 1
                 for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
                     float g[CHUNK];
-                    tmem_ld32(tbase + c, g);
+                    tmem_ld_chunk(tbase + c, g);
                     if (a >= 0)
                         store_gated(p, a, gate, c_col + c, g);
                 }
             } else {
 #pragma unroll 1
-            for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK) {
+            for (int c = half * (BN_OUT / 2); c < c_end; c += CHUNK, ++nchunk) {
                 float g[CHUNK], u[CHUNK];
                 uint32_t packed[CHUNK / 2];
-                tmem_ld32(tbase + c, g);
+                tmem_ld_chunk(tbase + c, g);
                 if (EPI == EPI_SWIGLU) {
-                    tmem_ld32(tbase + BN / 2 + c, u);
+                    tmem_ld_chunk(tbase + BN / 2 + c, u);
                     epilogue_chunk<EPI>(g, u, packed);
                 } else {
                     epilogue_chunk<EPI>(g, g, packed);
                 }
+                const int b = nchunk % STG_BUFS;   // this chunk's staging buffer
                 if (lane == 0)
-                    bulk_wait_read0();
+                    bulk_wait_read<STG_BUFS - 1>();
                 __syncwarp();
-                uint8_t *rowp = stg_ptr + lane * 64;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int phys = ch ^ ((lane >> 1) & 3);
-                    *reinterpret_cast<uint4 *>(rowp + phys * 16) =
-                        make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2],
-                                   packed[4 * ch + 3]);
-                }
+                stage_row(stg_ptr + b * STG_BYTES, lane, packed);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&p.tmC[t.set], stg, c_col + c, row, t.c_group);
+                    tma_store_3d(&p.tmC[t.set], stg + b * STG_BYTES, c_col + c, row, t.c_group);
                     bulk_commit();
                 }
             }
@@ -1365,26 +1339,22 @@ cudaError_t launch_2sm(const Params &p, cudaStream_t s)
     return cudaGetLastError();
 }
 
-template <int EPI, bool GATHER = false, int MT = 1>
+template <int EPI, bool GATHER = false>
 cudaError_t launch(const Params &p, cudaStream_t s)
 {
-    auto kern = grouped_gemm_kernel<EPI, GATHER, MT>;
-    constexpr int smem = Smem1<MT>::BYTES;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kern = grouped_gemm_kernel<EPI, GATHER>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess)
         return err;
     return launch_pdl(kern, dim3(sm_count()), dim3(THREADS + (GATHER ? 32 * GATHER_WARPS : 0)),
-                      smem, s, p);
+                      SMEM_BYTES, s, p);
 }
 
-// Single-SM tiles: two 128-row halves per tile (MT = 2, each weight tile
-// read once for up to 256 rows) unless rows are gathered from x.
 template <int EPI>
-cudaError_t launch_1sm(const Params &p, bool two_halves, cudaStream_t s)
+cudaError_t launch_1sm(const Params &p, cudaStream_t s)
 {
-    if (p.gather)
-        return launch<EPI, true, 1>(p, s);
-    return two_halves ? launch<EPI, false, 2>(p, s) : launch<EPI, false, 1>(p, s);
+    return p.gather ? launch<EPI, true>(p, s) : launch<EPI, false>(p, s);
 }
 
 // Diagnostic for the timeout path: one thread waits, with the same bounded
@@ -1426,10 +1396,6 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     // tiles (128 rows) for small segments, where a 256-row tile would mostly
     // compute padding.
     const bool pair = (int64_t)c.T * c.k >= (int64_t)512 * c.E;
-    // single-SM tiles of 256 rows in two halves once experts average more than
-    // 96 rows (many segments then span two 128-row tiles, whose weight tiles
-    // would otherwise be streamed twice)
-    const bool two_halves = !pair && (int64_t)c.T * c.k > (int64_t)96 * c.E;
     // B rows one TMA box brings into one CTA: half the 256-column accumulator
     // for SwiGLU (W1 and W3 halves) and for every SM-pair tile (one half per
     // CTA), the whole 256 otherwise.  The box must match what the kernel
@@ -1437,7 +1403,11 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     const int bn_b = (swiglu || pair) ? BN / 2 : BN;
     const int bn2_b = pair ? BN / 2 : BN;
     const int bn_out = swiglu ? BN / 2 : BN;
-    const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B, SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
+    // epilogue store boxes: CHUNK columns x 32 rows, swizzled as stage_row writes them
+    const CUtensorMapSwizzle SWC = SWZ_BITS == 1 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                  : (SWZ_BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                   : CU_TENSOR_MAP_SWIZZLE_128B);
     const bool shared = S > 0 && T > 0;
 
     // ---- GEMM1: H = act(x_perm W1^T [, x_perm W3^T]); H_sh likewise from x ----
@@ -1464,11 +1434,9 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     ok &= make_map(&p1.tmB[0], W1, d, F, E, d * 2, F * d * 2, BK, bn_b, SW128);
     if (swiglu)
         ok &= make_map(&p1.tmB3[0], W3, d, F, E, d * 2, F * d * 2, BK, bn_b, SW128);
-    ok &= make_map(&p1.tmC[0], H, F, R, 1, F * 2, 0, CHUNK, 32, SW64);
+    ok &= make_map(&p1.tmC[0], H, F, R, 1, F * 2, 0, CHUNK, 32, SWC);
     const int KB = pair ? KSUB * BK : BK;   // K per stage: the pair kernel takes 128
-    // single-SM tiles serve small segments, whose weight tiles are read by one
-    // or two row tiles: stream them through L2 evict-first
-    p1.b_stream = pair ? 0 : 1;
+
     p1.set[0] = SetDesc{1, 0, (int)ceil_div(F, bn_out), 1, (int)ceil_div(d, KB), 0, (int)F};
     if (shared) {
         ok &= make_map(&p1.tmA[1], x, d, T, 1, d * 2, 0, BK, BM, SW128);
@@ -1476,7 +1444,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
         if (swiglu)
             ok &= make_map(&p1.tmB3[1], Ws3, d, Fs, S, d * 2, Fs * d * 2, BK, bn_b, SW128);
         // H_sh [S][T][Fs]: shared expert s owns one [T][Fs] slab
-        ok &= make_map(&p1.tmC[1], H_sh, Fs, T, S, Fs * 2, T * Fs * 2, CHUNK, 32, SW64);
+        ok &= make_map(&p1.tmC[1], H_sh, Fs, T, S, Fs * 2, T * Fs * 2, CHUNK, 32, SWC);
         p1.set[1] = SetDesc{0, (int)T, (int)ceil_div(Fs, bn_out), (int)S, (int)ceil_div(d, KB), 0,
                             (int)Fs};
     }
@@ -1488,8 +1456,8 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
                                   : launch_2sm<EPI_GELU, true>(p1, s))
                         : (swiglu ? launch_2sm<EPI_SWIGLU>(p1, s) : launch_2sm<EPI_GELU>(p1, s));
     else
-        err = swiglu ? launch_1sm<EPI_SWIGLU>(p1, two_halves, s)
-                     : launch_1sm<EPI_GELU>(p1, two_halves, s);
+        err = swiglu ? launch_1sm<EPI_SWIGLU>(p1, s)
+                     : launch_1sm<EPI_GELU>(p1, s);
     if (err != cudaSuccess)
         return err;
 
@@ -1499,7 +1467,6 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
     p2.E = c.E;
     p2.offsets = offsets;
     p2.status = status;
-    p2.b_stream = pair ? 0 : 1;
     p2.timeout_ns = 2000000000ull;
     p2.nsets = shared ? 2 : 1;
     ok = true;
@@ -1515,21 +1482,21 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, const void *x_perm, const in
         p2.slot_out = static_cast<__nv_bfloat16 *>(slot_out);
         p2.slot_ld = (int)d;
     } else {
-        ok &= make_map(&p2.tmC[0], Y_perm, d, R, 1, d * 2, 0, CHUNK, 32, SW64);
+        ok &= make_map(&p2.tmC[0], Y_perm, d, R, 1, d * 2, 0, CHUNK, 32, SWC);
     }
     p2.set[0] = SetDesc{1, 0, (int)ceil_div(d, BN), 1, (int)ceil_div(F, KB), 0, (int)d};
     if (shared) {
         ok &= make_map(&p2.tmA[1], H_sh, Fs, T, S, Fs * 2, T * Fs * 2, BK, BM, SW128);
         ok &= make_map(&p2.tmB[1], Ws2, Fs, d, S, Fs * 2, d * Fs * 2, BK, bn2_b, SW128);
-        ok &= make_map(&p2.tmC[1], Y_sh, d, T, 1, d * 2, 0, CHUNK, 32, SW64);
+        ok &= make_map(&p2.tmC[1], Y_sh, d, T, 1, d * 2, 0, CHUNK, 32, SWC);
         const int kbg = (int)ceil_div(Fs, KB);
         p2.set[1] = SetDesc{0, (int)T, (int)ceil_div(d, BN), 1, kbg * (int)S, kbg, (int)d};
     }
     if (!ok)
         return cudaErrorInvalidValue;
     if (slot_out)
-        return pair ? launch_2sm<EPI_GATED>(p2, s) : launch_1sm<EPI_GATED>(p2, two_halves, s);
-    return pair ? launch_2sm<EPI_NONE>(p2, s) : launch_1sm<EPI_NONE>(p2, two_halves, s);
+        return pair ? launch_2sm<EPI_GATED>(p2, s) : launch_1sm<EPI_GATED>(p2, s);
+    return pair ? launch_2sm<EPI_NONE>(p2, s) : launch_1sm<EPI_NONE>(p2, s);
 }
 
 }  // namespace moe

@@ -268,28 +268,42 @@ __device__ __forceinline__ void select_token(const RouteParams &a, bool renorm, 
 // parts (P = cluster size, 1, 2 or 4); block `rank` owns K blocks
 // [rank kbp, (rank + 1) kbp).  The cluster walks token tiles of 128
 // (tile = cluster, cluster + clusters, ...), so one cluster may take several.
-//   prologue     the selection warps split this block's K part of W_r into the
-//                three bf16 terms, K-major in the 128-byte swizzle, once: the
-//                B operand of every tile stays in shared memory;
-//   warp 0       TMA ring of x tiles (one thread);
+//   prologue     warps 2-13 split this block's K part of W_r into the three
+//                bf16 terms, K-major in the 128-byte swizzle, once (all of a
+//                thread's loads issued before any conversion): the B operand
+//                of every tile stays in shared memory;
+//   warp 0       TMA ring of x tiles (one thread), as deep as shared memory
+//                allows;
 //   warp 1       one MMA of N = 3 NE per K step of 16 into one of two TMEM
 //                accumulators (tile i uses buffer i mod 2);
-//   warps 2-5    read an accumulator back (hi + (mid + lo)) into the block's
-//                partial-logit buffer i mod 2, then tell every block of the
-//                cluster (a remote mbarrier arrive, release at cluster scope);
-//   warps 6-13   select 128 / P tokens of the tile, summing the P partial
-//                logits of each (expert, token) in part order through
-//                distributed shared memory; then tell every block that its
-//                buffer may be reused.
-// So one tile's read-back and selection run while the next tile's x streams.
+//   warps 2-5    read an accumulator back (hi + (mid + lo)) and push each
+//                token's partial logits into buffer i mod 2 of the block that
+//                selects that token (st.shared::cluster, slot = this block's
+//                K part), then tell every block of the cluster (a remote
+//                mbarrier arrive, release at cluster scope);
+//   warps 6-13   select 128 / P tokens of the tile from their own buffer,
+//                summing the P parts in part order; then tell every block
+//                that the buffer may be filled again.
+// So one tile's read-back and selection run while the next tile's x streams,
+// and no warp waits on a remote load.
 
 constexpr int PR_THREADS = 448;   // 14 warps
 constexpr int RB_WARP0 = 2;       // warps 2-5: TMEM read-back
-constexpr int SEL_WARP0 = 6;      // warps 6-13: W split, then selection
+constexpr int SEL_WARP0 = 6;      // warps 6-13: selection
 constexpr int SEL_WARPS = 8;
 constexpr int SEL_THREADS = SEL_WARPS * 32;
-constexpr int MAX_STAGES = 4;
+constexpr int CONV_WARP0 = 2;     // warps 2-13 split W_r first
+constexpr int CONV_THREADS = PR_THREADS - CONV_WARP0 * 32;
+constexpr int MAX_STAGES = 8;
 constexpr int W_MAX_BYTES = 112 * 1024;   // resident split weights per block
+
+// Store four floats to shared memory of another block of the cluster.
+__device__ __forceinline__ void st_peer4(uint32_t a, float4 v)
+{
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
 
 // Named barriers (id 0 is __syncthreads).
 __device__ __forceinline__ void named_sync(int id, int threads)
@@ -395,13 +409,14 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
     uint8_t *Wres = smem + sm.w;
     uint8_t *X = smem + sm.x;
     const uint32_t lbase = saddr(smem + sm.l);
+    const int TPC = BM / P;   // tokens of a tile this block selects (128, 64 or 32)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             bar_init(saddr(&full[s]), 1);
             bar_init(saddr(&empty[s]), 1);
         }
-        bar_init(saddr(&wready), SEL_WARPS);
+        bar_init(saddr(&wready), CONV_THREADS / 32);
         for (int a = 0; a < 2; ++a) {
             bar_init(saddr(&tfull[a]), 1);
             bar_init(saddr(&tempty[a]), 4);
@@ -431,6 +446,67 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
     pdl_trigger();
     if (p.clear_status && blockIdx.x == 0 && threadIdx.x == 0)
         *p.status = 0;
+
+    if (warp >= CONV_WARP0) {
+        // ---- prologue: this block's K part of W_r -> three bf16 terms ----
+        // Chunk c = (K block i, 8-wide K group j, expert e), e fastest so that
+        // neighbouring threads read neighbouring W_r words; its 16 bytes of
+        // each term go to row e (+ NE, + 2 NE) of K block i's tile, at
+        // position j ^ (row & 7) of the row's eight (128-byte swizzle).  A
+        // thread issues the loads of CB chunks before converting any.
+        constexpr int CB = 4;
+        const int ct = threadIdx.x - CONV_WARP0 * 32;
+        const int E = p.E, nchunk = kbp * 8 * NE;
+        for (int c0 = ct; c0 < nchunk; c0 += CB * CONV_THREADS) {
+            float w[CB][8];
+#pragma unroll
+            for (int b = 0; b < CB; ++b) {
+                const int c = c0 + b * CONV_THREADS;
+                const int e = c % NE, j = (c / NE) % 8, i = c / (NE * 8);
+                const bool live = c < nchunk && e < E;
+                const int64_t k0 = (int64_t)(kb0 + i) * BK + 8 * j;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    w[b][u] = live ? p.W_r[(k0 + u) * E + e] : 0.f;
+            }
+#pragma unroll
+            for (int b = 0; b < CB; ++b) {
+                const int c = c0 + b * CONV_THREADS;
+                if (c >= nchunk)
+                    break;
+                const int e = c % NE, j = (c / NE) % 8, i = c / (NE * 8);
+                uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+                for (int u = 0; u < 8; u += 2) {
+                    __nv_bfloat16 h[2], md[2], l[2];
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const float x = w[b][u + r];
+                        h[r] = __float2bfloat16_rn(x);
+                        const float r1 = x - __bfloat162float(h[r]);
+                        md[r] = __float2bfloat16_rn(r1);
+                        l[r] = __float2bfloat16_rn(r1 - __bfloat162float(md[r]));
+                    }
+                    hi[u / 2] = pack2(h[0], h[1]);
+                    mid[u / 2] = pack2(md[0], md[1]);
+                    lo[u / 2] = pack2(l[0], l[1]);
+                }
+                uint8_t *tile = Wres + i * WT_BYTES;
+                const uint32_t *terms[3] = {hi, mid, lo};
+#pragma unroll
+                for (int sp = 0; sp < 3; ++sp) {
+                    const int row = sp * NE + e;
+                    *reinterpret_cast<uint4 *>(tile + row * 128 + ((j ^ (row & 7)) << 4)) =
+                        make_uint4(terms[sp][0], terms[sp][1], terms[sp][2], terms[sp][3]);
+                }
+            }
+        }
+        // generic-proxy stores, read next by the tensor core (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0)
+            bar_arrive(saddr(&wready));
+    }
 
     if (warp == 0) {
         if (lane == 0) {
@@ -540,7 +616,10 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             if (rb_fail)
                 break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            float *L = reinterpret_cast<float *>(smem + sm.l + a * L_BYTES) + (q * 32 + lane) * LS;
+            // this lane's token row goes to the block selecting it, slot `rank`
+            const int row = q * 32 + lane, owner = row / TPC, tl = row % TPC;
+            const uint32_t dst = peer_addr(lbase, (uint32_t)owner) +
+                                 (uint32_t)(a * L_BYTES + (rank * TPC + tl) * LS * 4);
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)a * ACC;
 #pragma unroll
             for (int c = 0; c < NE; c += 16) {
@@ -564,7 +643,7 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                     for (int u = 0; u < 4; ++u)   // x W_hi + (x W_mid + x W_lo)
                         v[u] = __uint_as_float(r[0][h + u]) +
                                (__uint_as_float(r[1][h + u]) + __uint_as_float(r[2][h + u]));
-                    *reinterpret_cast<float4 *>(L + c + h) = make_float4(v[0], v[1], v[2], v[3]);
+                    st_peer4(dst + (uint32_t)((c + h) * 4), make_float4(v[0], v[1], v[2], v[3]));
                 }
             }
             // accumulator free for the tile after next
@@ -572,68 +651,21 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             __syncwarp();
             if (lane == 0)
                 bar_arrive(saddr(&tempty[a]));
-            // the four read-back warps' rows are written: tell every block
+            // the four read-back warps' rows are pushed: tell every block
             named_sync(1, 128);
             if (warp == RB_WARP0 && lane == 0)
                 for (int r = 0; r < P; ++r)
                     arrive_remote(saddr(&lfull[a]), (uint32_t)r);
         }
     } else {
-        // ---- prologue: this block's K part of W_r -> three bf16 terms ----
-        // Chunk c = (K block i, 8-wide K group j, expert e), e fastest so that
-        // neighbouring threads read neighbouring W_r words; its 16 bytes of
-        // each term go to row e (+ NE, + 2 NE) of K block i's tile, at
-        // position j ^ (row & 7) of the row's eight (128-byte swizzle).
+        // ---- selection: this block's share of every tile's tokens ----
+        // buffer a holds [part q][token tl of the share][expert]
         const int st = threadIdx.x - SEL_WARP0 * 32;
         const int E = p.E;
-        for (int c = st; c < kbp * 8 * NE; c += SEL_THREADS) {
-            const int e = c % NE, j = (c / NE) % 8, i = c / (NE * 8);
-            float w[8];
-            const int64_t k0 = (int64_t)(kb0 + i) * BK + 8 * j;
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                w[u] = e < E ? p.W_r[(k0 + u) * E + e] : 0.f;
-            uint32_t hi[4], mid[4], lo[4];
-#pragma unroll
-            for (int u = 0; u < 8; u += 2) {
-                __nv_bfloat16 h[2], md[2], l[2];
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const float x = w[u + r];
-                    h[r] = __float2bfloat16_rn(x);
-                    const float r1 = x - __bfloat162float(h[r]);
-                    md[r] = __float2bfloat16_rn(r1);
-                    l[r] = __float2bfloat16_rn(r1 - __bfloat162float(md[r]));
-                }
-                hi[u / 2] = pack2(h[0], h[1]);
-                mid[u / 2] = pack2(md[0], md[1]);
-                lo[u / 2] = pack2(l[0], l[1]);
-            }
-            uint8_t *tile = Wres + i * WT_BYTES;
-            const uint32_t *terms[3] = {hi, mid, lo};
-#pragma unroll
-            for (int sp = 0; sp < 3; ++sp) {
-                const int row = sp * NE + e;
-                *reinterpret_cast<uint4 *>(tile + row * 128 + ((j ^ (row & 7)) << 4)) =
-                    make_uint4(terms[sp][0], terms[sp][1], terms[sp][2], terms[sp][3]);
-            }
-        }
-        // generic-proxy stores, read next by the tensor core (async proxy)
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0)
-            bar_arrive(saddr(&wready));
-
-        // ---- selection: this block's share of every tile's tokens ----
         const int sw = warp - SEL_WARP0;   // selection warp 0..7
-        const int TPC = BM / P;            // 128, 64 or 32 tokens
         const int tl0 = rank * TPC;
         const bool renorm = p.renorm < 0 ? (p.k > 1) : (p.renorm != 0);
         float *scratch = reinterpret_cast<float *>(smem + sm.scratch);
-        uint32_t rb[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            rb[q] = q < P ? peer_addr(lbase, (uint32_t)q) : 0u;
         float lb[PL], sb[PL];   // per-expert biases of this lane, loaded once
 #pragma unroll
         for (int i = 0; i < PL; ++i) {
@@ -655,7 +687,7 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             const int m0 = tile * BM;
             const int row0 = (m0 + tl0) / kPartialTokens;
             const int rows = TPC / kPartialTokens;
-            const uint32_t aoff = (uint32_t)(a * L_BYTES);
+            const float *Lb = reinterpret_cast<const float *>(smem + sm.l + a * L_BYTES);
             if constexpr (E_T > 0) {
                 // a group = the 32 / E_T tokens one warp holds at once; E_T
                 // groups make a row of the loss partials
@@ -672,7 +704,7 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                     if (m0 + tl < p.T && gl < E) {
                         z = 0.f;
                         for (int q = 0; q < P; ++q)
-                            z += ld_peer(rb[q] + aoff + (uint32_t)(tl * LS + gl) * 4u);
+                            z += Lb[(q * TPC + tl - tl0) * LS + gl];
                     }
                     float pc, zc;
                     small_epilogue<E_T>(ra, z, m0 + tg, lane, renorm, &pc, &zc);
@@ -715,7 +747,7 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                             if (e < E) {
                                 float s = 0.f;
                                 for (int q = 0; q < P; ++q)
-                                    s += ld_peer(rb[q] + aoff + (uint32_t)(tl * LS + e) * 4u);
+                                    s += Lb[(q * TPC + tl - tl0) * LS + e];
                                 if (p.logit_bias)
                                     s += lb[i];
                                 z[i] = s;
