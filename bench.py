@@ -45,27 +45,28 @@ from moe_inputs import CONFIGS, generate, seed_for  # noqa: E402
 
 METRIC = "MoE layer fwd tokens/s on 1 B200; grouped-GEMM % BF16 peak; dispatch % HBM BW"
 UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20   # written between cold stage timings: twice the 126 MB L2
 def route_kernels(shape) -> int:
     """Kernels of the router: bf16 layers with up to 64 experts whose split
-    router weights of a K part (3 x E padded x 64 x 2 bytes per K block) fit
-    in shared memory run one kernel, wider ones three (split, logits,
-    select); the fp32 layer one."""
+    router weights of a K part (3 x E padded rows, rounded up to a multiple of
+    16, x 64 x 2 bytes per K block; E padded to 8 up to 8 experts, else to a
+    multiple of 16) fit in shared memory run one kernel, wider ones three
+    (split, logits, select); the fp32 layer one."""
     if shape.dtype != 1:
         return 1
     if shape.E <= 64:
-        ne = 16 if shape.E <= 16 else (shape.E + 15) // 16 * 16
+        ne = 8 if shape.E <= 8 else (shape.E + 15) // 16 * 16
+        n3 = (3 * ne + 15) // 16 * 16
         kb = shape.d // 64
         p = 4
         while p > 1 and (kb % p or kb // p < 4):
             p //= 2
         kbp = kb // p
-        for stages in (4, 3, 2):
-            x = (kbp * 3 * ne * 128 + 1023) // 1024 * 1024
-            total = x + stages * 16384 + 2 * 128 * (ne + 4) * 4 + \
-                max(8 * (ne + 1), 32 * 9) * 4 + 1024
-            if total <= 227 * 1024:
-                break
-        if kbp * 3 * ne * 128 <= 112 * 1024 and total <= 227 * 1024:
+        w = kbp * n3 * 128
+        # the fewest x stages the kernel runs with (it takes up to 8 as room allows)
+        total = (w + 1023) // 1024 * 1024 + 2 * 16384 + 2 * 128 * (ne + 4) * 4 + \
+            max(8 * (ne + 1), 32 * 9) * 4 + 1024
+        if w <= 112 * 1024 and total <= 227 * 1024:
             return 1
     return 3
 
@@ -748,22 +749,49 @@ def run_stage(args):
     for _ in range(max(args.warmup, 1)):
         call()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
+    # warm: a graph of K back-to-back calls (x stays in L2 when it fits)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
         call()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(args.steps):
+                call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    graph.replay()
     e1.record()
     torch.cuda.synchronize()
+    warm_us = e0.elapsed_time(e1) * 1e3 / args.steps
+    del graph
+    # cold: each call timed alone after writing a buffer larger than L2
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    cold = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        cold.append((a, b))
+    torch.cuda.synchronize()
+    cold_us = sorted(a.elapsed_time(b) * 1e3 for a, b in cold)[len(cold) // 2]
     if moe.moe_device_status(ws) != 0:
         raise SystemExit("device status set: a bounded wait expired")
-    us = e0.elapsed_time(e1) * 1e3 / args.steps
     x_bytes = inp.x.numel() * inp.x.element_size()
     peaks, _ = load_peaks()
     print(json.dumps({"stage": "route", "workload": workload_name(shape), "calls": args.steps,
-                      "us_per_call": round(us, 2), "x_bytes": x_bytes,
-                      "GB/s": round(x_bytes / us / 1e3, 1),
-                      "hbm_frac": round(x_bytes / us / 1e3 / peaks["hbm_gbs"], 3),
-                      "timing": "back-to-back calls, CUDA events (launch gaps included)"}))
+                      "us_per_call": round(cold_us, 2), "x_bytes": x_bytes,
+                      "GB/s": round(x_bytes / cold_us / 1e3, 1),
+                      "hbm_frac": round(x_bytes / cold_us / 1e3 / peaks["hbm_gbs"], 3),
+                      "warm_us_per_call": round(warm_us, 2),
+                      "timing": "us_per_call: median of K calls each timed alone (CUDA events) "
+                                "after an L2 flush; warm: a graph of K back-to-back calls"}))
 
 
 def run_stage_ffn(args):

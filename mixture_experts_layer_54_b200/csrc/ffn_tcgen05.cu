@@ -53,8 +53,8 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;         // 320
 // once the TMA store issued from it STG_BUFS steps earlier has read it), as
 // 32 rows of 2 CHUNK bytes in the swizzle of the store map (16-byte chunk c of
 // row r at c ^ ((r >> (3 - SWZ_BITS)) & (2^SWZ_BITS - 1))).
-constexpr int CHUNK = 16;                            // epilogue columns per step
-constexpr int STG_BUFS = 2;
+constexpr int CHUNK = 32;                            // epilogue columns per step
+constexpr int STG_BUFS = 1;
 constexpr int STG_BYTES = 32 * CHUNK * 2;            // one buffer: 32 rows x CHUNK bf16
 constexpr int STG_WARP = STG_BUFS * STG_BYTES;       // a warp's buffers
 constexpr int SWZ_BITS = CHUNK == 16 ? 1 : (CHUNK == 32 ? 2 : 3);   // 32, 64 or 128 B rows
@@ -1295,22 +1295,22 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64
     return r == CUDA_SUCCESS;
 }
 
-int sm_count()
-{
-    int dev = 0, n = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-}
+int sm_count() { return device_sms(); }
 
 template <int EPI, bool GATHER = false>
 cudaError_t launch_2sm(const Params &p, cudaStream_t s)
 {
     auto kern = grouped_gemm_2sm_kernel<EPI, GATHER>;
-    cudaError_t err =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+    const int threads = THREADS + (GATHER ? 32 * GATHER_WARPS : 0);
+    cudaError_t err = raise_smem_limit((const void *)kern, SMEM2_BYTES);
     if (err != cudaSuccess)
         return err;
+    int clusters = 0;
+    err = cached_active_clusters((const void *)kern, threads, SMEM2_BYTES, 2, &clusters);
+    if (err != cudaSuccess)
+        return err;
+    if (clusters < 1)
+        return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1319,20 +1319,12 @@ cudaError_t launch_2sm(const Params &p, cudaStream_t s)
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.blockDim = dim3(THREADS + (GATHER ? 32 * GATHER_WARPS : 0), 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = SMEM2_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cfg.gridDim = dim3(2, 1, 1);
-    int clusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
-    if (err != cudaSuccess)
-        return err;
-    if (clusters < 1)
-        return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3(2 * clusters, 1, 1);
-    cfg.numAttrs = 2;   // and programmatic dependent launch
+    cfg.numAttrs = 2;   // cluster pair and programmatic dependent launch
     err = cudaLaunchKernelEx(&cfg, kern, p);
     if (err != cudaSuccess)
         return err;
@@ -1343,8 +1335,7 @@ template <int EPI, bool GATHER = false>
 cudaError_t launch(const Params &p, cudaStream_t s)
 {
     auto kern = grouped_gemm_kernel<EPI, GATHER>;
-    cudaError_t err =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t err = raise_smem_limit((const void *)kern, SMEM_BYTES);
     if (err != cudaSuccess)
         return err;
     return launch_pdl(kern, dim3(sm_count()), dim3(THREADS + (GATHER ? 32 * GATHER_WARPS : 0)),

@@ -53,6 +53,16 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return err != cudaSuccess ? err : cudaGetLastError();
 }
 
+// ---- launch-shape queries, answered once per device and kernel ----
+int device_sms();
+// Raises (never lowers) the kernel's dynamic shared-memory opt-in to bytes.
+cudaError_t raise_smem_limit(const void *kernel, int bytes);
+cudaError_t cached_blocks_per_sm(const void *kernel, int threads, int smem, int *out);
+// Clusters of `cluster` blocks resident at once (the kernel's opt-in must
+// already cover smem).
+cudaError_t cached_active_clusters(const void *kernel, int threads, int smem, int cluster,
+                                   int *out);
+
 // Shape limits and codes; also the capacity factor rule.
 moe_status validate(const moe_config &c);
 int64_t capacity_of(const moe_config &c);          // valid config only

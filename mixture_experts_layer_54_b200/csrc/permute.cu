@@ -325,10 +325,9 @@ combine_slots_kernel(const uint4 *__restrict__ Y_slot, const uint4 *__restrict__
 template <typename K>
 int grid_for(K kernel, int T)
 {
-    int dev = 0, sms = 148, per_sm = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, THREADS, 0) != cudaSuccess ||
+    const int sms = device_sms();
+    int per_sm = 1;
+    if (cached_blocks_per_sm((const void *)kernel, THREADS, 0, &per_sm) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     const int need = (T + WARPS - 1) / WARPS;

@@ -251,8 +251,7 @@ cudaError_t launch_tiled(const RouteArgs &a, int blocks, cudaStream_t s)
     const int Epad = NX * TN;
     size_t smem = sizeof(float) * (RT * (KC + 1) + KC * Epad + RT * (a.E + 1) + RT);
     auto kern = route_kernel<Tin, TM, TN>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
+    cudaError_t err = raise_smem_limit((const void *)kern, (int)smem);
     if (err != cudaSuccess)
         return err;
     kern<<<blocks, THREADS, smem, s>>>(a);

@@ -26,10 +26,13 @@ __device__ __forceinline__ bool better(float ka, int ia, float kb, int ib)
 // batch: lane L holds the logit of (token L / E_T, expert L % E_T).
 // On return, lanes 0..E_T-1 hold in *pc the batch's sum of expert lane's
 // probability (sigmoid: s / sum s) and every lane holds in *zc the batch's sum
-// of lse^2, both summed over the tokens in a fixed order.
+// of lse^2, both summed over the tokens in a fixed order.  lbias and sbias
+// are the logit and selection biases of expert lane % E_T (read only when
+// the layer has them), loaded once by the caller.
 template <int E_T>
 __device__ __forceinline__ void small_epilogue(const RouteArgs &a, float z, int t0, int lane,
-                                               bool renorm, float *pc_out, float *zc_out)
+                                               bool renorm, float lbias, float sbias,
+                                               float *pc_out, float *zc_out)
 {
     const int E = a.E, T = a.T;
     const int gl = lane % E_T;
@@ -38,7 +41,7 @@ __device__ __forceinline__ void small_epilogue(const RouteArgs &a, float z, int 
     const bool tok = t < T;
     const bool valid = tok && gl < E;
     if (valid && a.logit_bias)
-        z += a.logit_bias[gl];
+        z += lbias;
     float m = valid ? z : -INFINITY;
 #pragma unroll
     for (int o = 1; o < E_T; o <<= 1)
@@ -55,7 +58,7 @@ __device__ __forceinline__ void small_epilogue(const RouteArgs &a, float z, int 
         key = valid ? z : -INFINITY;
     } else {
         v = valid ? 1.f / (1.f + expf(-z)) : 0.f;
-        key = valid ? v + (a.select_bias ? a.select_bias[gl] : 0.f) : -INFINITY;
+        key = valid ? v + (a.select_bias ? sbias : 0.f) : -INFINITY;
     }
     float ssum = v;
 #pragma unroll
@@ -65,42 +68,37 @@ __device__ __forceinline__ void small_epilogue(const RouteArgs &a, float z, int 
         a.logits_out[(int64_t)t * E + gl] = z;
     if (valid && a.scores_out)
         a.scores_out[(int64_t)t * E + gl] = v;
-    // top-k: k rounds of a group argmax over (key, expert), lower index on ties
+    // top-k: k rounds of a group argmax over (key, expert), lower index on
+    // ties; lane gl == j keeps round j's expert and value, so the k outputs go
+    // out from k lanes at once (the gate sum adds the values in round order)
     bool taken = false;
-    int sel_idx[kMaxK];
-    float sel_v[kMaxK];
-    float sel_sum = 0.f;
+    int my_idx = 0;
+    float my_v = 0.f, sel_sum = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < a.k; ++j) {
+        float bk = (!taken && valid) ? key : -INFINITY;
+        int bi = (!taken && valid) ? gl : 0x7fffffff;
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-        sel_idx[j] = 0;
-        sel_v[j] = 0.f;
-        if (j < a.k) {
-            float bk = (!taken && valid) ? key : -INFINITY;
-            int bi = (!taken && valid) ? gl : 0x7fffffff;
-#pragma unroll
-            for (int o = 1; o < E_T; o <<= 1) {
-                const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (better(ok, oi, bk, bi)) {
-                    bk = ok;
-                    bi = oi;
-                }
+        for (int o = 1; o < E_T; o <<= 1) {
+            const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (better(ok, oi, bk, bi)) {
+                bk = ok;
+                bi = oi;
             }
-            const float bv = __shfl_sync(0xffffffffu, v, gbase + (bi < E_T ? bi : 0));
-            if (gl == bi)
-                taken = true;
-            sel_idx[j] = bi;
-            sel_v[j] = bv;
-            sel_sum += bv;
         }
+        const float bv = __shfl_sync(0xffffffffu, v, gbase + (bi < E_T ? bi : 0));
+        if (gl == bi)
+            taken = true;
+        if (gl == j) {
+            my_idx = bi;
+            my_v = bv;
+        }
+        sel_sum += bv;
     }
-    if (tok && gl == 0) {
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j < a.k) {
-                a.topk[(int64_t)t * a.k + j] = sel_idx[j];
-                a.gates[(int64_t)t * a.k + j] = renorm ? sel_v[j] / sel_sum : sel_v[j];
-            }
+    if (tok && gl < a.k) {
+        a.topk[(int64_t)t * a.k + gl] = my_idx;
+        a.gates[(int64_t)t * a.k + gl] = renorm ? my_v / sel_sum : my_v;
     }
     // loss sums over the batch's tokens (lanes of the same expert), fixed order
     float pc = valid ? (a.score == MOE_SCORE_SOFTMAX ? v : v / ssum) : 0.f;

@@ -54,23 +54,38 @@ __device__ __forceinline__ void bar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// Bounded wait (about 2 s of wall clock); false on expiry or once `abort` is set.
-__device__ __noinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                      int32_t *status)
+// Bounded wait (about 2 s of wall clock); false on expiry or once `abort` is
+// set.  Each try suspends the thread until the phase completes or about 20 us
+// pass (a suspended thread takes no issue slots from the warps still
+// working); CLUSTER: acquire at cluster scope, for barriers that blocks of the
+// cluster complete remotely.
+template <bool CLUSTER>
+__device__ __noinline__ bool bar_wait_t(uint32_t bar, uint32_t parity, volatile int *abort,
+                                        int32_t *status)
 {
+    constexpr uint32_t kSuspendNs = 20000;
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
+        if (CLUSTER)
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(bar), "r"(parity), "r"(kSuspendNs)
+                : "memory");
+        else
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(bar), "r"(parity), "r"(kSuspendNs)
+                : "memory");
         if (ok)
             return true;
-        if ((i & 31u) == 0) {
+        if ((i & 3u) == 0) {
             if (abort && *abort)
                 return false;
             uint64_t now;
@@ -86,6 +101,26 @@ __device__ __noinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile in
             }
         }
     }
+}
+
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                         int32_t *status)
+{
+    return bar_wait_t<false>(bar, parity, abort, status);
+}
+
+// The same wait for a whole warp: lane 0 polls, the warp learns the outcome
+// (and, through the warp barrier, sees what the completed phase published).
+template <bool CLUSTER>
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                          int32_t *status)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0)
+        ok = bar_wait_t<CLUSTER>(bar, parity, abort, status) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
 }
 
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t a)
@@ -151,115 +186,181 @@ struct __align__(64) RouteParams {
     int cs, k_parts, kb_per_part, k_blocks;
     int tiles, nclusters, stages;   // one-kernel router: token tiles, clusters, x stages
     int clear_status;               // 1: block 0 clears the status word first
+    int w_bulk;                     // 1: W_r is 16-byte aligned (its K parts copied in bulk)
     int32_t *status;
 };
 
 // ------------------------------------------------------------- selection
 
-// One token held by a whole warp, lane l holding experts l, l + 32, ... (PL of
-// them): softmax or sigmoid, top-k and gates; adds the token's loss terms to
-// pacc / zacc.  SB_REG: sb holds the lane's selection biases (0 without);
-// otherwise they are read from a.select_bias.  Each top-k round
-// is two integer warp reductions: the largest key, then the lowest expert
-// index holding it (ties go to the lower index).
-template <int PL, bool SB_REG>
-__device__ __forceinline__ void select_token(const RouteParams &a, bool renorm, int t, int lane,
-                                             const float (&z)[PL], const float (&sb)[PL],
-                                             float (&pacc)[PL], float &zacc)
+// The fields selection reads, copied out of the kernel parameters once so
+// that they stay in registers across a token's global stores (read through
+// the parameter block they could be re-read after every store).
+struct SelArgs {
+    int32_t *topk;
+    float *gates, *logits_out, *scores_out;
+    const float *select_bias;
+    int E, k, score;
+};
+__device__ __forceinline__ SelArgs sel_args(const RouteParams &p)
+{
+    return SelArgs{p.topk, p.gates, p.logits_out, p.scores_out, p.select_bias, p.E, p.k, p.score};
+}
+
+// NT tokens held by a whole warp, lane l holding experts l, l + 32, ... (PL
+// of them) of each: softmax or sigmoid, top-k and gates; adds the loss terms
+// of the tokens with tv set to pacc / zacc in token order.  The NT tokens'
+// steps are independent, so the warp keeps NT dependency chains in flight
+// instead of one.  SB_REG: sb holds the lane's selection biases (0 without);
+// otherwise they are read from a.select_bias.  Each top-k round is two integer
+// warp reductions: the largest key, then the lowest expert index holding it
+// (ties go to the lower index); lane j keeps round j's expert and value, so
+// the k outputs go out from k lanes at once (the gate sum still adds the
+// values in round order).  A token with tv clear takes part in the warp
+// reductions (with finite logits) and writes nothing.
+template <int PL, int NT, bool SB_REG>
+__device__ __forceinline__ void select_tokens(const SelArgs &a, bool renorm, const int (&t)[NT],
+                                              const bool (&tv)[NT], int lane,
+                                              const float (&z)[NT][PL], const float (&sb)[PL],
+                                              float (&pacc)[PL], float &zacc)
 {
     const int E = a.E;
-    uint32_t mo = 0;
+    float m[NT], sum[NT], lse[NT], ssum[NT], v[NT][PL];
+    uint32_t okey[NT][PL];   // 0: not an expert of this layer, or taken
 #pragma unroll
-    for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i < E)
-            mo = max(mo, ord_key(z[i]));
-    const float m = unord_key(__reduce_max_sync(0xffffffffu, mo));
-    float sum = 0.f;
+    for (int n = 0; n < NT; ++n) {
+        uint32_t mo = 0;
 #pragma unroll
-    for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i < E)
-            sum += expf(z[i] - m);
+        for (int i = 0; i < PL; ++i)
+            if (lane + 32 * i < E)
+                mo = max(mo, ord_key(z[n][i]));
+        m[n] = unord_key(__reduce_max_sync(0xffffffffu, mo));
+    }
+    float ex[NT][PL];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        sum[n] = 0.f;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+            ex[n][i] = lane + 32 * i < E ? expf(z[n][i] - m[n]) : 0.f;
+            sum[n] += ex[n][i];
+        }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
-        sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float lse = m + logf(sum);
-    float v[PL];
-    uint32_t okey[PL];   // 0: not an expert of this layer
-    float ssum = 0.f;
 #pragma unroll
-    for (int i = 0; i < PL; ++i) {
-        const int e = lane + 32 * i;
-        const bool okk = e < E;
-        float key;
-        if (a.score == MOE_SCORE_SOFTMAX) {
-            v[i] = okk ? expf(z[i] - m) / sum : 0.f;
-            key = z[i];
-        } else {
-            v[i] = okk ? 1.f / (1.f + expf(-z[i])) : 0.f;
-            key = v[i] + (SB_REG ? sb[i] : (a.select_bias && okk ? a.select_bias[e] : 0.f));
-            ssum += v[i];
+        for (int n = 0; n < NT; ++n)
+            sum[n] += __shfl_xor_sync(0xffffffffu, sum[n], o);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        lse[n] = m[n] + logf(sum[n]);
+        ssum[n] = 0.f;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+            const int e = lane + 32 * i;
+            const bool okk = e < E;
+            float key;
+            if (a.score == MOE_SCORE_SOFTMAX) {
+                v[n][i] = okk ? ex[n][i] / sum[n] : 0.f;
+                key = z[n][i];
+            } else {
+                v[n][i] = okk ? 1.f / (1.f + expf(-z[n][i])) : 0.f;
+                key = v[n][i] + (SB_REG ? sb[i] : (a.select_bias && okk ? a.select_bias[e] : 0.f));
+                ssum[n] += v[n][i];
+            }
+            okey[n][i] = okk ? ord_key(key) : 0u;
+            if (okk && tv[n] && a.logits_out)
+                a.logits_out[(int64_t)t[n] * E + e] = z[n][i];
+            if (okk && tv[n] && a.scores_out)
+                a.scores_out[(int64_t)t[n] * E + e] = v[n][i];
         }
-        okey[i] = okk ? ord_key(key) : 0u;
-        if (okk && a.logits_out)
-            a.logits_out[(int64_t)t * E + e] = z[i];
-        if (okk && a.scores_out)
-            a.scores_out[(int64_t)t * E + e] = v[i];
     }
     if (a.score == MOE_SCORE_SIGMOID) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
-            ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+                ssum[n] += __shfl_xor_sync(0xffffffffu, ssum[n], o);
     }
-    int sel_idx[kMaxK];
-    float sel_v[kMaxK];
-    float sel_sum = 0.f;
+    int my_idx[NT];
+    float my_v[NT], sel_sum[NT];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-        sel_idx[j] = 0;
-        sel_v[j] = 0.f;
-        if (j >= a.k)
-            continue;
-        uint32_t lk = 0;
+    for (int n = 0; n < NT; ++n) {
+        my_idx[n] = 0;
+        my_v[n] = 0.f;
+        sel_sum[n] = 0.f;
+    }
+#pragma unroll 1
+    for (int j = 0; j < a.k; ++j) {
+        uint32_t mk[NT];
 #pragma unroll
-        for (int i = 0; i < PL; ++i)
-            lk = max(lk, okey[i]);
-        const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
-        uint32_t li = 0xffffffffu;
-#pragma unroll
-        for (int i = PL - 1; i >= 0; --i)
-            if (okey[i] == mk && mk != 0u)
-                li = (uint32_t)(lane + 32 * i);
-        const uint32_t bi = __reduce_min_sync(0xffffffffu, li);
-        const int slot = (int)(bi >> 5);
-        float mine = v[0];
-#pragma unroll
-        for (int i = 1; i < PL; ++i)
-            if (slot == i)
-                mine = v[i];
-        const float bv = __shfl_sync(0xffffffffu, mine, (int)(bi & 31u));
-        if ((int)(bi & 31u) == lane) {
+        for (int n = 0; n < NT; ++n) {
+            uint32_t lk = 0;
 #pragma unroll
             for (int i = 0; i < PL; ++i)
-                if (slot == i)
-                    okey[i] = 0u;   // taken
+                lk = max(lk, okey[n][i]);
+            mk[n] = __reduce_max_sync(0xffffffffu, lk);
         }
-        sel_idx[j] = (int)bi;
-        sel_v[j] = bv;
-        sel_sum += bv;
-    }
-    if (lane == 0) {
+        uint32_t bi[NT];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j < a.k) {
-                a.topk[(int64_t)t * a.k + j] = sel_idx[j];
-                a.gates[(int64_t)t * a.k + j] = renorm ? sel_v[j] / sel_sum : sel_v[j];
+        for (int n = 0; n < NT; ++n) {
+            uint32_t li = 0xffffffffu;
+#pragma unroll
+            for (int i = PL - 1; i >= 0; --i)
+                if (okey[n][i] == mk[n] && mk[n] != 0u)
+                    li = (uint32_t)(lane + 32 * i);
+            bi[n] = __reduce_min_sync(0xffffffffu, li);
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int slot = (int)(bi[n] >> 5);
+            float mine = v[n][0];
+#pragma unroll
+            for (int i = 1; i < PL; ++i)
+                if (slot == i)
+                    mine = v[n][i];
+            const float bv = __shfl_sync(0xffffffffu, mine, (int)(bi[n] & 31u));
+            if ((int)(bi[n] & 31u) == lane) {
+#pragma unroll
+                for (int i = 0; i < PL; ++i)
+                    if (slot == i)
+                        okey[n][i] = 0u;   // taken
             }
-        zacc += lse * lse;
+            if (lane == j) {
+                my_idx[n] = (int)bi[n];
+                my_v[n] = bv;
+            }
+            sel_sum[n] += bv;
+        }
     }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        if (!tv[n])
+            continue;
+        if (lane < a.k) {
+            a.topk[(int64_t)t[n] * a.k + lane] = my_idx[n];
+            a.gates[(int64_t)t[n] * a.k + lane] = renorm ? my_v[n] / sel_sum[n] : my_v[n];
+        }
+        if (lane == 0)
+            zacc += lse[n] * lse[n];
+#pragma unroll
+        for (int i = 0; i < PL; ++i)
+            if (lane + 32 * i < E)
+                pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[n][i] : v[n][i] / ssum[n];
+    }
+}
+
+template <int PL, bool SB_REG>
+__device__ __forceinline__ void select_token(const SelArgs &a, bool renorm, int t, int lane,
+                                             const float (&z)[PL], const float (&sb)[PL],
+                                             float (&pacc)[PL], float &zacc)
+{
+    const int tt[1] = {t};
+    const bool tv[1] = {true};
+    float zz[1][PL];
 #pragma unroll
     for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i < E)
-            pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[i] : v[i] / ssum;
+        zz[0][i] = z[i];
+    select_tokens<PL, 1, SB_REG>(a, renorm, tt, tv, lane, zz, sb, pacc, zacc);
 }
 
 // ---------------------------------------------------------------- kernel
@@ -278,12 +379,13 @@ __device__ __forceinline__ void select_token(const RouteParams &a, bool renorm, 
 //                accumulators (tile i uses buffer i mod 2);
 //   warps 2-5    read an accumulator back (hi + (mid + lo)) and push each
 //                token's partial logits into buffer i mod 2 of the block that
-//                selects that token (st.shared::cluster, slot = this block's
-//                K part), then tell every block of the cluster (a remote
-//                mbarrier arrive, release at cluster scope);
-//   warps 6-13   select 128 / P tokens of the tile from their own buffer,
-//                summing the P parts in part order; then tell every block
-//                that the buffer may be filled again.
+//                selects that token (st.async, slot = this block's K part):
+//                each store's bytes count on that block's lfull barrier, so
+//                no fence or remote arrive follows the pushes;
+//   warps 6-13   select 128 / P tokens of the tile from their own buffer once
+//                its BM x NE floats have landed, summing the P parts in part
+//                order; then arm the buffer's barrier for its next use and
+//                tell every block that the buffer may be filled again.
 // So one tile's read-back and selection run while the next tile's x streams,
 // and no warp waits on a remote load.
 
@@ -292,16 +394,48 @@ constexpr int RB_WARP0 = 2;       // warps 2-5: TMEM read-back
 constexpr int SEL_WARP0 = 6;      // warps 6-13: selection
 constexpr int SEL_WARPS = 8;
 constexpr int SEL_THREADS = SEL_WARPS * 32;
+static_assert(RB_WARP0 == 2 && SEL_WARP0 == RB_WARP0 + 4, "warps 0, 1: TMA, MMA; then 4 read-back");
 constexpr int CONV_WARP0 = 2;     // warps 2-13 split W_r first
 constexpr int CONV_THREADS = PR_THREADS - CONV_WARP0 * 32;
 constexpr int MAX_STAGES = 8;
 constexpr int W_MAX_BYTES = 112 * 1024;   // resident split weights per block
 
-// Store four floats to shared memory of another block of the cluster.
-__device__ __forceinline__ void st_peer4(uint32_t a, float4 v)
+// This warp's 32 TMEM lanes x 16 (or 8) consecutive fp32 columns from taddr.
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[16])
 {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v.x),
-                 "f"(v.y), "f"(v.z), "f"(v.w)
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
+// Asynchronous store of four floats to shared memory of a block of the
+// cluster (a and bar are cluster shared addresses of that block): when the 16
+// bytes have landed they count against the transaction bytes the block's
+// mbarrier bar expects, so the reader needs no fence or arrive from the writer.
+__device__ __forceinline__ void st_async4(uint32_t a, float4 v, uint32_t bar)
+{
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+        "[%5];" ::"r"(a),
+        "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+        : "memory");
+}
+
+// Arrive on a barrier of this block, first raising the transaction bytes its
+// current phase waits for.
+__device__ __forceinline__ void arrive_expect(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
 
@@ -312,45 +446,12 @@ __device__ __forceinline__ void named_sync(int id, int threads)
 }
 
 // Arrive on the mbarrier at the same shared offset in block `rank` of the
-// cluster, releasing this thread's earlier writes at cluster scope.
-__device__ __forceinline__ void arrive_remote(uint32_t bar, uint32_t rank)
+// cluster, with no memory ordering: a bare "go" signal.
+__device__ __forceinline__ void arrive_remote_relaxed(uint32_t bar, uint32_t rank)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                      peer_addr(bar, rank))
                  : "memory");
-}
-
-// Bounded wait that acquires at cluster scope (for barriers that blocks of
-// the cluster arrive on remotely).
-__device__ __noinline__ bool bar_wait_cluster(uint32_t bar, uint32_t parity, volatile int *abort,
-                                              int32_t *status)
-{
-    uint64_t t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (ok)
-            return true;
-        if ((i & 31u) == 0) {
-            if (*abort)
-                return false;
-            uint64_t now;
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
-            if (i == 0) {
-                t0 = now;
-            } else if (now - t0 > 2000000000ull) {
-                *abort = 1;
-                atomicExch(status, (int32_t)MOE_ERR_DEVICE_TIMEOUT);
-                return false;
-            }
-        }
-    }
 }
 
 // Shared-memory plan of the kernel (host and device agree on it).
@@ -360,7 +461,7 @@ struct RouteSmem {
 __host__ __device__ inline RouteSmem route_smem(int NE, int kbp, int stages)
 {
     RouteSmem s;
-    const int N3 = 3 * NE;
+    const int N3 = (3 * NE + 15) / 16 * 16;   // the MMA's N: hi, mid, lo rows, padded
     s.w = 0;
     s.x = (kbp * N3 * 128 + 1023) / 1024 * 1024;
     s.l = s.x + stages * A_BYTES;
@@ -378,7 +479,7 @@ __host__ __device__ inline RouteSmem route_smem(int NE, int kbp, int stages)
 template <int NE, int E_T, int PL>
 __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_constant__ RouteParams p)
 {
-    constexpr int N3 = 3 * NE;                       // hi, mid, lo rows of B
+    constexpr int N3 = (3 * NE + 15) / 16 * 16;      // hi, mid, lo rows of B (+ zero rows)
     constexpr int WT_BYTES = N3 * 128;               // one K block of B
     constexpr uint32_t ACC = N3 <= 64 ? 64 : (N3 <= 128 ? 128 : 256);   // columns per buffer
     constexpr uint32_t TMEM_COLS = 2 * ACC;
@@ -386,12 +487,14 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                                ((uint32_t)(BM >> 4) << 24);
     constexpr int LS = NE + 4;                       // row stride (floats) of a logit buffer
     constexpr int L_BYTES = BM * LS * 4;
+    constexpr int L_PUSH = BM * NE * 4;              // bytes pushed into a buffer per tile
     static_assert(N3 % 16 == 0 && N3 <= 256, "MMA N");
+    static_assert(NE == 8 || NE % 16 == 0, "experts per MMA: 8 or a multiple of 16");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], wready, tfull[2],
+    __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], wready, wbar, tfull[2],
         tempty[2], lfull[2], lempty[2], drain;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
@@ -417,16 +520,22 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             bar_init(saddr(&empty[s]), 1);
         }
         bar_init(saddr(&wready), CONV_THREADS / 32);
+        bar_init(saddr(&wbar), 1);
         for (int a = 0; a < 2; ++a) {
             bar_init(saddr(&tfull[a]), 1);
             bar_init(saddr(&tempty[a]), 4);
-            bar_init(saddr(&lfull[a]), (uint32_t)P);
+            // a phase of lfull[a]: this block's own arrive, which also sets the
+            // bytes the cluster's read-back pushes into buffer a (BM rows of NE
+            // floats: TPC rows from each of the P blocks)
+            bar_init(saddr(&lfull[a]), 1);
             bar_init(saddr(&lempty[a]), (uint32_t)P);
         }
         bar_init(saddr(&drain), 1);
         abort_flag = 0;
         rb_fail = 0;
         sel_fail = 0;
+        for (int a = 0; a < 2; ++a)   // the first use of each buffer
+            arrive_expect(saddr(&lfull[a]), (uint32_t)L_PUSH);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -449,57 +558,75 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
 
     if (warp >= CONV_WARP0) {
         // ---- prologue: this block's K part of W_r -> three bf16 terms ----
-        // Chunk c = (K block i, 8-wide K group j, expert e), e fastest so that
-        // neighbouring threads read neighbouring W_r words; its 16 bytes of
-        // each term go to row e (+ NE, + 2 NE) of K block i's tile, at
-        // position j ^ (row & 7) of the row's eight (128-byte swizzle).  A
-        // thread issues the loads of CB chunks before converting any.
-        constexpr int CB = 4;
+        // Chunk c = (K block i, 8-wide K group j, expert e < E), e fastest;
+        // its 16 bytes of each term go to row e (+ NE, + 2 NE) of K block i's
+        // tile, at position j ^ (row & 7) of the row's eight (128-byte
+        // swizzle).  The part (kbp x 64 rows of E floats, contiguous in W_r)
+        // arrives by bulk copies into the tail of the split-weight region,
+        // issued by the TMA thread ahead of any x tile; every thread reads all
+        // of its chunks (at most CB: 8 kbp E <= 8 kbp NE <= CB x 384 on every
+        // layer this kernel takes) before any thread writes a term over the
+        // staged part.  Without 16-byte alignment the threads load the part
+        // from global memory themselves.
+        constexpr int CB = 6;
         const int ct = threadIdx.x - CONV_WARP0 * 32;
-        const int E = p.E, nchunk = kbp * 8 * NE;
-        for (int c0 = ct; c0 < nchunk; c0 += CB * CONV_THREADS) {
-            float w[CB][8];
+        const int E = p.E, nchunk = kbp * 8 * E;
+        const float *stage =
+            reinterpret_cast<const float *>(Wres + kbp * WT_BYTES - kbp * BK * E * 4);
+        if (p.w_bulk)   // expiry: recorded, go on
+            warp_wait<false>(saddr(&wbar), 0, &abort_flag, p.status);
+        float w[CB][8];
 #pragma unroll
-            for (int b = 0; b < CB; ++b) {
-                const int c = c0 + b * CONV_THREADS;
-                const int e = c % NE, j = (c / NE) % 8, i = c / (NE * 8);
-                const bool live = c < nchunk && e < E;
-                const int64_t k0 = (int64_t)(kb0 + i) * BK + 8 * j;
+        for (int b = 0; b < CB; ++b) {
+            const int c = ct + b * CONV_THREADS;
+            const int e = c % E, j = (c / E) % 8, i = c / (E * 8);
+            const int r0 = i * BK + 8 * j;   // row of the part
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    w[b][u] = live ? p.W_r[(k0 + u) * E + e] : 0.f;
-            }
+            for (int u = 0; u < 8; ++u)
+                w[b][u] = c >= nchunk ? 0.f
+                          : p.w_bulk  ? stage[(r0 + u) * E + e]
+                                      : p.W_r[((int64_t)kb0 * BK + r0 + u) * E + e];
+        }
+        named_sync(3, CONV_THREADS);   // the staged part is read: terms may overwrite it
 #pragma unroll
-            for (int b = 0; b < CB; ++b) {
-                const int c = c0 + b * CONV_THREADS;
-                if (c >= nchunk)
-                    break;
-                const int e = c % NE, j = (c / NE) % 8, i = c / (NE * 8);
-                uint32_t hi[4], mid[4], lo[4];
+        for (int b = 0; b < CB; ++b) {
+            const int c = ct + b * CONV_THREADS;
+            if (c >= nchunk)
+                break;
+            const int e = c % E, j = (c / E) % 8, i = c / (E * 8);
+            uint32_t hi[4], mid[4], lo[4];
 #pragma unroll
-                for (int u = 0; u < 8; u += 2) {
-                    __nv_bfloat16 h[2], md[2], l[2];
+            for (int u = 0; u < 8; u += 2) {
+                __nv_bfloat16 h[2], md[2], l[2];
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const float x = w[b][u + r];
-                        h[r] = __float2bfloat16_rn(x);
-                        const float r1 = x - __bfloat162float(h[r]);
-                        md[r] = __float2bfloat16_rn(r1);
-                        l[r] = __float2bfloat16_rn(r1 - __bfloat162float(md[r]));
-                    }
-                    hi[u / 2] = pack2(h[0], h[1]);
-                    mid[u / 2] = pack2(md[0], md[1]);
-                    lo[u / 2] = pack2(l[0], l[1]);
+                for (int r = 0; r < 2; ++r) {
+                    const float x = w[b][u + r];
+                    h[r] = __float2bfloat16_rn(x);
+                    const float r1 = x - __bfloat162float(h[r]);
+                    md[r] = __float2bfloat16_rn(r1);
+                    l[r] = __float2bfloat16_rn(r1 - __bfloat162float(md[r]));
                 }
-                uint8_t *tile = Wres + i * WT_BYTES;
-                const uint32_t *terms[3] = {hi, mid, lo};
-#pragma unroll
-                for (int sp = 0; sp < 3; ++sp) {
-                    const int row = sp * NE + e;
-                    *reinterpret_cast<uint4 *>(tile + row * 128 + ((j ^ (row & 7)) << 4)) =
-                        make_uint4(terms[sp][0], terms[sp][1], terms[sp][2], terms[sp][3]);
-                }
+                hi[u / 2] = pack2(h[0], h[1]);
+                mid[u / 2] = pack2(md[0], md[1]);
+                lo[u / 2] = pack2(l[0], l[1]);
             }
+            uint8_t *tile = Wres + i * WT_BYTES;
+            const uint32_t *terms[3] = {hi, mid, lo};
+#pragma unroll
+            for (int sp = 0; sp < 3; ++sp) {
+                const int row = sp * NE + e;
+                *reinterpret_cast<uint4 *>(tile + row * 128 + ((j ^ (row & 7)) << 4)) =
+                    make_uint4(terms[sp][0], terms[sp][1], terms[sp][2], terms[sp][3]);
+            }
+        }
+        // zero rows: the padding experts E .. NE - 1 of every term, and the
+        // rows 3 NE .. N3 - 1 that round the MMA's N up to a multiple of 16
+        const int dead = NE - E, zrows = 3 * dead + (N3 - 3 * NE), nz = kbp * zrows * 8;
+        for (int z = ct; z < nz; z += CONV_THREADS) {
+            const int q16 = z % 8, zr = (z / 8) % zrows, i = z / (8 * zrows);
+            const int row = zr < 3 * dead ? (zr / dead) * NE + E + zr % dead : 3 * NE + zr - 3 * dead;
+            *reinterpret_cast<uint4 *>(Wres + i * WT_BYTES + row * 128 + q16 * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
         }
         // generic-proxy stores, read next by the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -515,7 +642,29 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             int last_issue[MAX_STAGES];
             for (int s = 0; s < MAX_STAGES; ++s)
                 last_issue[s] = -1;
-            bool ok = true;
+            // this block's K part of W_r first, in pieces of up to 16 KB
+            const uint32_t wbytes = (uint32_t)(kbp * BK * p.E * 4);
+            if (p.w_bulk) {
+                const uint32_t wb = saddr(&wbar);
+                const uint32_t dst = saddr(Wres + kbp * WT_BYTES) - wbytes;
+                const char *src = reinterpret_cast<const char *>(p.W_r + (int64_t)kb0 * BK * p.E);
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(wb),
+                             "r"(wbytes)
+                             : "memory");
+                for (uint32_t o = 0; o < wbytes; o += 16384) {
+                    const uint32_t n = wbytes - o < 16384 ? wbytes - o : 16384;
+                    asm volatile(
+                        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], "
+                        "%2, [%3];" ::"r"(dst + o),
+                        "l"(src + o), "r"(n), "r"(wb)
+                        : "memory");
+                }
+            }
+            // x waits until the terms are written: issued together, the whole
+            // grid's first x tiles (stages x 16 KB per block) would share the
+            // memory system with W_r, and the converters' proxy fence would
+            // wait for them to land
+            bool ok = bar_wait(saddr(&wready), 0, &abort_flag, p.status);
             for (int tile = cl; ok && tile < p.tiles; tile += ncl) {
                 for (int i = 0; i < kbp; ++i, ++it) {
                     const int s = it % ST;
@@ -538,6 +687,8 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                 }
             }
             // copies in flight land before the block moves on (bounded)
+            if (p.w_bulk)
+                bar_wait(saddr(&wbar), 0, nullptr, nullptr);
             for (int s = 0; s < ST; ++s)
                 if (last_issue[s] >= 0)
                     bar_wait(saddr(&full[s]), (uint32_t)((last_issue[s] / ST) & 1), nullptr,
@@ -603,47 +754,41 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
         int tc = 0;
         for (int tile = cl; tile < p.tiles; tile += ncl, ++tc) {
             const int a = tc & 1, n = tc >> 1;
-            bool okw = __all_sync(0xffffffffu, bar_wait(saddr(&tfull[a]), (uint32_t)(n & 1),
-                                                        &abort_flag, p.status));
+            bool okw = warp_wait<false>(saddr(&tfull[a]), (uint32_t)(n & 1), &abort_flag, p.status);
             // the cluster's selection of the tile that last used this buffer is done
             if (okw)
-                okw = __all_sync(0xffffffffu, bar_wait_cluster(saddr(&lempty[a]),
-                                                               (uint32_t)((n & 1) ^ 1),
-                                                               &abort_flag, p.status));
+                okw = warp_wait<false>(saddr(&lempty[a]), (uint32_t)((n & 1) ^ 1), &abort_flag,
+                                       p.status);
             if (!okw && lane == 0)
                 rb_fail = 1;
             named_sync(1, 128);
             if (rb_fail)
                 break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            // this lane's token row goes to the block selecting it, slot `rank`
+            // this lane's token row goes to the block selecting it, slot
+            // `rank`; the owner's lfull[a] counts the bytes as they land
             const int row = q * 32 + lane, owner = row / TPC, tl = row % TPC;
             const uint32_t dst = peer_addr(lbase, (uint32_t)owner) +
                                  (uint32_t)(a * L_BYTES + (rank * TPC + tl) * LS * 4);
+            const uint32_t dbar = peer_addr(saddr(&lfull[a]), (uint32_t)owner);
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)a * ACC;
+            constexpr int CW = NE < 16 ? NE : 16;   // columns per load and term
 #pragma unroll
-            for (int c = 0; c < NE; c += 16) {
-                uint32_t r[3][16];
+            for (int c = 0; c < NE; c += CW) {
+                uint32_t r[3][CW];
 #pragma unroll
                 for (int sp = 0; sp < 3; ++sp)
-                    asm volatile(
-                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-                        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
-                        "[%16];"
-                        : "=r"(r[sp][0]), "=r"(r[sp][1]), "=r"(r[sp][2]), "=r"(r[sp][3]),
-                          "=r"(r[sp][4]), "=r"(r[sp][5]), "=r"(r[sp][6]), "=r"(r[sp][7]),
-                          "=r"(r[sp][8]), "=r"(r[sp][9]), "=r"(r[sp][10]), "=r"(r[sp][11]),
-                          "=r"(r[sp][12]), "=r"(r[sp][13]), "=r"(r[sp][14]), "=r"(r[sp][15])
-                        : "r"(tb + (uint32_t)(sp * NE + c)));
+                    tmem_ld_cols(tb + (uint32_t)(sp * NE + c), r[sp]);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                for (int h = 0; h < 16; h += 4) {
+                for (int h = 0; h < CW; h += 4) {
                     float v[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u)   // x W_hi + (x W_mid + x W_lo)
                         v[u] = __uint_as_float(r[0][h + u]) +
                                (__uint_as_float(r[1][h + u]) + __uint_as_float(r[2][h + u]));
-                    st_peer4(dst + (uint32_t)((c + h) * 4), make_float4(v[0], v[1], v[2], v[3]));
+                    st_async4(dst + (uint32_t)((c + h) * 4), make_float4(v[0], v[1], v[2], v[3]),
+                              dbar);
                 }
             }
             // accumulator free for the tile after next
@@ -651,11 +796,6 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             __syncwarp();
             if (lane == 0)
                 bar_arrive(saddr(&tempty[a]));
-            // the four read-back warps' rows are pushed: tell every block
-            named_sync(1, 128);
-            if (warp == RB_WARP0 && lane == 0)
-                for (int r = 0; r < P; ++r)
-                    arrive_remote(saddr(&lfull[a]), (uint32_t)r);
         }
     } else {
         // ---- selection: this block's share of every tile's tokens ----
@@ -665,6 +805,7 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
         const int sw = warp - SEL_WARP0;   // selection warp 0..7
         const int tl0 = rank * TPC;
         const bool renorm = p.renorm < 0 ? (p.k > 1) : (p.renorm != 0);
+        const SelArgs sa = sel_args(p);
         float *scratch = reinterpret_cast<float *>(smem + sm.scratch);
         float lb[PL], sb[PL];   // per-expert biases of this lane, loaded once
 #pragma unroll
@@ -673,12 +814,15 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             lb[i] = p.logit_bias && e < E ? p.logit_bias[e] : 0.f;
             sb[i] = p.select_bias && e < E ? p.select_bias[e] : 0.f;
         }
+        // narrow layers: lane L serves expert L % E_T
+        const int gle = E_T > 0 ? lane % (E_T > 0 ? E_T : 1) : 0;
+        const float lbv = E_T > 0 && p.logit_bias && gle < E ? p.logit_bias[gle] : 0.f;
+        const float sbv = E_T > 0 && p.select_bias && gle < E ? p.select_bias[gle] : 0.f;
         int tc = 0;
         for (int tile = cl; tile < p.tiles; tile += ncl, ++tc) {
             const int a = tc & 1, n = tc >> 1;
-            const bool okw = __all_sync(0xffffffffu, bar_wait_cluster(saddr(&lfull[a]),
-                                                                      (uint32_t)(n & 1),
-                                                                      &abort_flag, p.status));
+            const bool okw =
+                warp_wait<true>(saddr(&lfull[a]), (uint32_t)(n & 1), &abort_flag, p.status);
             if (!okw && lane == 0)
                 sel_fail = 1;
             named_sync(2, SEL_THREADS);
@@ -707,7 +851,7 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                             z += Lb[(q * TPC + tl - tl0) * LS + gl];
                     }
                     float pc, zc;
-                    small_epilogue<E_T>(ra, z, m0 + tg, lane, renorm, &pc, &zc);
+                    small_epilogue<E_T>(ra, z, m0 + tg, lane, renorm, lbv, sbv, &pc, &zc);
                     if (lane < E_T)
                         scratch[g * (E_T + 1) + lane] = pc;
                     if (lane == 0)
@@ -725,36 +869,39 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                 }
                 named_sync(2, SEL_THREADS);   // scratch free, every read of the buffers done
             } else {
-                // a warp per token: selection warp w takes tokens w, w + 8, ...
-                // of each row of 32; the row's sums meet in shared memory in
-                // warp order
+                // selection warp w takes tokens w, w + 8, w + 16 and w + 24 of
+                // each row of 32, all four at once, a whole warp per token; the
+                // row's sums meet in shared memory in warp order
                 for (int r = 0; r < rows; ++r) {
                     float pacc[PL];
 #pragma unroll
                     for (int i = 0; i < PL; ++i)
                         pacc[i] = 0.f;
                     float zacc = 0.f;
-                    for (int u = sw; u < kPartialTokens; u += SEL_WARPS) {
-                        const int tl = tl0 + r * kPartialTokens + u;
-                        const int t = m0 + tl;
-                        if (t >= p.T)
-                            break;
-                        float z[PL];
+                    // the warp's tokens of the row (sw, sw + 8, ...) at once
+                    constexpr int NT = kPartialTokens / SEL_WARPS;
+                    int tt[NT];
+                    bool tv[NT];
+                    float z[NT][PL];
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        const int tl = tl0 + r * kPartialTokens + sw + n * SEL_WARPS;
+                        tt[n] = m0 + tl;
+                        tv[n] = tt[n] < p.T;
 #pragma unroll
                         for (int i = 0; i < PL; ++i) {
                             const int e = lane + 32 * i;
-                            z[i] = -INFINITY;
-                            if (e < E) {
-                                float s = 0.f;
+                            float sum = 0.f;
+                            if (e < E && tv[n]) {
                                 for (int q = 0; q < P; ++q)
-                                    s += Lb[(q * TPC + tl - tl0) * LS + e];
+                                    sum += Lb[(q * TPC + tl - tl0) * LS + e];
                                 if (p.logit_bias)
-                                    s += lb[i];
-                                z[i] = s;
+                                    sum += lb[i];
                             }
+                            z[n][i] = sum;
                         }
-                        select_token<PL, true>(p, renorm, t, lane, z, sb, pacc, zacc);
                     }
+                    select_tokens<PL, NT, true>(sa, renorm, tt, tv, lane, z, sb, pacc, zacc);
 #pragma unroll
                     for (int i = 0; i < PL; ++i)
                         if (lane + 32 * i < E)
@@ -774,10 +921,15 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
                     named_sync(2, SEL_THREADS);
                 }
             }
-            // this block is done reading every block's buffer a for the tile
-            if (st == 0)
+            // this block is done reading buffer a: arm it for its next use,
+            // then let every block of the cluster push into it again
+            if (st == 0) {
+                arrive_expect(saddr(&lfull[a]), (uint32_t)L_PUSH);
+                // relaxed: every read of the buffer returned its value before
+                // the named barrier above, so later pushes cannot change them
                 for (int r = 0; r < P; ++r)
-                    arrive_remote(saddr(&lempty[a]), (uint32_t)r);
+                    arrive_remote_relaxed(saddr(&lempty[a]), (uint32_t)r);
+            }
         }
     }
 
@@ -1035,7 +1187,8 @@ __global__ void __launch_bounds__(32 * kPartialTokens, 1)
                 z[i] = s;
             }
         }
-        select_token<PL, false>(a, renorm, t, lane, z, sb, pacc, zacc);
+        const SelArgs sa = sel_args(a);
+        select_token<PL, false>(sa, renorm, t, lane, z, sb, pacc, zacc);
     }
 #pragma unroll
     for (int i = 0; i < PL; ++i)
@@ -1121,29 +1274,25 @@ cudaError_t launch(RouteParams p, cudaStream_t s)
 {
     auto kern = route_kernel<NE, E_T, PL>;
     const int smem = route_smem(NE, p.kb_per_part, p.stages).total;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t err = raise_smem_limit((const void *)kern, smem);
     if (err != cudaSuccess)
         return err;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof cfg);
-    cfg.blockDim = dim3(PR_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    LaunchAttrs la(p.cs, false);
-    cfg.attrs = la.at;
-    cfg.numAttrs = la.n;
     // as many clusters as fit at once (every block must be resident: blocks of
     // a cluster wait on one another), at most one per tile, the tiles spread
     // evenly over them
-    cfg.gridDim = dim3((unsigned)p.cs);
     int fit = 0;
-    err = cudaOccupancyMaxActiveClusters(&fit, kern, &cfg);
+    err = cached_active_clusters((const void *)kern, PR_THREADS, smem, p.cs, &fit);
     if (err != cudaSuccess)
         return err;
     if (fit < 1)
         return cudaErrorInvalidConfiguration;
     const int per = (int)ceil_div(p.tiles, fit);
     p.nclusters = (int)ceil_div(p.tiles, per);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.blockDim = dim3(PR_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
     cfg.gridDim = dim3((unsigned)(p.nclusters * p.cs));
     LaunchAttrs lp(p.cs, true);
     cfg.attrs = lp.at;
@@ -1156,7 +1305,7 @@ cudaError_t launch_logits(const LogitParams &p, dim3 grid, cudaStream_t s)
 {
     constexpr int smem = STAGES * (A_BYTES + 3 * N * BK * 2) + 1024;
     auto kern = logits_kernel<N>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t err = raise_smem_limit((const void *)kern, smem);
     if (err != cudaSuccess)
         return err;
     kern<<<grid, LOGIT_THREADS, smem, s>>>(p);
@@ -1172,10 +1321,13 @@ RoutePlan route_plan(const moe_config &c)
     r.k_blocks = (int)ceil_div(c.d, rtc::BK);
     const int m_tiles = (int)ceil_div(c.T, rtc::BM);
     // One kernel up to 64 experts when a block's K part of the split weights
-    // (3 E_pad rows x 128 bytes per K block) stays resident in shared memory:
-    // K split in P = 4 parts (or 2, 1 for short K), at least 4 K blocks each.
+    // (3 E_pad rows, padded to a multiple of 16, x 128 bytes per K block;
+    // E_pad = 8 up to 8 experts, else E rounded up to 16) stays resident in
+    // shared memory: K split in P = 4 parts (or 2, 1 for short K), at least 4
+    // K blocks each.
     if (c.E <= 64) {
-        const int E_pad = c.E <= 16 ? 16 : (int)align_up((size_t)c.E, 16);
+        const int E_pad = c.E <= 8 ? 8 : (int)align_up((size_t)c.E, 16);
+        const int N3 = (3 * E_pad + 15) / 16 * 16;
         int P = 4;
         while (P > 1 && (r.k_blocks % P != 0 || r.k_blocks / P < 4))
             P /= 2;
@@ -1183,7 +1335,7 @@ RoutePlan route_plan(const moe_config &c)
         int stages = rtc::MAX_STAGES;
         while (stages > 2 && rtc::route_smem(E_pad, kbp, stages).total > 227 * 1024)
             --stages;
-        if (kbp * 3 * E_pad * 128 <= rtc::W_MAX_BYTES &&
+        if (kbp * N3 * 128 <= rtc::W_MAX_BYTES &&
             rtc::route_smem(E_pad, kbp, stages).total <= 227 * 1024) {
             r.fused = true;
             r.E_pad = E_pad;
@@ -1253,13 +1405,16 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
     p.k_blocks = r.k_blocks;
     p.status = status;
     p.clear_status = clear_status ? 1 : 0;
+    // a K part of W_r (kbp x 64 rows of E floats, contiguous) comes in by bulk
+    // copies when W_r is 16-byte aligned, else by per-thread loads
+    p.w_bulk = reinterpret_cast<uintptr_t>(W_r) % 16 == 0 ? 1 : 0;
     if (r.fused) {
         p.tiles = (int)ceil_div(c.T, BM);
         p.stages = r.stages;
         if (c.E <= 4)
-            return launch<16, 4, 1>(p, s);
+            return launch<8, 4, 1>(p, s);
         if (c.E <= 8)
-            return launch<16, 8, 1>(p, s);
+            return launch<8, 8, 1>(p, s);
         if (c.E <= 16)
             return launch<16, 0, 1>(p, s);
         if (c.E <= 32)

@@ -398,6 +398,27 @@ def test_route_selection_every_width(E, k, score):
     _check_route(1000, 256, E, k, score, E * 10 + k + score)
 
 
+@pytest.mark.parametrize("T,d,E,k", [(1000, 1024, 8, 2), (777, 512, 40, 3),
+                                     (16384, 1024, 64, 6), (500, 512, 100, 8)])
+def test_route_with_unaligned_router_weights_gives_the_same_bits(T, d, E, k):
+    """W_r 16-byte aligned (each block's K part copied in bulk) and W_r four
+    bytes off (per-thread loads) give the same top-k, gates, loss partials
+    and logits, bit for bit."""
+    g = torch.Generator(device=DEV).manual_seed(T + E)
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    W_r = torch.randn((d, E), generator=g, device=DEV) * 0.05
+    buf = torch.empty(d * E + 1, device=DEV)
+    W_off = buf[1:].view(d, E)
+    W_off.copy_(W_r)
+    assert W_r.data_ptr() % 16 == 0 and W_off.data_ptr() % 16 == 4
+    cfg = moe.moe_config(T=T, d=d, E=E, k=k, d_ff=64, dtype=1, cf=1.0)
+    a = moe.moe_route(cfg, x, W_r, want_logits=True)
+    b = moe.moe_route(cfg, x, W_off, want_logits=True)
+    torch.cuda.synchronize()
+    for u, v in zip(a[:4], b[:4]):
+        assert torch.equal(u, v)
+
+
 @pytest.mark.parametrize("T,d,E,k", [
     (1000, 1024, 4, 1),    # one kernel: 4 experts per token group, K in 4 parts (cluster of 4)
     (777, 512, 8, 2),      # 8 experts per token group, K in 2 parts
