@@ -698,7 +698,10 @@ def run_ours(args):
                 "algorithmic_bytes": ffn["algorithmic_bytes"],
                 "kernel": "moe_expert_ffn: grouped tcgen05 GEMM1 (act fused) + GEMM2",
                 "flops_per_launch": ffn["flops"],
-                "peak_source": f"{peak_src} bf16 {peak_kind} (MEASURED_PEAKS.json)",
+                "peak_source": (f"measured bf16 {peak_kind} (MEASURED_PEAKS.json)"
+                                if peak_src == "measured" else
+                                f"fallback bf16 {peak_kind}: MEASURED_PEAKS.json absent, the "
+                                "profiling recipe's figures"),
                 "timed_region_s": sm["timed_region_s"],
                 "frac_of_burst": round(ach / peaks["bf16_tflops"], 4),
                 "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4)}
