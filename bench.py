@@ -47,28 +47,11 @@ METRIC = "MoE layer fwd tokens/s on 1 B200; grouped-GEMM % BF16 peak; dispatch %
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20   # written between cold stage timings: twice the 126 MB L2
 def route_kernels(shape) -> int:
-    """Kernels of the router: bf16 layers with up to 64 experts whose split
-    router weights of a K part (3 x E padded rows, rounded up to a multiple of
-    16, x 64 x 2 bytes per K block; E padded to 8 up to 8 experts, else to a
-    multiple of 16) fit in shared memory run one kernel, wider ones three
-    (split, logits, select); the fp32 layer one."""
+    """Kernels of the router: bf16 layers with up to 16 experts run one kernel,
+    wider ones three (split, logits, select); the fp32 layer one."""
     if shape.dtype != 1:
         return 1
-    if shape.E <= 64:
-        ne = 8 if shape.E <= 8 else (shape.E + 15) // 16 * 16
-        n3 = (3 * ne + 15) // 16 * 16
-        kb = shape.d // 64
-        p = 4
-        while p > 1 and (kb % p or kb // p < 4):
-            p //= 2
-        kbp = kb // p
-        w = kbp * n3 * 128
-        # the fewest x stages the kernel runs with (it takes up to 8 as room allows)
-        total = (w + 1023) // 1024 * 1024 + 2 * 16384 + 2 * 128 * (ne + 4) * 4 + \
-            max(8 * (ne + 1), 32 * 9) * 4 + 1024
-        if w <= 112 * 1024 and total <= 227 * 1024:
-            return 1
-    return 3
+    return 1 if shape.E <= 16 else 3
 
 
 def kernels_per_step(shape) -> int:
@@ -88,7 +71,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of the same workload, valid only for the GEMM source it was taken on.
 GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_54_b200", "csrc", "ffn_tcgen05.cu")
 MEASURED_TRAFFIC = {
-    ("mixtral", "872c0a36b644350c28d3aa0b8c0abd44d4e57e623453bff990cab6d72699abde"): 4.964e9,
+    ("mixtral", "2672a43efa7fa1986e967ab95bf785cfbe76a776dc5d64b52997fef08a675984"): 5.612e9,
 }
 
 

@@ -71,14 +71,13 @@ int route_blocks(const moe_config &c);   // blocks of the tiled route kernel
 int partial_rows(const moe_config &c);   // rows of the loss partials, ceil(T / 32)
 int cap_blocks(const moe_config &c);
 
-// Tensor-core router layout (bf16 layers).  Fused (E <= 64 and the split
-// weights of a K part fit in shared memory): one persistent kernel, clusters
-// of k_parts blocks walking 128-token tiles.  Otherwise three launches:
+// Tensor-core router layout (bf16 layers).  Fused (E <= 16): one kernel, a
+// cluster of k_parts blocks per 128-token tile.  Otherwise three launches:
 // experts padded to E_pad in n_chunks chunks of n_chunk, K (k_blocks of 64)
 // split in k_parts of kb_per_part, through scratch.
 struct RoutePlan {
     bool tensor_cores, fused;
-    int E_pad, n_chunk, n_chunks, k_blocks, k_parts, kb_per_part, cluster, blocks, stages;
+    int E_pad, n_chunk, n_chunks, k_blocks, k_parts, kb_per_part, cluster, blocks;
 };
 RoutePlan route_plan(const moe_config &c);
 size_t route_scratch_bytes(const moe_config &c);

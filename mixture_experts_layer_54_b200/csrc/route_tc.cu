@@ -12,15 +12,14 @@
 //     z = x W_hi + x W_mid + x W_lo
 // in fp32 is the fp32 router.
 //
-// Up to 64 experts: one persistent kernel (details at route_kernel).  The
-// blocks of a thread-block cluster split K; each splits its part of W_r into
-// the three terms once, keeps them in shared memory as the MMA's B operand
-// (hi, mid and lo stacked as 3 E_pad rows, so one MMA per K step gives the
-// three products side by side in TMEM), and streams 128-token x tiles by TMA
-// through a double-buffered TMEM accumulator.  Each block then selects its
-// share of a tile's tokens, summing the K parts' partial logits in order
-// through distributed shared memory: softmax or sigmoid, top-k (ties to the
-// lower index), gates, optional logits/scores, and the rows of the loss
+// Up to 16 experts: one kernel (details at route_kernel).  The blocks of a
+// thread-block cluster split K for one 128-token tile; each splits its part of
+// W_r into the three terms stage by stage as the tile's x streams (hi, mid and
+// lo stacked as 3 x 16 rows of the MMA's B operand, so one MMA per K step
+// gives the three products side by side in TMEM).  Each block then selects
+// its share of the tile's tokens, summing the K parts' partial logits in
+// order through distributed shared memory: softmax or sigmoid, top-k (ties to
+// the lower index), gates, optional logits/scores, and the rows of the loss
 // partials (32 tokens per row) in a fixed order.
 //
 // More experts: three launches (split once, logits, select), below.
@@ -34,8 +33,14 @@ namespace moe {
 namespace rtc {
 
 constexpr int BM = 128, BK = 64;
-constexpr int STAGES = 4;              // TMA ring of the three-launch logits kernel
+constexpr int THREADS = 512;   // one-kernel router: 16 warps, roles below, then all select
+constexpr int WARPS = THREADS / 32;
+constexpr int STAGES = 4;              // TMA ring of either kernel
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB: one x tile of a K block
+constexpr int CONV_WARP0 = 4;          // warps 4-7 split W_r, then read TMEM
+constexpr int COPY_WARP0 = 8;          // warps 8-11 copy W_r
+constexpr int CONV_LANES = 128;        // lanes of either role
+constexpr int MAX_CLUSTER = 4;
 
 // -------------------------------------------------------------- PTX helpers
 
@@ -108,16 +113,6 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile
     return bar_wait_t<false>(bar, parity, abort, status);
 }
 
-// The same wait for a whole warp: every lane polls, the warp agrees on the
-// outcome.  (Polling by lane 0 alone, the others waiting at a shuffle,
-// measured slower: 9.4 against 12.1 us for the Switch-shaped router.)
-template <bool CLUSTER>
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          int32_t *status)
-{
-    return __all_sync(0xffffffffu, bar_wait_t<CLUSTER>(bar, parity, abort, status));
-}
-
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t a)
 {
     return (uint64_t)((a & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)64 << 32) |
@@ -152,6 +147,24 @@ __device__ __forceinline__ float ld_peer(uint32_t a)
     return v;
 }
 
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Arrives on the mbarrier once this thread's earlier cp.async copies land.
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // fp32 -> unsigned integer of the same order (-0 made +0; keys are never NaN),
 // and back: lets a warp take a max with one redux.sync instead of a shuffle
 // tree.
@@ -179,9 +192,7 @@ struct __align__(64) RouteParams {
     float *gates, *loss_partials, *logits_out, *scores_out;
     int T, d, E, k, score, renorm;
     int cs, k_parts, kb_per_part, k_blocks;
-    int tiles, nclusters, stages;   // one-kernel router: token tiles, clusters, x stages
     int clear_status;               // 1: block 0 clears the status word first
-    int w_bulk;                     // 1: W_r is 16-byte aligned (its K parts copied in bulk)
     int32_t *status;
 };
 
@@ -359,181 +370,63 @@ __device__ __forceinline__ void select_token(const SelArgs &a, bool renorm, int 
 }
 
 // ---------------------------------------------------------------- kernel
-//
-// One kernel for up to 64 experts.  The blocks of a cluster split K into P
-// parts (P = cluster size, 1, 2 or 4); block `rank` owns K blocks
-// [rank kbp, (rank + 1) kbp).  The cluster walks token tiles of 128
-// (tile = cluster, cluster + clusters, ...), so one cluster may take several.
-//   prologue     warps 2-13 split this block's K part of W_r into the three
-//                bf16 terms, K-major in the 128-byte swizzle, once (all of a
-//                thread's loads issued before any conversion): the B operand
-//                of every tile stays in shared memory;
-//   warp 0       TMA ring of x tiles (one thread), as deep as shared memory
-//                allows;
-//   warp 1       one MMA of N = 3 NE per K step of 16 into one of two TMEM
-//                accumulators (tile i uses buffer i mod 2);
-//   warps 2-5    read an accumulator back (hi + (mid + lo)) and push each
-//                token's partial logits into buffer i mod 2 of the block that
-//                selects that token (st.async, slot = this block's K part):
-//                each store's bytes count on that block's lfull barrier, so
-//                no fence or remote arrive follows the pushes;
-//   warps 6-13   select 128 / P tokens of the tile from their own buffer once
-//                its BM x NE floats have landed, summing the P parts in part
-//                order; then arm the buffer's barrier for its next use and
-//                tell every block that the buffer may be filled again.
-// So one tile's read-back and selection run while the next tile's x streams,
-// and no warp waits on a remote load.
 
-constexpr int PR_THREADS = 448;   // 14 warps
-constexpr int RB_WARP0 = 2;       // warps 2-5: TMEM read-back
-constexpr int SEL_WARP0 = 6;      // warps 6-13: selection
-constexpr int SEL_WARPS = 8;
-constexpr int SEL_THREADS = SEL_WARPS * 32;
-static_assert(RB_WARP0 == 2 && SEL_WARP0 == RB_WARP0 + 4, "warps 0, 1: TMA, MMA; then 4 read-back");
-constexpr int CONV_WARP0 = 2;     // warps 2-13 split W_r first
-constexpr int CONV_THREADS = PR_THREADS - CONV_WARP0 * 32;
-constexpr int MAX_STAGES = 8;
-constexpr int W_MAX_BYTES = 112 * 1024;   // resident split weights per block
-
-// This warp's 32 TMEM lanes x 16 (or 8) consecutive fp32 columns from taddr.
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[16])
+// One 128-token tile per cluster of k_parts blocks (block `rank` owns K
+// blocks [rank kbp, (rank + 1) kbp)), two blocks per SM, 16 warps:
+//   warp 0       TMA ring of x tiles (4 stages, one thread);
+//   warp 1       one MMA of N = 3 x 16 per K step of 16 into TMEM;
+//   warps 8-11   copy each stage's fp32 W_r slice into a staging slot
+//                (4-byte cp.async, arriving on the stage's barrier when landed);
+//   warps 4-7    split the staged slice into the three bf16 terms (128-byte
+//                swizzle, the stage's B operand), then read the accumulator
+//                back (hi + (mid + lo)) into the block's partial-logit tile;
+//   all 16       after a cluster barrier, select the block's 128 / P tokens,
+//                summing the P partial tiles in part order (ld.shared::cluster).
+// So W_r is split while x streams, and the stage ring is the only pipeline.
+// N: experts per block (launched with 16).  Selection: E_T > 0 takes E <= E_T
+// experts with E_T lanes per token (32 / E_T tokens per warp at once); E_T == 0
+// takes a warp per token with PL experts per lane.
+template <int N, int E_T, int PL>
+__global__ void __launch_bounds__(THREADS, N <= 16 ? 2 : 1)
+    route_kernel(const __grid_constant__ RouteParams p)
 {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[8])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                   "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-}
-
-// Asynchronous store of four floats to shared memory of a block of the
-// cluster (a and bar are cluster shared addresses of that block): when the 16
-// bytes have landed they count against the transaction bytes the block's
-// mbarrier bar expects, so the reader needs no fence or arrive from the writer.
-__device__ __forceinline__ void st_async4(uint32_t a, float4 v, uint32_t bar)
-{
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
-        "[%5];" ::"r"(a),
-        "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
-        : "memory");
-}
-
-// Arrive on a barrier of this block, first raising the transaction bytes its
-// current phase waits for.
-__device__ __forceinline__ void arrive_expect(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-// Named barriers (id 0 is __syncthreads).
-__device__ __forceinline__ void named_sync(int id, int threads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// Arrive on the mbarrier at the same shared offset in block `rank` of the
-// cluster, with no memory ordering: a bare "go" signal.
-__device__ __forceinline__ void arrive_remote_relaxed(uint32_t bar, uint32_t rank)
-{
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                     peer_addr(bar, rank))
-                 : "memory");
-}
-
-// Shared-memory plan of the kernel (host and device agree on it).
-struct RouteSmem {
-    int w, x, l, scratch, total;
-};
-__host__ __device__ inline RouteSmem route_smem(int NE, int kbp, int stages)
-{
-    RouteSmem s;
-    const int N3 = (3 * NE + 15) / 16 * 16;   // the MMA's N: hi, mid, lo rows, padded
-    s.w = 0;
-    s.x = (kbp * N3 * 128 + 1023) / 1024 * 1024;
-    s.l = s.x + stages * A_BYTES;
-    const int l_bytes = BM * (NE + 4) * 4;
-    s.scratch = s.l + 2 * l_bytes;
-    // selection sums: a row per selection warp, or (E <= 8) up to 32 groups of 9
-    const int sc = SEL_WARPS * (NE + 1) > 32 * 9 ? SEL_WARPS * (NE + 1) : 32 * 9;
-    s.total = s.scratch + sc * 4 + 1024;   // + alignment slack
-    return s;
-}
-
-// NE: experts per MMA (E padded to 8, 16, 32, 48 or 64).  Selection: E_T > 0
-// (NE = 8) takes E <= E_T experts with E_T lanes per token (32 / E_T tokens per
-// warp at once); E_T == 0 takes a warp per token with NE / 32 (rounded up)
-// experts per lane, four tokens per warp at once.
-template <int NE, int E_T>
-__global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_constant__ RouteParams p)
-{
-    constexpr int N3 = (3 * NE + 15) / 16 * 16;      // hi, mid, lo rows of B (+ zero rows)
-    constexpr int WT_BYTES = N3 * 128;               // one K block of B
-    constexpr uint32_t ACC = N3 <= 64 ? 64 : (N3 <= 128 ? 128 : 256);   // columns per buffer
-    constexpr uint32_t TMEM_COLS = 2 * ACC;
+    constexpr int B_BYTES = N * BK * 2;   // one bf16 term of the W slice
+    constexpr int STAGE = A_BYTES + 3 * B_BYTES;
+    constexpr int RAW = BK * N * 4;        // fp32 W_r slice of a stage, as staged
+    constexpr int N3 = 3 * N;   // hi, mid, lo rows of the B operand
+    constexpr uint32_t TMEM_COLS = N3 <= 64 ? 64 : (N3 <= 128 ? 128 : 256);   // power of two
     constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N3 >> 3) << 17) |
                                ((uint32_t)(BM >> 4) << 24);
-    constexpr int LS = NE + 4;                       // row stride (floats) of a logit buffer
+    constexpr int LS = N + 4;   // row stride (floats) of the partial-logit tile
     constexpr int L_BYTES = BM * LS * 4;
-    constexpr int L_PUSH = BM * NE * 4;              // bytes pushed into a buffer per tile
-    static_assert(N3 % 16 == 0 && N3 <= 256, "MMA N");
-    static_assert(NE == 8 || NE % 16 == 0, "experts per MMA: 8 or a multiple of 16");
-    static_assert((E_T > 0) == (NE == 8), "narrow selection exactly on the 8-expert layout");
-    constexpr int PL = (NE + 31) / 32;               // experts per lane, a warp per token
+    constexpr int CPL = N * 8 / CONV_LANES;   // 16-byte W chunks per converter lane per stage
+    static_assert(N * 8 % CONV_LANES == 0, "chunk split");
+    static_assert(L_BYTES + WARPS * (kMaxE + 1) * 4 <= STAGES * STAGE, "select scratch");
+    static_assert(STAGES * (STAGE + RAW) + 1024 <= 227 * 1024, "shared memory");
+    static_assert(COPY_WARP0 + CONV_LANES / 32 <= WARPS, "roles");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], wready, wbar, tfull[2],
-        tempty[2], lfull[2], lempty[2], drain;
+    __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], wfull[STAGES], done;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
-    // Set by a read-back (selection) warp whose bounded wait gave up, read by
-    // its whole group after a named barrier, so the group leaves its loop
-    // together and no warp waits at a named barrier for one that left.
-    __shared__ int rb_fail, sel_fail;
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int P = p.cs, ST = p.stages;
     const int rank = (int)cluster_rank();
-    const int cl = blockIdx.x / P, ncl = p.nclusters;
-    const int kbp = p.kb_per_part, kb0 = rank * kbp;
-    const RouteSmem sm = route_smem(NE, kbp, ST);
-    uint8_t *Wres = smem + sm.w;
-    uint8_t *X = smem + sm.x;
-    const uint32_t lbase = saddr(smem + sm.l);
-    const int TPC = BM / P;   // tokens of a tile this block selects (128, 64 or 32)
+    const int chunk = rank / p.k_parts, part = rank % p.k_parts;
+    const int m0 = (blockIdx.x / p.cs) * BM, n0 = chunk * N;
+    const int kb0 = part * p.kb_per_part;
+    const int kb1 = min(kb0 + p.kb_per_part, p.k_blocks);
+    const int nk = kb1 > kb0 ? kb1 - kb0 : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < ST; ++s) {
-            bar_init(saddr(&full[s]), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            bar_init(saddr(&full[s]), 1 + CONV_LANES / 32);
             bar_init(saddr(&empty[s]), 1);
+            bar_init(saddr(&wfull[s]), CONV_LANES);
         }
-        bar_init(saddr(&wready), CONV_THREADS / 32);
-        bar_init(saddr(&wbar), 1);
-        for (int a = 0; a < 2; ++a) {
-            bar_init(saddr(&tfull[a]), 1);
-            bar_init(saddr(&tempty[a]), 4);
-            // a phase of lfull[a]: this block's own arrive, which also sets the
-            // bytes the cluster's read-back pushes into buffer a (BM rows of NE
-            // floats: TPC rows from each of the P blocks)
-            bar_init(saddr(&lfull[a]), 1);
-            bar_init(saddr(&lempty[a]), (uint32_t)P);
-        }
-        bar_init(saddr(&drain), 1);
+        bar_init(saddr(&done), 1);
         abort_flag = 0;
-        rb_fail = 0;
-        sel_fail = 0;
-        for (int a = 0; a < 2; ++a)   // the first use of each buffer
-            arrive_expect(saddr(&lfull[a]), (uint32_t)L_PUSH);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -544,267 +437,274 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    cluster_sync();   // every block's barriers exist before anyone arrives remotely
+    __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tmem_slot;
-
     // inputs (x, W_r, biases) may come from the previous kernel in the stream
     pdl_wait();
     pdl_trigger();
     if (p.clear_status && blockIdx.x == 0 && threadIdx.x == 0)
         *p.status = 0;
 
-    if (warp >= CONV_WARP0) {
-        // ---- prologue: this block's K part of W_r -> three bf16 terms ----
-        // Chunk c = (K block i, 8-wide K group j, expert e < E), e fastest;
-        // its 16 bytes of each term go to row e (+ NE, + 2 NE) of K block i's
-        // tile, at position j ^ (row & 7) of the row's eight (128-byte
-        // swizzle).  The part (kbp x 64 rows of E floats, contiguous in W_r)
-        // arrives by bulk copies into the tail of the split-weight region,
-        // issued by the TMA thread ahead of any x tile; every thread reads all
-        // of its chunks (at most CB: 8 kbp E <= 8 kbp NE <= CB x 384 on every
-        // layer this kernel takes) before any thread writes a term over the
-        // staged part.  Without 16-byte alignment the threads load the part
-        // from global memory themselves.
-        constexpr int CB = 6;
-        const int ct = threadIdx.x - CONV_WARP0 * 32;
-        const int E = p.E, nchunk = kbp * 8 * E;
-        const float *stage =
-            reinterpret_cast<const float *>(Wres + kbp * WT_BYTES - kbp * BK * E * 4);
-        if (p.w_bulk)   // expiry: recorded, go on
-            warp_wait<false>(saddr(&wbar), 0, &abort_flag, p.status);
-        float w[CB][8];
-#pragma unroll
-        for (int b = 0; b < CB; ++b) {
-            const int c = ct + b * CONV_THREADS;
-            const int e = c % E, j = (c / E) % 8, i = c / (E * 8);
-            const int r0 = i * BK + 8 * j;   // row of the part
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                w[b][u] = c >= nchunk ? 0.f
-                          : p.w_bulk  ? stage[(r0 + u) * E + e]
-                                      : p.W_r[((int64_t)kb0 * BK + r0 + u) * E + e];
-        }
-        named_sync(3, CONV_THREADS);   // the staged part is read: terms may overwrite it
-#pragma unroll
-        for (int b = 0; b < CB; ++b) {
-            const int c = ct + b * CONV_THREADS;
-            if (c >= nchunk)
-                break;
-            const int e = c % E, j = (c / E) % 8, i = c / (E * 8);
-            uint32_t hi[4], mid[4], lo[4];
-#pragma unroll
-            for (int u = 0; u < 8; u += 2) {
-                __nv_bfloat16 h[2], md[2], l[2];
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const float x = w[b][u + r];
-                    h[r] = __float2bfloat16_rn(x);
-                    const float r1 = x - __bfloat162float(h[r]);
-                    md[r] = __float2bfloat16_rn(r1);
-                    l[r] = __float2bfloat16_rn(r1 - __bfloat162float(md[r]));
-                }
-                hi[u / 2] = pack2(h[0], h[1]);
-                mid[u / 2] = pack2(md[0], md[1]);
-                lo[u / 2] = pack2(l[0], l[1]);
-            }
-            uint8_t *tile = Wres + i * WT_BYTES;
-            const uint32_t *terms[3] = {hi, mid, lo};
-#pragma unroll
-            for (int sp = 0; sp < 3; ++sp) {
-                const int row = sp * NE + e;
-                *reinterpret_cast<uint4 *>(tile + row * 128 + ((j ^ (row & 7)) << 4)) =
-                    make_uint4(terms[sp][0], terms[sp][1], terms[sp][2], terms[sp][3]);
-            }
-        }
-        // zero rows: the padding experts E .. NE - 1 of every term, and the
-        // rows 3 NE .. N3 - 1 that round the MMA's N up to a multiple of 16
-        const int dead = NE - E, zrows = 3 * dead + (N3 - 3 * NE), nz = kbp * zrows * 8;
-        for (int z = ct; z < nz; z += CONV_THREADS) {
-            const int q16 = z % 8, zr = (z / 8) % zrows, i = z / (8 * zrows);
-            const int row = zr < 3 * dead ? (zr / dead) * NE + E + zr % dead : 3 * NE + zr - 3 * dead;
-            *reinterpret_cast<uint4 *>(Wres + i * WT_BYTES + row * 128 + q16 * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-        }
-        // generic-proxy stores, read next by the tensor core (async proxy)
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0)
-            bar_arrive(saddr(&wready));
-    }
-
     if (warp == 0) {
         if (lane == 0) {
-            // ---- TMA producer: the x tile of every K block of every tile ----
-            int it = 0;
-            int last_issue[MAX_STAGES];
-            for (int s = 0; s < MAX_STAGES; ++s)
+            // ---- TMA producer: the x tile of each K block ----
+            int last_issue[STAGES];
+            for (int s = 0; s < STAGES; ++s)
                 last_issue[s] = -1;
-            // this block's K part of W_r first, in pieces of up to 16 KB
-            const uint32_t wbytes = (uint32_t)(kbp * BK * p.E * 4);
-            if (p.w_bulk) {
-                const uint32_t wb = saddr(&wbar);
-                const uint32_t dst = saddr(Wres + kbp * WT_BYTES) - wbytes;
-                const char *src = reinterpret_cast<const char *>(p.W_r + (int64_t)kb0 * BK * p.E);
-                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(wb),
-                             "r"(wbytes)
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % STAGES;
+                if (i >= STAGES && !bar_wait(saddr(&empty[s]), (uint32_t)(((i / STAGES) - 1) & 1),
+                                             &abort_flag, p.status))
+                    break;
+                const uint32_t fb = saddr(&full[s]);
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb),
+                             "r"(A_BYTES)
                              : "memory");
-                for (uint32_t o = 0; o < wbytes; o += 16384) {
-                    const uint32_t n = wbytes - o < 16384 ? wbytes - o : 16384;
-                    asm volatile(
-                        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], "
-                        "%2, [%3];" ::"r"(dst + o),
-                        "l"(src + o), "r"(n), "r"(wb)
-                        : "memory");
-                }
-            }
-            // x waits until the terms are written: issued together, the whole
-            // grid's first x tiles (stages x 16 KB per block) would share the
-            // memory system with W_r, and the converters' proxy fence would
-            // wait for them to land
-            bool ok = bar_wait(saddr(&wready), 0, &abort_flag, p.status);
-            for (int tile = cl; ok && tile < p.tiles; tile += ncl) {
-                for (int i = 0; i < kbp; ++i, ++it) {
-                    const int s = it % ST;
-                    if (it >= ST && !bar_wait(saddr(&empty[s]), (uint32_t)(((it / ST) - 1) & 1),
-                                              &abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = saddr(&full[s]);
-                    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb),
-                                 "r"(A_BYTES)
-                                 : "memory");
-                    asm volatile(
-                        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::"
-                        "bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(saddr(X + s * A_BYTES)),
-                        "l"(reinterpret_cast<uint64_t>(&p.tmX)), "r"((kb0 + i) * BK),
-                        "r"(tile * BM), "r"(0), "r"(fb)
-                        : "memory");
-                    last_issue[s] = it;
-                }
+                asm volatile(
+                    "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                    " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(saddr(smem + s * STAGE)),
+                    "l"(reinterpret_cast<uint64_t>(&p.tmX)), "r"((kb0 + i) * BK), "r"(m0), "r"(0),
+                    "r"(fb)
+                    : "memory");
+                last_issue[s] = i;
             }
             // copies in flight land before the block moves on (bounded)
-            if (p.w_bulk)
-                bar_wait(saddr(&wbar), 0, nullptr, nullptr);
-            for (int s = 0; s < ST; ++s)
+            for (int s = 0; s < STAGES; ++s)
                 if (last_issue[s] >= 0)
-                    bar_wait(saddr(&full[s]), (uint32_t)((last_issue[s] / ST) & 1), nullptr,
+                    bar_wait(saddr(&full[s]), (uint32_t)((last_issue[s] / STAGES) & 1), nullptr,
                              nullptr);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ---- MMA issuer ----
-            bool ok = bar_wait(saddr(&wready), 0, &abort_flag, p.status);
+            // ---- MMA issuer: one bf16 MMA of N = 3 x chunk per K step of 16 ----
             bool any = false;
-            int it = 0, tc = 0;
-            for (int tile = cl; ok && tile < p.tiles; tile += ncl, ++tc) {
-                const int a = tc & 1;
-                if (!bar_wait(saddr(&tempty[a]), (uint32_t)(((tc >> 1) & 1) ^ 1), &abort_flag,
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % STAGES;
+                if (!bar_wait(saddr(&full[s]), (uint32_t)((i / STAGES) & 1), &abort_flag,
                               p.status))
                     break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint32_t d = tmem + (uint32_t)a * ACC;
-                for (int i = 0; i < kbp; ++i, ++it) {
-                    const int s = it % ST;
-                    if (!bar_wait(saddr(&full[s]), (uint32_t)((it / ST) & 1), &abort_flag,
-                                  p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                    const uint32_t xa = saddr(X + s * A_BYTES), wb = saddr(Wres + i * WT_BYTES);
+                const uint32_t a = saddr(smem + s * STAGE);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
-                        asm volatile(
-                            "{\n\t.reg .pred q;\n\t"
-                            "setp.ne.b32 q, %4, 0;\n\t"
-                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, q;\n\t}" ::"r"(d),
-                            "l"(sdesc_sw128(xa + kk * 32)), "l"(sdesc_sw128(wb + kk * 32)),
-                            "r"(IDESC), "r"(acc)
-                            : "memory");
-                    }
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
                     asm volatile(
-                        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-                        "[%0];" ::"r"(saddr(&empty[s]))
+                        "{\n\t.reg .pred q;\n\t"
+                        "setp.ne.b32 q, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, q;\n\t}" ::"r"(tmem),
+                        "l"(sdesc_sw128(a + kk * 32)), "l"(sdesc_sw128(a + A_BYTES + kk * 32)),
+                        "r"(IDESC), "r"(acc)
                         : "memory");
-                    any = true;
                 }
-                if (!ok)
-                    break;
                 asm volatile(
                     "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-                    "[%0];" ::"r"(saddr(&tfull[a]))
+                    "[%0];" ::"r"(saddr(&empty[s]))
                     : "memory");
+                any = true;
             }
-            if (any) {   // every MMA issued has completed before TMEM is freed
+            if (any)
                 asm volatile(
                     "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-                    "[%0];" ::"r"(saddr(&drain))
+                    "[%0];" ::"r"(saddr(&done))
                     : "memory");
-                bar_wait(saddr(&drain), 0, nullptr, p.status);
-            }
+            else
+                bar_arrive(saddr(&done));
         }
-    } else if (warp < SEL_WARP0) {
-        // ---- accumulator -> this block's partial-logit buffer ----
-        const int q = warp & 3;   // TMEM lanes 32 q .. 32 q + 31
-        int tc = 0;
-        for (int tile = cl; tile < p.tiles; tile += ncl, ++tc) {
-            const int a = tc & 1, n = tc >> 1;
-            bool okw = warp_wait<false>(saddr(&tfull[a]), (uint32_t)(n & 1), &abort_flag, p.status);
-            // the cluster's selection of the tile that last used this buffer is done
-            if (okw)
-                okw = warp_wait<false>(saddr(&lempty[a]), (uint32_t)((n & 1) ^ 1), &abort_flag,
-                                       p.status);
-            if (!okw && lane == 0)
-                rb_fail = 1;
-            named_sync(1, 128);
-            if (rb_fail)
-                break;
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            // this lane's token row goes to the block selecting it, slot
-            // `rank`; the owner's lfull[a] counts the bytes as they land
-            const int row = q * 32 + lane, owner = row / TPC, tl = row % TPC;
-            const uint32_t dst = peer_addr(lbase, (uint32_t)owner) +
-                                 (uint32_t)(a * L_BYTES + (rank * TPC + tl) * LS * 4);
-            const uint32_t dbar = peer_addr(saddr(&lfull[a]), (uint32_t)owner);
-            const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)a * ACC;
-            constexpr int CW = NE < 16 ? NE : 16;   // columns per load and term
+    } else if (warp >= COPY_WARP0 && warp < COPY_WARP0 + CONV_LANES / 32) {
+        // ---- W_r slice of each K block -> staging slot, 4-byte cp.async ----
+        // Lane cl stages the 8 K values of its chunks c = cl + 128 u, where
+        // chunk c = (expert row el = c % N, 8-wide K group j = c / N); value q
+        // of chunk u sits at (8 u + q) x 128 + cl, so a warp's copies fill
+        // consecutive words.
+        const int cl = threadIdx.x - COPY_WARP0 * 32;
+        float *raw = reinterpret_cast<float *>(smem + STAGES * STAGE);
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % STAGES;
+            if (i >= STAGES) {
+                int ok = 0;
+                if (lane == 0)
+                    ok = bar_wait(saddr(&empty[s]), (uint32_t)(((i / STAGES) - 1) & 1),
+                                  &abort_flag, p.status);
+                if (!__shfl_sync(0xffffffffu, ok, 0))
+                    break;
+            }
+            const int kc = (kb0 + i) * BK;
+            float *dst = raw + s * (RAW / 4);
 #pragma unroll
-            for (int c = 0; c < NE; c += CW) {
-                uint32_t r[3][CW];
+            for (int u = 0; u < CPL; ++u) {
+                const int c = cl + CONV_LANES * u;
+                const int el = c % N, j = c / N;
+                const int e = n0 + el;
+                if (e < p.E) {
+                    const float *src = p.W_r + (int64_t)(kc + 8 * j) * p.E + e;
 #pragma unroll
-                for (int sp = 0; sp < 3; ++sp)
-                    tmem_ld_cols(tb + (uint32_t)(sp * NE + c), r[sp]);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-                for (int h = 0; h < CW; h += 4) {
-                    float v[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)   // x W_hi + (x W_mid + x W_lo)
-                        v[u] = __uint_as_float(r[0][h + u]) +
-                               (__uint_as_float(r[1][h + u]) + __uint_as_float(r[2][h + u]));
-                    st_async4(dst + (uint32_t)((c + h) * 4), make_float4(v[0], v[1], v[2], v[3]),
-                              dbar);
+                    for (int q = 0; q < 8; ++q)
+                        cp_async4(saddr(dst + (u * 8 + q) * CONV_LANES + cl),
+                                  src + (int64_t)q * p.E);
                 }
             }
-            // accumulator free for the tile after next
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            cp_async_arrive(saddr(&wfull[s]));
+        }
+        cp_async_wait_all();
+    } else if (warp >= CONV_WARP0 && warp < CONV_WARP0 + CONV_LANES / 32) {
+        // ---- staged W_r slice -> three bf16 terms, 128-byte swizzle ----
+        // Chunk c's 16 bytes sit at row el, position j ^ (el & 7) of the
+        // row's eight.  A stage's staging slot is complete once wfull fires,
+        // which also means the MMA reading the slot's previous B tiles is done
+        // (the copies waited for it).
+        const int cl = threadIdx.x - CONV_WARP0 * 32;
+        const float *raw = reinterpret_cast<const float *>(smem + STAGES * STAGE);
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % STAGES;
+            if (!__all_sync(0xffffffffu, bar_wait(saddr(&wfull[s]), (uint32_t)((i / STAGES) & 1),
+                                                  &abort_flag, p.status)))
+                break;
+            uint8_t *b = smem + s * STAGE + A_BYTES;
+            const float *src = raw + s * (RAW / 4);
+#pragma unroll
+            for (int u = 0; u < CPL; ++u) {
+                const int c = cl + CONV_LANES * u;
+                const int el = c % N, j = c / N;
+                float w[8];
+                const bool live = n0 + el < p.E;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    w[q] = live ? src[(u * 8 + q) * CONV_LANES + cl] : 0.f;
+                uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+                for (int q = 0; q < 8; q += 2) {
+                    __nv_bfloat16 h[2], md[2], l[2];
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const float x = w[q + r];
+                        h[r] = __float2bfloat16_rn(x);
+                        const float r1 = x - __bfloat162float(h[r]);
+                        md[r] = __float2bfloat16_rn(r1);
+                        l[r] = __float2bfloat16_rn(r1 - __bfloat162float(md[r]));
+                    }
+                    hi[q / 2] = pack2(h[0], h[1]);
+                    mid[q / 2] = pack2(md[0], md[1]);
+                    lo[q / 2] = pack2(l[0], l[1]);
+                }
+                const int off = el * 128 + ((j ^ (el & 7)) << 4);
+                *reinterpret_cast<uint4 *>(b + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(b + B_BYTES + off) =
+                    make_uint4(mid[0], mid[1], mid[2], mid[3]);
+                *reinterpret_cast<uint4 *>(b + 2 * B_BYTES + off) =
+                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            // generic-proxy stores, read next by the tensor core (async proxy)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0)
-                bar_arrive(saddr(&tempty[a]));
+                bar_arrive(saddr(&full[s]));
+        }
+
+        // ---- accumulator rows -> fp32 partial-logit tile (reuses the ring) ----
+        const int ew = warp - CONV_WARP0;   // TMEM lanes 32 ew .. 32 ew + 31
+        const bool ok = bar_wait(saddr(&done), 0, nullptr, p.status) && !abort_flag;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        float *L = reinterpret_cast<float *>(smem) + (ew * 32 + lane) * LS;
+#pragma unroll
+        for (int c = 0; c < N; c += 16) {
+            uint32_t r[3][16];
+            if (nk > 0) {
+#pragma unroll
+                for (int sp = 0; sp < 3; ++sp)
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
+                        "[%16];"
+                        : "=r"(r[sp][0]), "=r"(r[sp][1]), "=r"(r[sp][2]), "=r"(r[sp][3]),
+                          "=r"(r[sp][4]), "=r"(r[sp][5]), "=r"(r[sp][6]), "=r"(r[sp][7]),
+                          "=r"(r[sp][8]), "=r"(r[sp][9]), "=r"(r[sp][10]), "=r"(r[sp][11]),
+                          "=r"(r[sp][12]), "=r"(r[sp][13]), "=r"(r[sp][14]), "=r"(r[sp][15])
+                        : "r"(tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(sp * N + c)));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            }
+#pragma unroll
+            for (int q = 0; q < 16; q += 4) {
+                float v[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    // x W_hi + (x W_mid + x W_lo)
+                    const float z = __uint_as_float(r[0][q + h]) +
+                                    (__uint_as_float(r[1][q + h]) + __uint_as_float(r[2][q + h]));
+                    v[h] = nk == 0 ? 0.f : (ok ? z : NAN);
+                }
+                *reinterpret_cast<float4 *>(L + c + q) = make_float4(v[0], v[1], v[2], v[3]);
+            }
+        }
+    }
+    __syncwarp();
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    cluster_sync();   // every block's partial-logit tile is written
+    if (warp == 1) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+
+    // ---- selection: this block's share of the tile's tokens ----
+    const int TPC = BM / p.cs;                // 128, 64 or 32 tokens
+    const int tl0 = rank * TPC;               // first token of the share, within the tile
+    const int row0 = (m0 + tl0) / kPartialTokens;
+    const bool renorm = p.renorm < 0 ? (p.k > 1) : (p.renorm != 0);
+    const uint32_t lbase = saddr(smem);
+    uint32_t rb[MAX_CLUSTER];
+#pragma unroll
+    for (int q = 0; q < MAX_CLUSTER; ++q)
+        rb[q] = q < p.cs ? peer_addr(lbase, (uint32_t)q) : 0u;
+    float *scratch = reinterpret_cast<float *>(smem + L_BYTES);
+    const int E = p.E;
+
+    if constexpr (E_T > 0) {
+        // a group = the 32 / E_T tokens one warp holds at once; E_T groups
+        // make a row of the loss partials
+        constexpr int TB = 32 / E_T;
+        const int groups = TPC / TB;
+        const int gl = lane % E_T;
+        RouteArgs ra{nullptr, nullptr, p.logit_bias, p.select_bias, p.topk, p.gates,
+                     p.loss_partials, p.logits_out, p.scores_out, p.T, 0, E, p.k, p.score,
+                     p.renorm};
+        // the biases of this lane's expert, loaded once
+        const float lbv = p.logit_bias && gl < E ? p.logit_bias[gl] : 0.f;
+        const float sbv = p.select_bias && gl < E ? p.select_bias[gl] : 0.f;
+        for (int g = warp; g < groups; g += WARPS) {
+            const int tg = tl0 + g * TB;
+            const int tl = tg + lane / E_T;
+            float z = -INFINITY;
+            if (m0 + tl < p.T && gl < E) {
+                z = 0.f;
+                for (int q = 0; q < p.k_parts; ++q)
+                    z += ld_peer(rb[q] + (uint32_t)(tl * LS + gl) * 4u);
+            }
+            float pc, zc;
+            small_epilogue<E_T>(ra, z, m0 + tg, lane, renorm, lbv, sbv, &pc, &zc);
+            if (lane < E_T)
+                scratch[g * (E_T + 1) + lane] = pc;
+            if (lane == 0)
+                scratch[g * (E_T + 1) + E_T] = zc;
+        }
+        __syncthreads();
+        const int rows = TPC / kPartialTokens;
+        for (int idx = threadIdx.x; idx < rows * (E + 1); idx += THREADS) {
+            const int r = idx / (E + 1), e = idx % (E + 1);
+            if ((int64_t)(row0 + r) * kPartialTokens >= p.T)
+                continue;
+            float acc = 0.f;
+            for (int w = 0; w < E_T; ++w)
+                acc += scratch[(r * E_T + w) * (E_T + 1) + (e < E ? e : E_T)];
+            p.loss_partials[(int64_t)(row0 + r) * (E + 1) + e] = acc;
         }
     } else {
-        // ---- selection: this block's share of every tile's tokens ----
-        // buffer a holds [part q][token tl of the share][expert]
-        const int st = threadIdx.x - SEL_WARP0 * 32;
-        const int E = p.E;
-        const int sw = warp - SEL_WARP0;   // selection warp 0..7
-        const int tl0 = rank * TPC;
-        const bool renorm = p.renorm < 0 ? (p.k > 1) : (p.renorm != 0);
+        // a warp per token: warp w takes tokens w, w + 16 of each row of 32;
+        // the row's sums meet in shared memory in warp order
+        float(*pw)[kMaxE + 1] = reinterpret_cast<float(*)[kMaxE + 1]>(scratch);
         const SelArgs sa = sel_args(p);
-        float *scratch = reinterpret_cast<float *>(smem + sm.scratch);
+        const int rows = TPC / kPartialTokens;
         float lb[PL], sb[PL];   // per-expert biases of this lane, loaded once
 #pragma unroll
         for (int i = 0; i < PL; ++i) {
@@ -812,135 +712,54 @@ __global__ void __launch_bounds__(PR_THREADS, 1) route_kernel(const __grid_const
             lb[i] = p.logit_bias && e < E ? p.logit_bias[e] : 0.f;
             sb[i] = p.select_bias && e < E ? p.select_bias[e] : 0.f;
         }
-        // narrow layers: lane L serves expert L % E_T
-        const int gle = E_T > 0 ? lane % (E_T > 0 ? E_T : 1) : 0;
-        const float lbv = E_T > 0 && p.logit_bias && gle < E ? p.logit_bias[gle] : 0.f;
-        const float sbv = E_T > 0 && p.select_bias && gle < E ? p.select_bias[gle] : 0.f;
-        int tc = 0;
-        for (int tile = cl; tile < p.tiles; tile += ncl, ++tc) {
-            const int a = tc & 1, n = tc >> 1;
-            const bool okw =
-                warp_wait<true>(saddr(&lfull[a]), (uint32_t)(n & 1), &abort_flag, p.status);
-            if (!okw && lane == 0)
-                sel_fail = 1;
-            named_sync(2, SEL_THREADS);
-            if (sel_fail)
-                break;
-            const int m0 = tile * BM;
-            const int row0 = (m0 + tl0) / kPartialTokens;
-            const int rows = TPC / kPartialTokens;
-            const float *Lb = reinterpret_cast<const float *>(smem + sm.l + a * L_BYTES);
-            if constexpr (E_T > 0) {
-                // a group = the 32 / E_T tokens one warp holds at once; E_T
-                // groups make a row of the loss partials
-                constexpr int TB = 32 / E_T;
-                const int groups = TPC / TB;
-                const int gl = lane % E_T;
-                RouteArgs ra{nullptr, nullptr, p.logit_bias, p.select_bias, p.topk, p.gates,
-                             p.loss_partials, p.logits_out, p.scores_out, p.T, 0, E, p.k,
-                             p.score, p.renorm};
-                for (int g = sw; g < groups; g += SEL_WARPS) {
-                    const int tg = tl0 + g * TB;
-                    const int tl = tg + lane / E_T;
-                    float z = -INFINITY;
-                    if (m0 + tl < p.T && gl < E) {
-                        z = 0.f;
-                        for (int q = 0; q < P; ++q)
-                            z += Lb[(q * TPC + tl - tl0) * LS + gl];
+        for (int r = 0; r < rows; ++r) {
+            float pacc[PL];
+#pragma unroll
+            for (int i = 0; i < PL; ++i)
+                pacc[i] = 0.f;
+            float zacc = 0.f;
+            for (int u = warp; u < kPartialTokens; u += WARPS) {
+                const int tl = tl0 + r * kPartialTokens + u;
+                const int t = m0 + tl;
+                if (t >= p.T)
+                    break;
+                float z[PL];
+#pragma unroll
+                for (int i = 0; i < PL; ++i) {
+                    const int e = lane + 32 * i;
+                    z[i] = -INFINITY;
+                    if (e < E) {
+                        const int ch = e / N, el = e - ch * N;
+                        float s = 0.f;
+                        for (int q = 0; q < p.k_parts; ++q)
+                            s += ld_peer(rb[ch * p.k_parts + q] + (uint32_t)(tl * LS + el) * 4u);
+                        if (p.logit_bias)
+                            s += lb[i];
+                        z[i] = s;
                     }
-                    float pc, zc;
-                    small_epilogue<E_T>(ra, z, m0 + tg, lane, renorm, lbv, sbv, &pc, &zc);
-                    if (lane < E_T)
-                        scratch[g * (E_T + 1) + lane] = pc;
-                    if (lane == 0)
-                        scratch[g * (E_T + 1) + E_T] = zc;
                 }
-                named_sync(2, SEL_THREADS);   // every group's sums are in scratch
-                for (int idx = st; idx < rows * (E + 1); idx += SEL_THREADS) {
-                    const int r = idx / (E + 1), e = idx % (E + 1);
-                    if ((int64_t)(row0 + r) * kPartialTokens >= p.T)
-                        continue;
+                select_token<PL, true>(sa, renorm, t, lane, z, sb, pacc, zacc);
+            }
+#pragma unroll
+            for (int i = 0; i < PL; ++i)
+                if (lane + 32 * i < E)
+                    pw[warp][lane + 32 * i] = pacc[i];
+            if (lane == 0)
+                pw[warp][E] = zacc;
+            __syncthreads();
+            if ((int64_t)(row0 + r) * kPartialTokens < p.T) {
+                float *out = p.loss_partials + (int64_t)(row0 + r) * (E + 1);
+                for (int e = threadIdx.x; e <= E; e += THREADS) {
                     float acc = 0.f;
-                    for (int w = 0; w < E_T; ++w)
-                        acc += scratch[(r * E_T + w) * (E_T + 1) + (e < E ? e : E_T)];
-                    p.loss_partials[(int64_t)(row0 + r) * (E + 1) + e] = acc;
-                }
-                named_sync(2, SEL_THREADS);   // scratch free, every read of the buffers done
-            } else {
-                // selection warp w takes tokens w, w + 8, w + 16 and w + 24 of
-                // each row of 32, all four at once, a whole warp per token; the
-                // row's sums meet in shared memory in warp order
-                for (int r = 0; r < rows; ++r) {
-                    float pacc[PL];
-#pragma unroll
-                    for (int i = 0; i < PL; ++i)
-                        pacc[i] = 0.f;
-                    float zacc = 0.f;
-                    // the warp's tokens of the row (sw, sw + 8, ...) at once
-                    constexpr int NT = kPartialTokens / SEL_WARPS;
-                    int tt[NT];
-                    bool tv[NT];
-                    float z[NT][PL];
-#pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        const int tl = tl0 + r * kPartialTokens + sw + n * SEL_WARPS;
-                        tt[n] = m0 + tl;
-                        tv[n] = tt[n] < p.T;
-#pragma unroll
-                        for (int i = 0; i < PL; ++i) {
-                            const int e = lane + 32 * i;
-                            float sum = 0.f;
-                            if (e < E && tv[n]) {
-                                for (int q = 0; q < P; ++q)
-                                    sum += Lb[(q * TPC + tl - tl0) * LS + e];
-                                if (p.logit_bias)
-                                    sum += lb[i];
-                            }
-                            z[n][i] = sum;
-                        }
-                    }
-                    select_tokens<PL, NT, true>(sa, renorm, tt, tv, lane, z, sb, pacc, zacc);
-#pragma unroll
-                    for (int i = 0; i < PL; ++i)
-                        if (lane + 32 * i < E)
-                            scratch[sw * (NE + 1) + lane + 32 * i] = pacc[i];
-                    if (lane == 0)
-                        scratch[sw * (NE + 1) + E] = zacc;
-                    named_sync(2, SEL_THREADS);
-                    if ((int64_t)(row0 + r) * kPartialTokens < p.T) {
-                        float *out = p.loss_partials + (int64_t)(row0 + r) * (E + 1);
-                        for (int e = st; e <= E; e += SEL_THREADS) {
-                            float acc = 0.f;
-                            for (int w = 0; w < SEL_WARPS; ++w)
-                                acc += scratch[w * (NE + 1) + e];
-                            out[e] = acc;
-                        }
-                    }
-                    named_sync(2, SEL_THREADS);
+                    for (int w = 0; w < WARPS; ++w)
+                        acc += pw[w][e];
+                    out[e] = acc;
                 }
             }
-            // this block is done reading buffer a: arm it for its next use,
-            // then let every block of the cluster push into it again
-            if (st == 0) {
-                arrive_expect(saddr(&lfull[a]), (uint32_t)L_PUSH);
-                // relaxed: every read of the buffer returned its value before
-                // the named barrier above, so later pushes cannot change them
-                for (int r = 0; r < P; ++r)
-                    arrive_remote_relaxed(saddr(&lempty[a]), (uint32_t)r);
-            }
+            __syncthreads();
         }
     }
-
-    // ---- tear-down: no block leaves while the cluster may read its buffers ----
-    __syncwarp();
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    cluster_sync();
-    if (warp == 1) {
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(TMEM_COLS)
-                     : "memory");
-    }
+    cluster_sync();   // the cluster's reads of this block's tile are done
 }
 
 // ======================================================= three-launch path
@@ -1267,34 +1086,23 @@ struct LaunchAttrs {
     }
 };
 
-template <int NE, int E_T>
-cudaError_t launch(RouteParams p, cudaStream_t s)
+template <int N, int E_T, int PL>
+cudaError_t launch(const RouteParams &p, unsigned grid, cudaStream_t s)
 {
-    auto kern = route_kernel<NE, E_T>;
-    const int smem = route_smem(NE, p.kb_per_part, p.stages).total;
+    constexpr int smem = STAGES * (A_BYTES + 3 * N * BK * 2 + BK * N * 4) + 1024;
+    auto kern = route_kernel<N, E_T, PL>;
     cudaError_t err = raise_smem_limit((const void *)kern, smem);
     if (err != cudaSuccess)
         return err;
-    // as many clusters as fit at once (every block must be resident: blocks of
-    // a cluster wait on one another), at most one per tile, the tiles spread
-    // evenly over them
-    int fit = 0;
-    err = cached_active_clusters((const void *)kern, PR_THREADS, smem, p.cs, &fit);
-    if (err != cudaSuccess)
-        return err;
-    if (fit < 1)
-        return cudaErrorInvalidConfiguration;
-    const int per = (int)ceil_div(p.tiles, fit);
-    p.nclusters = (int)ceil_div(p.tiles, per);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof cfg);
-    cfg.blockDim = dim3(PR_THREADS);
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cfg.gridDim = dim3((unsigned)(p.nclusters * p.cs));
-    LaunchAttrs lp(p.cs, true);
-    cfg.attrs = lp.at;
-    cfg.numAttrs = lp.n;
+    LaunchAttrs la(p.cs, true);   // cluster of the K parts; programmatic dependent launch
+    cfg.attrs = la.at;
+    cfg.numAttrs = la.n;
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -1318,34 +1126,27 @@ RoutePlan route_plan(const moe_config &c)
     r.tensor_cores = c.dtype == MOE_DTYPE_BF16 && c.d % rtc::BK == 0;
     r.k_blocks = (int)ceil_div(c.d, rtc::BK);
     const int m_tiles = (int)ceil_div(c.T, rtc::BM);
-    // One kernel up to 64 experts when a block's K part of the split weights
-    // (3 E_pad rows, padded to a multiple of 16, x 128 bytes per K block;
-    // E_pad = 8 up to 8 experts, else E rounded up to 16) stays resident in
-    // shared memory: K split in P = 4 parts (or 2, 1 for short K), at least 4
-    // K blocks each.
-    if (c.E <= 64) {
-        const int E_pad = c.E <= 8 ? 8 : (int)align_up((size_t)c.E, 16);
-        const int N3 = (3 * E_pad + 15) / 16 * 16;
-        int P = 4;
-        while (P > 1 && (r.k_blocks % P != 0 || r.k_blocks / P < 4))
-            P /= 2;
-        const int kbp = r.k_blocks / P;
-        int stages = rtc::MAX_STAGES;
-        while (stages > 2 && rtc::route_smem(E_pad, kbp, stages).total > 227 * 1024)
-            --stages;
-        if (kbp * N3 * 128 <= rtc::W_MAX_BYTES &&
-            rtc::route_smem(E_pad, kbp, stages).total <= 227 * 1024) {
-            r.fused = true;
-            r.E_pad = E_pad;
-            r.n_chunk = E_pad;
-            r.n_chunks = 1;
-            r.k_parts = P;
-            r.kb_per_part = kbp;
-            r.cluster = P;
-            r.stages = stages;
-            r.blocks = m_tiles * P;   // upper bound; the launch sizes the persistent grid
-            return r;
-        }
+    // One kernel up to 16 experts: each block splits its 16-expert slice of
+    // W_r stage by stage as its x tiles stream.  Wider expert sets split W_r
+    // once (three launches): a one-kernel form measured slower inside the
+    // layer step on the 64- and 256-expert layers.
+    if (c.E <= 16) {
+        r.fused = true;
+        r.n_chunk = 16;
+        r.n_chunks = 1;
+        r.E_pad = 16;
+        // K parts: the most of 4, 2, 1 that keeps the grid within one wave
+        // (two blocks per SM) and at least 4 K blocks per part
+        r.k_parts = 1;
+        for (int kp = rtc::MAX_CLUSTER; kp >= 2; kp /= 2)
+            if ((int64_t)m_tiles * kp <= 296 && r.k_blocks / kp >= 4) {
+                r.k_parts = kp;
+                break;
+            }
+        r.kb_per_part = (int)ceil_div(r.k_blocks, r.k_parts);
+        r.cluster = r.k_parts;
+        r.blocks = m_tiles * r.cluster;
+        return r;
     }
     r.fused = false;
     r.E_pad = c.E <= 64 ? (int)align_up((size_t)c.E, 16) : (int)align_up((size_t)c.E, 64);
@@ -1403,23 +1204,13 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
     p.k_blocks = r.k_blocks;
     p.status = status;
     p.clear_status = clear_status ? 1 : 0;
-    // a K part of W_r (kbp x 64 rows of E floats, contiguous) comes in by bulk
-    // copies when W_r is 16-byte aligned, else by per-thread loads
-    p.w_bulk = reinterpret_cast<uintptr_t>(W_r) % 16 == 0 ? 1 : 0;
     if (r.fused) {
-        p.tiles = (int)ceil_div(c.T, BM);
-        p.stages = r.stages;
+        const unsigned grid = (unsigned)r.blocks;
         if (c.E <= 4)
-            return launch<8, 4>(p, s);
+            return launch<16, 4, 1>(p, grid, s);
         if (c.E <= 8)
-            return launch<8, 8>(p, s);
-        if (c.E <= 16)
-            return launch<16, 0>(p, s);
-        if (c.E <= 32)
-            return launch<32, 0>(p, s);
-        if (c.E <= 48)
-            return launch<48, 0>(p, s);
-        return launch<64, 0>(p, s);
+            return launch<16, 8, 1>(p, grid, s);
+        return launch<16, 0, 1>(p, grid, s);
     }
 
     // three launches: split, logits, select

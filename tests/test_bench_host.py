@@ -104,9 +104,9 @@ def test_layer_summary_rates_and_roofline():
 
 
 def test_launch_count_follows_the_forward():
-    # router 1 (<= 64 experts, split weights fit) or 3, capacity 2, dispatch 1,
-    # two GEMMs, combine 1 unless top-1 without shared experts
+    # router 1 (bf16, <= 16 experts) or 3, capacity 2, dispatch 1, two GEMMs,
+    # combine 1 unless top-1 without shared experts
     assert bench.kernels_per_step(CONFIGS["mixtral"]) == 1 + 2 + 1 + 2 + 1
     assert bench.kernels_per_step(CONFIGS["switch"]) == 1 + 2 + 1 + 2
-    assert bench.kernels_per_step(CONFIGS["deepseekmoe"]) == 1 + 2 + 1 + 2 + 1
+    assert bench.kernels_per_step(CONFIGS["deepseekmoe"]) == 3 + 2 + 1 + 2 + 1
     assert bench.kernels_per_step(CONFIGS["deepseek_v3"]) == 3 + 2 + 1 + 2 + 1

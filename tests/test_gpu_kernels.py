@@ -401,9 +401,9 @@ def test_route_selection_every_width(E, k, score):
 @pytest.mark.parametrize("T,d,E,k", [(1000, 1024, 8, 2), (777, 512, 40, 3),
                                      (16384, 1024, 64, 6), (500, 512, 100, 8)])
 def test_route_with_unaligned_router_weights_gives_the_same_bits(T, d, E, k):
-    """W_r 16-byte aligned (each block's K part copied in bulk) and W_r four
-    bytes off (per-thread loads) give the same top-k, gates, loss partials
-    and logits, bit for bit."""
+    """W_r 16-byte aligned and W_r four bytes off give the same top-k, gates,
+    loss partials and logits, bit for bit (the one-kernel router copies W_r in
+    4-byte pieces, the three-launch split reads it per element)."""
     g = torch.Generator(device=DEV).manual_seed(T + E)
     x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
     W_r = torch.randn((d, E), generator=g, device=DEV) * 0.05
@@ -423,12 +423,11 @@ def test_route_with_unaligned_router_weights_gives_the_same_bits(T, d, E, k):
     (1000, 1024, 4, 1),    # one kernel: 4 experts per token group, K in 4 parts (cluster of 4)
     (777, 512, 8, 2),      # 8 experts per token group, K in 2 parts
     (1000, 1024, 16, 4),   # a warp per token, K in 4 parts
-    (600, 512, 40, 3),     # 48 padded experts, two per lane, K in 2 parts
-    (333, 1024, 64, 6),    # 64 experts (3 x 64 = 192-wide MMA), 3 x stages, ragged last tile
-    (16384, 1024, 8, 2),   # 128 tiles: every cluster walks several (both accumulators and
-                           # logit buffers reused many times)
-    (16384, 1024, 64, 6),  # DeepSeekMoE-shaped: 4 tiles per cluster of 4
-    (20000, 512, 32, 4),   # 157 tiles on clusters of 2, ragged last tile
+    (600, 512, 40, 3),     # three launches: 48 padded experts, two per lane
+    (333, 1024, 64, 6),    # three launches: 64 experts in one chunk, ragged last tile
+    (16384, 1024, 8, 2),   # one kernel: 128 tiles, a cluster of 2 per tile (grid within one wave)
+    (16384, 1024, 64, 6),  # DeepSeekMoE-shaped: three launches
+    (20000, 512, 32, 4),   # three launches, 157 tiles, ragged last tile
     (500, 512, 100, 8),    # three launches: 2 expert chunks x 2 K parts
     (64, 256, 8, 2),       # less than one 128-token tile (one block, K whole)
     (40, 256, 200, 8),     # three launches: 4 expert chunks, two rows of the loss partials
@@ -436,6 +435,6 @@ def test_route_with_unaligned_router_weights_gives_the_same_bits(T, d, E, k):
 @pytest.mark.parametrize("score", [0, 1], ids=["softmax", "sigmoid"])
 def test_route_cluster_shapes(T, d, E, k, score):
     """Every way the router splits the work (one kernel: K parts over a
-    cluster of 1, 2 or 4 blocks, one or many 128-token tiles per cluster;
-    three launches: expert chunks and K parts): the same checks as above."""
+    cluster of 1, 2 or 4 blocks per 128-token tile; three launches: expert
+    chunks and K parts): the same checks as above."""
     _check_route(T, d, E, k, score, T + d + E + k + score)
