@@ -788,6 +788,8 @@ __global__ void __launch_bounds__(256) split_kernel(const float *__restrict__ W_
                                                     int E_pad, __nv_bfloat16 *__restrict__ W3,
                                                     int32_t *status)
 {
+    pdl_wait();   // W_r may come from the previous kernel in the stream
+    pdl_trigger();
     if (status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         *status = 0;   // cleared before the launches whose waits may set it
     __shared__ float tile[32][33];
@@ -856,6 +858,8 @@ __global__ void __launch_bounds__(LOGIT_THREADS, 1) logits_kernel(const __grid_c
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tmem_slot;
+    pdl_wait();   // the split weights (and x) come from earlier kernels
+    pdl_trigger();
 
     if (warp == 0 && lane == 0) {
         // ---- TMA producer ----
@@ -979,6 +983,8 @@ __global__ void __launch_bounds__(32 * kPartialTokens, 1)
 {
     constexpr int W = kPartialTokens;
     __shared__ float pw[W][kMaxE + 1];
+    pdl_wait();   // the partial logits come from the logits kernel
+    pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = a.E;
     const bool renorm = a.renorm < 0 ? (a.k > 1) : (a.renorm != 0);
@@ -1114,8 +1120,7 @@ cudaError_t launch_logits(const LogitParams &p, dim3 grid, cudaStream_t s)
     cudaError_t err = raise_smem_limit((const void *)kern, smem);
     if (err != cudaSuccess)
         return err;
-    kern<<<grid, LOGIT_THREADS, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(LOGIT_THREADS), smem, s, p);
 }
 
 }  // namespace rtc
@@ -1218,8 +1223,8 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
     float *plog = reinterpret_cast<float *>(static_cast<char *>(scratch) +
                                             align_up((size_t)3 * r.E_pad * c.d * 2, 256));
     dim3 sg((unsigned)ceil_div(c.d, 32), (unsigned)ceil_div(r.E_pad, 32));
-    split_kernel<<<sg, 256, 0, s>>>(W_r, c.d, c.E, r.E_pad, W3, clear_status ? status : nullptr);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(split_kernel, sg, dim3(256), 0, s, W_r, c.d, c.E, r.E_pad, W3,
+                                 clear_status ? status : nullptr);
     if (err != cudaSuccess)
         return err;
     LogitParams lp;
@@ -1246,14 +1251,18 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
         return err;
     const unsigned rows = (unsigned)ceil_div(c.T, kPartialTokens);
     if (c.E <= 32)
-        select_kernel<1><<<rows, 32 * kPartialTokens, 0, s>>>(p, plog, r.k_parts, r.E_pad);
+        err = launch_pdl(select_kernel<1>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+                         (const float *)plog, r.k_parts, r.E_pad);
     else if (c.E <= 64)
-        select_kernel<2><<<rows, 32 * kPartialTokens, 0, s>>>(p, plog, r.k_parts, r.E_pad);
+        err = launch_pdl(select_kernel<2>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+                         (const float *)plog, r.k_parts, r.E_pad);
     else if (c.E <= 128)
-        select_kernel<4><<<rows, 32 * kPartialTokens, 0, s>>>(p, plog, r.k_parts, r.E_pad);
+        err = launch_pdl(select_kernel<4>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+                         (const float *)plog, r.k_parts, r.E_pad);
     else
-        select_kernel<8><<<rows, 32 * kPartialTokens, 0, s>>>(p, plog, r.k_parts, r.E_pad);
-    return cudaGetLastError();
+        err = launch_pdl(select_kernel<8>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+                         (const float *)plog, r.k_parts, r.E_pad);
+    return err;
 }
 
 }  // namespace moe
