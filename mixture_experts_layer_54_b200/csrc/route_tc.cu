@@ -60,33 +60,22 @@ __device__ __forceinline__ void bar_arrive(uint32_t bar)
 }
 
 // Bounded wait (about 2 s of wall clock); false on expiry or once `abort` is
-// set.  CLUSTER: acquire at cluster scope, for barriers that blocks of the
-// cluster complete remotely.  (A suspend-time hint on the tries, letting the
-// thread sleep until the phase completes, measured slower here: woken threads
-// resumed up to microseconds after the phase completed.)
-template <bool CLUSTER>
-__device__ __noinline__ bool bar_wait_t(uint32_t bar, uint32_t parity, volatile int *abort,
-                                        int32_t *status)
+// set.  (A suspend-time hint on the tries, letting the thread sleep until the
+// phase completes, measured slower here: woken threads resumed up to
+// microseconds after the phase completed.)
+__device__ __noinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                      int32_t *status)
 {
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t ok;
-        if (CLUSTER)
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-                "selp.u32 %0, 1, 0, p;\n\t}"
-                : "=r"(ok)
-                : "r"(bar), "r"(parity)
-                : "memory");
-        else
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                "selp.u32 %0, 1, 0, p;\n\t}"
-                : "=r"(ok)
-                : "r"(bar), "r"(parity)
-                : "memory");
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
         if (ok)
             return true;
         if ((i & 31u) == 0) {
@@ -105,12 +94,6 @@ __device__ __noinline__ bool bar_wait_t(uint32_t bar, uint32_t parity, volatile 
             }
         }
     }
-}
-
-__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                         int32_t *status)
-{
-    return bar_wait_t<false>(bar, parity, abort, status);
 }
 
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t a)
@@ -212,161 +195,106 @@ __device__ __forceinline__ SelArgs sel_args(const RouteParams &p)
     return SelArgs{p.topk, p.gates, p.logits_out, p.scores_out, p.select_bias, p.E, p.k, p.score};
 }
 
-// NT tokens held by a whole warp, lane l holding experts l, l + 32, ... (PL
-// of them) of each: softmax or sigmoid, top-k and gates; adds the loss terms
-// of the tokens with tv set to pacc / zacc in token order.  The NT tokens'
-// steps are independent, so the warp keeps NT dependency chains in flight
-// instead of one.  SB_REG: sb holds the lane's selection biases (0 without);
+// One token held by a whole warp, lane l holding experts l, l + 32, ... (PL of
+// them): softmax or sigmoid, top-k and gates; adds the token's loss terms to
+// pacc / zacc.  SB_REG: sb holds the lane's selection biases (0 without);
 // otherwise they are read from a.select_bias.  Each top-k round is two integer
 // warp reductions: the largest key, then the lowest expert index holding it
 // (ties go to the lower index); lane j keeps round j's expert and value, so
-// the k outputs go out from k lanes at once (the gate sum still adds the
-// values in round order).  A token with tv clear takes part in the warp
-// reductions (with finite logits) and writes nothing.
-template <int PL, int NT, bool SB_REG>
-__device__ __forceinline__ void select_tokens(const SelArgs &a, bool renorm, const int (&t)[NT],
-                                              const bool (&tv)[NT], int lane,
-                                              const float (&z)[NT][PL], const float (&sb)[PL],
-                                              float (&pacc)[PL], float &zacc)
-{
-    const int E = a.E;
-    float m[NT], sum[NT], lse[NT], ssum[NT], v[NT][PL];
-    uint32_t okey[NT][PL];   // 0: not an expert of this layer, or taken
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        uint32_t mo = 0;
-#pragma unroll
-        for (int i = 0; i < PL; ++i)
-            if (lane + 32 * i < E)
-                mo = max(mo, ord_key(z[n][i]));
-        m[n] = unord_key(__reduce_max_sync(0xffffffffu, mo));
-    }
-    float ex[NT][PL];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        sum[n] = 0.f;
-#pragma unroll
-        for (int i = 0; i < PL; ++i) {
-            ex[n][i] = lane + 32 * i < E ? expf(z[n][i] - m[n]) : 0.f;
-            sum[n] += ex[n][i];
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-            sum[n] += __shfl_xor_sync(0xffffffffu, sum[n], o);
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        lse[n] = m[n] + logf(sum[n]);
-        ssum[n] = 0.f;
-#pragma unroll
-        for (int i = 0; i < PL; ++i) {
-            const int e = lane + 32 * i;
-            const bool okk = e < E;
-            float key;
-            if (a.score == MOE_SCORE_SOFTMAX) {
-                v[n][i] = okk ? ex[n][i] / sum[n] : 0.f;
-                key = z[n][i];
-            } else {
-                v[n][i] = okk ? 1.f / (1.f + expf(-z[n][i])) : 0.f;
-                key = v[n][i] + (SB_REG ? sb[i] : (a.select_bias && okk ? a.select_bias[e] : 0.f));
-                ssum[n] += v[n][i];
-            }
-            okey[n][i] = okk ? ord_key(key) : 0u;
-            if (okk && tv[n] && a.logits_out)
-                a.logits_out[(int64_t)t[n] * E + e] = z[n][i];
-            if (okk && tv[n] && a.scores_out)
-                a.scores_out[(int64_t)t[n] * E + e] = v[n][i];
-        }
-    }
-    if (a.score == MOE_SCORE_SIGMOID) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-                ssum[n] += __shfl_xor_sync(0xffffffffu, ssum[n], o);
-    }
-    int my_idx[NT];
-    float my_v[NT], sel_sum[NT];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        my_idx[n] = 0;
-        my_v[n] = 0.f;
-        sel_sum[n] = 0.f;
-    }
-#pragma unroll 1
-    for (int j = 0; j < a.k; ++j) {
-        uint32_t mk[NT];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            uint32_t lk = 0;
-#pragma unroll
-            for (int i = 0; i < PL; ++i)
-                lk = max(lk, okey[n][i]);
-            mk[n] = __reduce_max_sync(0xffffffffu, lk);
-        }
-        uint32_t bi[NT];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            uint32_t li = 0xffffffffu;
-#pragma unroll
-            for (int i = PL - 1; i >= 0; --i)
-                if (okey[n][i] == mk[n] && mk[n] != 0u)
-                    li = (uint32_t)(lane + 32 * i);
-            bi[n] = __reduce_min_sync(0xffffffffu, li);
-        }
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int slot = (int)(bi[n] >> 5);
-            float mine = v[n][0];
-#pragma unroll
-            for (int i = 1; i < PL; ++i)
-                if (slot == i)
-                    mine = v[n][i];
-            const float bv = __shfl_sync(0xffffffffu, mine, (int)(bi[n] & 31u));
-            if ((int)(bi[n] & 31u) == lane) {
-#pragma unroll
-                for (int i = 0; i < PL; ++i)
-                    if (slot == i)
-                        okey[n][i] = 0u;   // taken
-            }
-            if (lane == j) {
-                my_idx[n] = (int)bi[n];
-                my_v[n] = bv;
-            }
-            sel_sum[n] += bv;
-        }
-    }
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        if (!tv[n])
-            continue;
-        if (lane < a.k) {
-            a.topk[(int64_t)t[n] * a.k + lane] = my_idx[n];
-            a.gates[(int64_t)t[n] * a.k + lane] = renorm ? my_v[n] / sel_sum[n] : my_v[n];
-        }
-        if (lane == 0)
-            zacc += lse[n] * lse[n];
-#pragma unroll
-        for (int i = 0; i < PL; ++i)
-            if (lane + 32 * i < E)
-                pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[n][i] : v[n][i] / ssum[n];
-    }
-}
-
+// the k outputs and their divisions go out from k lanes at once (the gate sum
+// still adds the values in round order).
 template <int PL, bool SB_REG>
 __device__ __forceinline__ void select_token(const SelArgs &a, bool renorm, int t, int lane,
                                              const float (&z)[PL], const float (&sb)[PL],
                                              float (&pacc)[PL], float &zacc)
 {
-    const int tt[1] = {t};
-    const bool tv[1] = {true};
-    float zz[1][PL];
+    const int E = a.E;
+    uint32_t mo = 0;
 #pragma unroll
     for (int i = 0; i < PL; ++i)
-        zz[0][i] = z[i];
-    select_tokens<PL, 1, SB_REG>(a, renorm, tt, tv, lane, zz, sb, pacc, zacc);
+        if (lane + 32 * i < E)
+            mo = max(mo, ord_key(z[i]));
+    const float m = unord_key(__reduce_max_sync(0xffffffffu, mo));
+    float ex[PL], sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+        ex[i] = lane + 32 * i < E ? expf(z[i] - m) : 0.f;
+        sum += ex[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float lse = m + logf(sum);
+    float v[PL], ssum = 0.f;
+    uint32_t okey[PL];   // 0: not an expert of this layer, or taken
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+        const int e = lane + 32 * i;
+        const bool okk = e < E;
+        float key;
+        if (a.score == MOE_SCORE_SOFTMAX) {
+            v[i] = okk ? ex[i] / sum : 0.f;
+            key = z[i];
+        } else {
+            v[i] = okk ? 1.f / (1.f + expf(-z[i])) : 0.f;
+            key = v[i] + (SB_REG ? sb[i] : (a.select_bias && okk ? a.select_bias[e] : 0.f));
+            ssum += v[i];
+        }
+        okey[i] = okk ? ord_key(key) : 0u;
+        if (okk && a.logits_out)
+            a.logits_out[(int64_t)t * E + e] = z[i];
+        if (okk && a.scores_out)
+            a.scores_out[(int64_t)t * E + e] = v[i];
+    }
+    if (a.score == MOE_SCORE_SIGMOID) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+    }
+    int my_idx = 0;
+    float my_v = 0.f, sel_sum = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < a.k; ++j) {
+        uint32_t lk = 0;
+#pragma unroll
+        for (int i = 0; i < PL; ++i)
+            lk = max(lk, okey[i]);
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
+        uint32_t li = 0xffffffffu;
+#pragma unroll
+        for (int i = PL - 1; i >= 0; --i)
+            if (okey[i] == mk && mk != 0u)
+                li = (uint32_t)(lane + 32 * i);
+        const uint32_t bi = __reduce_min_sync(0xffffffffu, li);
+        const int slot = (int)(bi >> 5);
+        float mine = v[0];
+#pragma unroll
+        for (int i = 1; i < PL; ++i)
+            if (slot == i)
+                mine = v[i];
+        const float bv = __shfl_sync(0xffffffffu, mine, (int)(bi & 31u));
+        if ((int)(bi & 31u) == lane) {
+#pragma unroll
+            for (int i = 0; i < PL; ++i)
+                if (slot == i)
+                    okey[i] = 0u;   // taken
+        }
+        if (lane == j) {
+            my_idx = (int)bi;
+            my_v = bv;
+        }
+        sel_sum += bv;
+    }
+    if (lane < a.k) {
+        a.topk[(int64_t)t * a.k + lane] = my_idx;
+        a.gates[(int64_t)t * a.k + lane] = renorm ? my_v / sel_sum : my_v;
+    }
+    if (lane == 0)
+        zacc += lse * lse;
+#pragma unroll
+    for (int i = 0; i < PL; ++i)
+        if (lane + 32 * i < E)
+            pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[i] : v[i] / ssum;
 }
 
 // ---------------------------------------------------------------- kernel
