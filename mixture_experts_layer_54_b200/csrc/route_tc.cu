@@ -134,10 +134,6 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const float *src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit()
-{
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
 // Arrives on the mbarrier once this thread's earlier cp.async copies land.
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar)
 {
