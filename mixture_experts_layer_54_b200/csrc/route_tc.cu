@@ -191,106 +191,161 @@ __device__ __forceinline__ SelArgs sel_args(const RouteParams &p)
     return SelArgs{p.topk, p.gates, p.logits_out, p.scores_out, p.select_bias, p.E, p.k, p.score};
 }
 
-// One token held by a whole warp, lane l holding experts l, l + 32, ... (PL of
-// them): softmax or sigmoid, top-k and gates; adds the token's loss terms to
-// pacc / zacc.  SB_REG: sb holds the lane's selection biases (0 without);
+// NT tokens held by a whole warp, lane l holding experts l, l + 32, ... (PL
+// of them) of each: softmax or sigmoid, top-k and gates; adds the loss terms
+// of the tokens with tv set to pacc / zacc in token order.  The NT tokens'
+// steps are independent, so the warp keeps NT dependency chains in flight
+// instead of one.  SB_REG: sb holds the lane's selection biases (0 without);
 // otherwise they are read from a.select_bias.  Each top-k round is two integer
 // warp reductions: the largest key, then the lowest expert index holding it
 // (ties go to the lower index); lane j keeps round j's expert and value, so
-// the k outputs and their divisions go out from k lanes at once (the gate sum
-// still adds the values in round order).
+// the k outputs go out from k lanes at once (the gate sum still adds the
+// values in round order).  A token with tv clear takes part in the warp
+// reductions (with finite logits) and writes nothing.
+template <int PL, int NT, bool SB_REG>
+__device__ __forceinline__ void select_tokens(const SelArgs &a, bool renorm, const int (&t)[NT],
+                                              const bool (&tv)[NT], int lane,
+                                              const float (&z)[NT][PL], const float (&sb)[PL],
+                                              float (&pacc)[PL], float &zacc)
+{
+    const int E = a.E;
+    float m[NT], sum[NT], lse[NT], ssum[NT], v[NT][PL];
+    uint32_t okey[NT][PL];   // 0: not an expert of this layer, or taken
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        uint32_t mo = 0;
+#pragma unroll
+        for (int i = 0; i < PL; ++i)
+            if (lane + 32 * i < E)
+                mo = max(mo, ord_key(z[n][i]));
+        m[n] = unord_key(__reduce_max_sync(0xffffffffu, mo));
+    }
+    float ex[NT][PL];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        sum[n] = 0.f;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+            ex[n][i] = lane + 32 * i < E ? expf(z[n][i] - m[n]) : 0.f;
+            sum[n] += ex[n][i];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+            sum[n] += __shfl_xor_sync(0xffffffffu, sum[n], o);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        lse[n] = m[n] + logf(sum[n]);
+        ssum[n] = 0.f;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+            const int e = lane + 32 * i;
+            const bool okk = e < E;
+            float key;
+            if (a.score == MOE_SCORE_SOFTMAX) {
+                v[n][i] = okk ? ex[n][i] / sum[n] : 0.f;
+                key = z[n][i];
+            } else {
+                v[n][i] = okk ? 1.f / (1.f + expf(-z[n][i])) : 0.f;
+                key = v[n][i] + (SB_REG ? sb[i] : (a.select_bias && okk ? a.select_bias[e] : 0.f));
+                ssum[n] += v[n][i];
+            }
+            okey[n][i] = okk ? ord_key(key) : 0u;
+            if (okk && tv[n] && a.logits_out)
+                a.logits_out[(int64_t)t[n] * E + e] = z[n][i];
+            if (okk && tv[n] && a.scores_out)
+                a.scores_out[(int64_t)t[n] * E + e] = v[n][i];
+        }
+    }
+    if (a.score == MOE_SCORE_SIGMOID) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+                ssum[n] += __shfl_xor_sync(0xffffffffu, ssum[n], o);
+    }
+    int my_idx[NT];
+    float my_v[NT], sel_sum[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        my_idx[n] = 0;
+        my_v[n] = 0.f;
+        sel_sum[n] = 0.f;
+    }
+#pragma unroll 1
+    for (int j = 0; j < a.k; ++j) {
+        uint32_t mk[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            uint32_t lk = 0;
+#pragma unroll
+            for (int i = 0; i < PL; ++i)
+                lk = max(lk, okey[n][i]);
+            mk[n] = __reduce_max_sync(0xffffffffu, lk);
+        }
+        uint32_t bi[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            uint32_t li = 0xffffffffu;
+#pragma unroll
+            for (int i = PL - 1; i >= 0; --i)
+                if (okey[n][i] == mk[n] && mk[n] != 0u)
+                    li = (uint32_t)(lane + 32 * i);
+            bi[n] = __reduce_min_sync(0xffffffffu, li);
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int slot = (int)(bi[n] >> 5);
+            float mine = v[n][0];
+#pragma unroll
+            for (int i = 1; i < PL; ++i)
+                if (slot == i)
+                    mine = v[n][i];
+            const float bv = __shfl_sync(0xffffffffu, mine, (int)(bi[n] & 31u));
+            if ((int)(bi[n] & 31u) == lane) {
+#pragma unroll
+                for (int i = 0; i < PL; ++i)
+                    if (slot == i)
+                        okey[n][i] = 0u;   // taken
+            }
+            if (lane == j) {
+                my_idx[n] = (int)bi[n];
+                my_v[n] = bv;
+            }
+            sel_sum[n] += bv;
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        if (!tv[n])
+            continue;
+        if (lane < a.k) {
+            a.topk[(int64_t)t[n] * a.k + lane] = my_idx[n];
+            a.gates[(int64_t)t[n] * a.k + lane] = renorm ? my_v[n] / sel_sum[n] : my_v[n];
+        }
+        if (lane == 0)
+            zacc += lse[n] * lse[n];
+#pragma unroll
+        for (int i = 0; i < PL; ++i)
+            if (lane + 32 * i < E)
+                pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[n][i] : v[n][i] / ssum[n];
+    }
+}
+
 template <int PL, bool SB_REG>
 __device__ __forceinline__ void select_token(const SelArgs &a, bool renorm, int t, int lane,
                                              const float (&z)[PL], const float (&sb)[PL],
                                              float (&pacc)[PL], float &zacc)
 {
-    const int E = a.E;
-    uint32_t mo = 0;
+    const int tt[1] = {t};
+    const bool tv[1] = {true};
+    float zz[1][PL];
 #pragma unroll
     for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i < E)
-            mo = max(mo, ord_key(z[i]));
-    const float m = unord_key(__reduce_max_sync(0xffffffffu, mo));
-    float ex[PL], sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < PL; ++i) {
-        ex[i] = lane + 32 * i < E ? expf(z[i] - m) : 0.f;
-        sum += ex[i];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float lse = m + logf(sum);
-    float v[PL], ssum = 0.f;
-    uint32_t okey[PL];   // 0: not an expert of this layer, or taken
-#pragma unroll
-    for (int i = 0; i < PL; ++i) {
-        const int e = lane + 32 * i;
-        const bool okk = e < E;
-        float key;
-        if (a.score == MOE_SCORE_SOFTMAX) {
-            v[i] = okk ? ex[i] / sum : 0.f;
-            key = z[i];
-        } else {
-            v[i] = okk ? 1.f / (1.f + expf(-z[i])) : 0.f;
-            key = v[i] + (SB_REG ? sb[i] : (a.select_bias && okk ? a.select_bias[e] : 0.f));
-            ssum += v[i];
-        }
-        okey[i] = okk ? ord_key(key) : 0u;
-        if (okk && a.logits_out)
-            a.logits_out[(int64_t)t * E + e] = z[i];
-        if (okk && a.scores_out)
-            a.scores_out[(int64_t)t * E + e] = v[i];
-    }
-    if (a.score == MOE_SCORE_SIGMOID) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
-    }
-    int my_idx = 0;
-    float my_v = 0.f, sel_sum = 0.f;
-#pragma unroll 1
-    for (int j = 0; j < a.k; ++j) {
-        uint32_t lk = 0;
-#pragma unroll
-        for (int i = 0; i < PL; ++i)
-            lk = max(lk, okey[i]);
-        const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
-        uint32_t li = 0xffffffffu;
-#pragma unroll
-        for (int i = PL - 1; i >= 0; --i)
-            if (okey[i] == mk && mk != 0u)
-                li = (uint32_t)(lane + 32 * i);
-        const uint32_t bi = __reduce_min_sync(0xffffffffu, li);
-        const int slot = (int)(bi >> 5);
-        float mine = v[0];
-#pragma unroll
-        for (int i = 1; i < PL; ++i)
-            if (slot == i)
-                mine = v[i];
-        const float bv = __shfl_sync(0xffffffffu, mine, (int)(bi & 31u));
-        if ((int)(bi & 31u) == lane) {
-#pragma unroll
-            for (int i = 0; i < PL; ++i)
-                if (slot == i)
-                    okey[i] = 0u;   // taken
-        }
-        if (lane == j) {
-            my_idx = (int)bi;
-            my_v = bv;
-        }
-        sel_sum += bv;
-    }
-    if (lane < a.k) {
-        a.topk[(int64_t)t * a.k + lane] = my_idx;
-        a.gates[(int64_t)t * a.k + lane] = renorm ? my_v / sel_sum : my_v;
-    }
-    if (lane == 0)
-        zacc += lse * lse;
-#pragma unroll
-    for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i < E)
-            pacc[i] += a.score == MOE_SCORE_SOFTMAX ? v[i] : v[i] / ssum;
+        zz[0][i] = z[i];
+    select_tokens<PL, 1, SB_REG>(a, renorm, tt, tv, lane, zz, sb, pacc, zacc);
 }
 
 // ---------------------------------------------------------------- kernel
@@ -900,43 +955,54 @@ __global__ void __launch_bounds__(LOGIT_THREADS, 1) logits_kernel(const __grid_c
 // Selection of the three-launch path: one block per row of 32 tokens, a warp
 // per token, the K parts summed in order; the warps' sums meet in shared
 // memory in warp order.
-template <int PL>
-__global__ void __launch_bounds__(32 * kPartialTokens, 1)
+// One block per row of 32 tokens (a row of the loss partials): 32 / NT warps,
+// warp w taking tokens w, w + 32 / NT, ... of the row, its NT tokens at once.
+// The row's sums meet in shared memory in warp order.  Launched with NT = 4 up
+// to 64 experts (four blocks per SM fit, so one wave; 5% faster on the
+// DeepSeekMoE shape) and NT = 1 above (eight experts per lane: two tokens per
+// warp in 16-warp blocks measured 18% slower on the DeepSeek-V3 shape).
+template <int PL, int NT>
+__global__ void __launch_bounds__(32 * kPartialTokens / NT)
     select_kernel(const __grid_constant__ RouteParams a, const float *__restrict__ partial,
                   int parts, int E_pad)
 {
-    constexpr int W = kPartialTokens;
+    constexpr int W = kPartialTokens / NT;   // warps per block
     __shared__ float pw[W][kMaxE + 1];
     pdl_wait();   // the partial logits come from the logits kernel
     pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = a.E;
     const bool renorm = a.renorm < 0 ? (a.k > 1) : (a.renorm != 0);
-    const int t = blockIdx.x * kPartialTokens + warp;
     float pacc[PL];
 #pragma unroll
     for (int i = 0; i < PL; ++i)
         pacc[i] = 0.f;
     float zacc = 0.f;
-    if (t < a.T) {
-        float z[PL], sb[PL];
+    int tt[NT];
+    bool tv[NT];
+    float z[NT][PL], sb[PL];
+#pragma unroll
+    for (int i = 0; i < PL; ++i)
+        sb[i] = 0.f;   // unused: the selection biases are read in place
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        tt[n] = blockIdx.x * kPartialTokens + warp + n * W;
+        tv[n] = tt[n] < a.T;
 #pragma unroll
         for (int i = 0; i < PL; ++i) {
             const int e = lane + 32 * i;
-            z[i] = -INFINITY;
-            sb[i] = 0.f;   // unused: the biases are read in place
-            if (e < E) {
-                float s = 0.f;
+            float s = 0.f;
+            if (e < E && tv[n]) {
                 for (int q = 0; q < parts; ++q)
-                    s += partial[((int64_t)q * a.T + t) * E_pad + e];
+                    s += partial[((int64_t)q * a.T + tt[n]) * E_pad + e];
                 if (a.logit_bias)
                     s += a.logit_bias[e];
-                z[i] = s;
             }
+            z[n][i] = s;
         }
-        const SelArgs sa = sel_args(a);
-        select_token<PL, false>(sa, renorm, t, lane, z, sb, pacc, zacc);
     }
+    const SelArgs sa = sel_args(a);
+    select_tokens<PL, NT, false>(sa, renorm, tt, tv, lane, z, sb, pacc, zacc);
 #pragma unroll
     for (int i = 0; i < PL; ++i)
         if (lane + 32 * i < E)
@@ -1175,16 +1241,16 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
         return err;
     const unsigned rows = (unsigned)ceil_div(c.T, kPartialTokens);
     if (c.E <= 32)
-        err = launch_pdl(select_kernel<1>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+        err = launch_pdl(select_kernel<1, 4>, dim3(rows), dim3(32 * kPartialTokens / 4), 0, s, p,
                          (const float *)plog, r.k_parts, r.E_pad);
     else if (c.E <= 64)
-        err = launch_pdl(select_kernel<2>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+        err = launch_pdl(select_kernel<2, 4>, dim3(rows), dim3(32 * kPartialTokens / 4), 0, s, p,
                          (const float *)plog, r.k_parts, r.E_pad);
     else if (c.E <= 128)
-        err = launch_pdl(select_kernel<4>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+        err = launch_pdl(select_kernel<4, 1>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
                          (const float *)plog, r.k_parts, r.E_pad);
     else
-        err = launch_pdl(select_kernel<8>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
+        err = launch_pdl(select_kernel<8, 1>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
                          (const float *)plog, r.k_parts, r.E_pad);
     return err;
 }
