@@ -130,6 +130,23 @@ __device__ __forceinline__ float ld_peer(uint32_t a)
     return v;
 }
 
+// Sum of the float at offset off in the parts blocks whose shared bases are
+// rb[0 .. parts - 1] (parts <= MAX_CLUSTER), in part order.  Every remote load
+// is issued before the first add, so the parts cost one round trip.
+__device__ __forceinline__ float sum_parts(const uint32_t *rb, int parts, uint32_t off)
+{
+    float v[MAX_CLUSTER];
+#pragma unroll
+    for (int q = 0; q < MAX_CLUSTER; ++q)
+        v[q] = q < parts ? ld_peer(rb[q] + off) : 0.f;
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < MAX_CLUSTER; ++q)
+        if (q < parts)
+            s += v[q];
+    return s;
+}
+
 __device__ __forceinline__ void cp_async4(uint32_t dst, const float *src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -383,6 +400,7 @@ __global__ void __launch_bounds__(THREADS, N <= 16 ? 2 : 1)
     static_assert(L_BYTES + WARPS * (kMaxE + 1) * 4 <= STAGES * STAGE, "select scratch");
     static_assert(STAGES * (STAGE + RAW) + 1024 <= 227 * 1024, "shared memory");
     static_assert(COPY_WARP0 + CONV_LANES / 32 <= WARPS, "roles");
+    static_assert(N == 16, "one block per K part covers the layer's E <= 16 experts");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -655,11 +673,8 @@ __global__ void __launch_bounds__(THREADS, N <= 16 ? 2 : 1)
             const int tg = tl0 + g * TB;
             const int tl = tg + lane / E_T;
             float z = -INFINITY;
-            if (m0 + tl < p.T && gl < E) {
-                z = 0.f;
-                for (int q = 0; q < p.k_parts; ++q)
-                    z += ld_peer(rb[q] + (uint32_t)(tl * LS + gl) * 4u);
-            }
+            if (m0 + tl < p.T && gl < E)
+                z = sum_parts(rb, p.k_parts, (uint32_t)(tl * LS + gl) * 4u);
             float pc, zc;
             small_epilogue<E_T>(ra, z, m0 + tg, lane, renorm, lbv, sbv, &pc, &zc);
             if (lane < E_T)
@@ -708,10 +723,8 @@ __global__ void __launch_bounds__(THREADS, N <= 16 ? 2 : 1)
                     const int e = lane + 32 * i;
                     z[i] = -INFINITY;
                     if (e < E) {
-                        const int ch = e / N, el = e - ch * N;
-                        float s = 0.f;
-                        for (int q = 0; q < p.k_parts; ++q)
-                            s += ld_peer(rb[ch * p.k_parts + q] + (uint32_t)(tl * LS + el) * 4u);
+                        // one block per tile covers all experts (E <= N)
+                        float s = sum_parts(rb, p.k_parts, (uint32_t)(tl * LS + e) * 4u);
                         if (p.logit_bias)
                             s += lb[i];
                         z[i] = s;
