@@ -86,6 +86,7 @@ void carve_stage_into(const moe_config &c, Carver &cv, StageScratch &s)
     Carver route_cv{cv.base, off}, cap_cv{cv.base, off}, ffn_cv{cv.base, off};
     s.route = route_cv.take(route_scratch_bytes(c));
     s.hist = static_cast<int32_t *>(cap_cv.take(hk));
+    s.loss_ps = static_cast<double *>(cap_cv.take(kLossUnits * sizeof(double)));
     s.count_base = static_cast<int32_t *>(cap_cv.take((size_t)c.E * 4));
     s.keys = static_cast<unsigned long long *>(
         cap_cv.take(c.priority == MOE_PRIORITY_SCORE ? (size_t)c.T * c.k * 8 : 0));
@@ -588,7 +589,7 @@ moe_status moe_forward(const moe_config *cfg, const moe_weights *w, const void *
         st = cuda_status(launch_capacity(c, capacity_of(c), f.topk, f.counts, f.pos, f.keep,
                                          f.kept, f.offsets, f.dropped, f.n_dropped, s.hist,
                                          reinterpret_cast<cudaStream_t>(stream), nullptr,
-                                         f.partials, out->aux, out->zloss));
+                                         f.partials, s.loss_ps, out->aux, out->zloss));
     if (st != MOE_OK)
         return st;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);

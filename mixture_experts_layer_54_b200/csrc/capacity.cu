@@ -42,8 +42,20 @@ namespace {
 constexpr int CT = kCapTokens;   // tokens per block (also the thread count)
 
 __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int T, int k, int E,
-                                                       int32_t *hist)
+                                                       int32_t *hist, int nblk,
+                                                       const float *partials, int prows,
+                                                       double *loss_ps)
 {
+    if ((int)blockIdx.x >= nblk) {
+        // the whole forward's extra blocks: phase sums of the loss partials,
+        // thread u of these blocks taking work unit u (losses_common.cuh)
+        pdl_wait();   // the partials come from the router
+        pdl_trigger();
+        const int C = E + 1, u = ((int)blockIdx.x - nblk) * CT + (int)threadIdx.x;
+        if (u < loss_phases(C) * C)
+            loss_ps[u] = loss_phase_sum(partials, prows, C, u);
+        return;
+    }
     extern __shared__ int32_t h[];   // [k][E]
     for (int i = threadIdx.x; i < k * E; i += CT)
         h[i] = 0;
@@ -98,12 +110,13 @@ __device__ void capacity_totals(const int32_t *__restrict__ hist, int nblk, int 
                                 long long C, const int32_t *__restrict__ count_base, int T,
                                 int32_t *__restrict__ counts, int32_t *__restrict__ kept,
                                 int32_t *__restrict__ offsets, int32_t *__restrict__ n_dropped,
-                                const float *partials, int prows, float *aux, float *zloss,
+                                const double *loss_ps, float *aux, float *zloss,
                                 int32_t *colsum)
 {
     __shared__ int32_t cnt[kMaxE];
     __shared__ int32_t kept_s[kMaxE];
     __shared__ double term[kMaxE + 1];
+    __shared__ double ps[kLossUnits];
     hist_sums(hist, nblk, k * E, nblk, colsum, nullptr);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -154,8 +167,14 @@ __device__ void capacity_totals(const int32_t *__restrict__ hist, int nblk, int 
             *n_dropped = (int32_t)drop;
         }
     }
-    if (partials)
-        block_losses(cnt, partials, prows, T > 0 ? T : 1, k, E, aux, zloss, term);
+    if (loss_ps) {
+        // the phase sums from the count launch's extra blocks, then the terms
+        const int units = loss_phases(E + 1) * (E + 1);
+        for (int u = threadIdx.x; u < units; u += blockDim.x)
+            ps[u] = loss_ps[u];
+        __syncthreads();
+        losses_from_phase_sums(cnt, ps, T > 0 ? T : 1, k, E, aux, zloss, term);
+    }
 }
 
 // Each warp owns 32 consecutive tokens of the block.  Per pass (token order:
@@ -175,8 +194,7 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
                  int nblk, int32_t *__restrict__ pos, uint8_t *__restrict__ keep,
                  uint8_t *__restrict__ dropped, int32_t *__restrict__ counts,
                  int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
-                 int32_t *__restrict__ n_dropped, const float *partials, int prows, float *aux,
-                 float *zloss)
+                 int32_t *__restrict__ n_dropped, const double *loss_ps, float *aux, float *zloss)
 {
     __shared__ int32_t wrun[CT / 32][kMaxE];
     __shared__ uint8_t keep_s[CT * kMaxK];
@@ -186,7 +204,7 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
     const int cols = k * E;
     if (blockIdx.x == nblk) {
         capacity_totals(hist, nblk, k, E, C, count_base, T, counts, kept, offsets, n_dropped,
-                        partials, prows, aux, zloss, before);
+                        loss_ps, aux, zloss, before);
         return;
     }
     const bool token_order = priority == MOE_PRIORITY_TOKEN;
@@ -438,20 +456,23 @@ cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep, int32_t *kept,
                             int32_t *offsets, uint8_t *dropped, int32_t *n_dropped,
                             int32_t *hist, cudaStream_t s, const int32_t *count_base,
-                            const float *partials, float *aux, float *zloss)
+                            const float *partials, double *loss_ps, float *aux, float *zloss)
 {
     const int nblk = cap_blocks(c);
-    if (nblk > 0) {
-        cudaError_t err = launch_pdl(cap_count_kernel, dim3(nblk), dim3(CT),
-                                     sizeof(int32_t) * c.k * c.E, s, topk, c.T, c.k, c.E, hist);
+    // with the losses: extra count blocks for the phase sums of the partials
+    const int lblk = partials ? (loss_phases(c.E + 1) * (c.E + 1) + CT - 1) / CT : 0;
+    if (nblk + lblk > 0) {
+        cudaError_t err = launch_pdl(cap_count_kernel, dim3(nblk + lblk), dim3(CT),
+                                     sizeof(int32_t) * c.k * c.E, s, topk, c.T, c.k, c.E, hist,
+                                     nblk, partials, partial_rows(c), loss_ps);
         if (err != cudaSuccess)
             return err;
     }
     // placement blocks, then the totals block (and the losses when asked)
     return launch_pdl(cap_place_kernel, dim3(nblk + 1), dim3(CT), 0, s, topk, c.T, c.k, c.E,
                       c.priority, (long long)C, count_base, (const int32_t *)hist, nblk, pos,
-                      keep, dropped, counts, kept, offsets, n_dropped, partials, partial_rows(c),
-                      aux, zloss);
+                      keep, dropped, counts, kept, offsets, n_dropped,
+                      partials ? (const double *)loss_ps : nullptr, aux, zloss);
 }
 
 }  // namespace moe

@@ -15,6 +15,7 @@ constexpr int kMaxK = 8;
 constexpr int kRouteTokens = 32;   // tokens per block of the tiled route kernel
 constexpr int kPartialTokens = 32;  // tokens per row of the loss partials
 constexpr int kCapTokens = 256;    // tokens per capacity block
+constexpr int kLossUnits = 1024;   // most (row phase, column) units of the loss reduction
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -89,6 +90,7 @@ struct StageScratch {
     int32_t *status;      // device status word (timeouts)
     void *route;          // tensor-core router (three launches): split weights, partial logits
     int32_t *hist;        // [cap_blocks][k][E]
+    double *loss_ps;      // [kLossUnits] the whole forward's loss phase sums
     int32_t *count_base;  // [E] sharded capacity: earlier shards' assignments
     unsigned long long *keys;   // [T k] batch-prioritized capacity: per-expert lists
     void *H;              // [perm_rows][F] dtype
@@ -114,14 +116,15 @@ cudaError_t launch_shard_base(const moe_config &c, const int32_t *shard_counts, 
 // hist: scratch [cap_blocks][k][E] int32.  count_base (nullable, [E]):
 // assignments to each expert in earlier shards of the same global batch
 // (token order); C is then the global batch's capacity.  partials (nullable,
-// the router's loss partials): the same launch also writes aux and zloss.
+// the router's loss partials): the same two launches also write aux and
+// zloss, with the phase sums in loss_ps (scratch of kLossUnits doubles).
 cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
                             int32_t *counts, int32_t *pos, uint8_t *keep,
                             int32_t *kept, int32_t *offsets, uint8_t *dropped,
                             int32_t *n_dropped, int32_t *hist, cudaStream_t s,
                             const int32_t *count_base = nullptr,
-                            const float *partials = nullptr, float *aux = nullptr,
-                            float *zloss = nullptr);
+                            const float *partials = nullptr, double *loss_ps = nullptr,
+                            float *aux = nullptr, float *zloss = nullptr);
 
 cudaError_t launch_capacity_scored(const moe_config &c, int64_t C, const int32_t *topk,
                                    const float *scores, int32_t *counts, int32_t *pos,

@@ -11,19 +11,24 @@
 namespace moe {
 namespace {
 
-constexpr int THREADS = 1024;
+constexpr int THREADS = kLossUnits;
 
-// One block: column c of the partials (expert c, or the lse^2 column c = E)
-// is summed by warp c mod 32 in the fixed order of loss_column_sum, then one
-// thread adds the E terms in expert order.
+// One block: thread u computes the phase sum of work unit u (losses_common.cuh)
+// into shared memory, then the terms in the fixed order of
+// losses_from_phase_sums: the same bits as the forward's capacity stage.
 __global__ void __launch_bounds__(THREADS)
 losses_kernel(const int32_t *__restrict__ counts, const float *__restrict__ partials, int rows,
               int T, int k, int E, float *aux, float *zloss)
 {
     __shared__ double term[kMaxE + 1];
+    __shared__ double ps[kLossUnits];
     pdl_wait();   // counts and partials come from the capacity and route stages
     pdl_trigger();
-    block_losses(counts, partials, rows, T, k, E, aux, zloss, term);
+    const int C = E + 1;
+    if ((int)threadIdx.x < loss_phases(C) * C)
+        ps[threadIdx.x] = loss_phase_sum(partials, rows, C, threadIdx.x);
+    __syncthreads();
+    losses_from_phase_sums(counts, ps, T, k, E, aux, zloss, term);
 }
 
 }  // namespace

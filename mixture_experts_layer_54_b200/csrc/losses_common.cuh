@@ -1,6 +1,6 @@
 // The fixed-order reduction of the loss partials, shared by the losses kernel
 // and the capacity stage of the whole forward (which computes the losses in
-// the same launch), so that both give the same bits.
+// its two launches), so that both give the same bits.
 //
 // Page "Lab 18 - Mixture of experts", section 2:
 //   L_aux = E * sum_i f_i P_i, f_i = counts_i / (T k), P_i = mean_t p_{t,i}
@@ -12,37 +12,55 @@
 
 namespace moe {
 
-// Column col of the partials [rows][C] (expert col < E, or the lse^2 column
-// col = E), summed by one warp: lane l adds rows l, l + 32, ... in order in
-// double, then the 32 lane sums meet by xor shuffles in a fixed pattern.  The
-// result (in every lane) does not depend on timing or on which warp runs it.
-__device__ __forceinline__ double loss_column_sum(const float *partials, int rows, int C, int col,
-                                                  int lane)
+// The partials are [rows][C], C = E + 1 (expert columns, then the lse^2
+// column).  Column col is summed in G = max(1, 1024 / C) row phases: phase g
+// adds rows g, g + G, g + 2G, ... in order in double, and the G phase sums are
+// then added in phase order.  G depends on C alone, so whichever threads or
+// blocks compute the phases, the bits are the same.  Phase g of column col is
+// work unit u = g * C + col (G * C <= kLossUnits units).
+constexpr int kLossBatch = 32;   // loads in flight per unit
+
+__host__ __device__ __forceinline__ int loss_phases(int C)
 {
+    return C >= kLossUnits ? 1 : kLossUnits / C;
+}
+
+// The phase sum of work unit u (u < loss_phases(C) * C).  Consecutive units
+// read consecutive columns of one row (coalesced).
+__device__ __forceinline__ double loss_phase_sum(const float *partials, int rows, int C, int u)
+{
+    const int G = loss_phases(C), col = u % C, g = u / C;
     double s = 0.0;
-#pragma unroll 4
-    for (int r = lane; r < rows; r += 32)
-        s += (double)partials[(int64_t)r * C + col];
+    for (int r0 = g; r0 < rows; r0 += kLossBatch * G) {
+        float v[kLossBatch];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        s += __shfl_xor_sync(0xffffffffu, s, o);
+        for (int i = 0; i < kLossBatch; ++i) {
+            const int r = r0 + i * G;
+            v[i] = r < rows ? partials[(int64_t)r * C + col] : 0.f;
+        }
+        // adding +0 for the rows past the end leaves s unchanged (s >= 0)
+#pragma unroll
+        for (int i = 0; i < kLossBatch; ++i)
+            s += (double)v[i];
+    }
     return s;
 }
 
-// The block's warps take the columns in turn (warp w: columns w, w + warps,
-// ...); then one thread adds the E terms in expert order.  counts[e]: the
-// assignments of expert e before capacity.  term: shared scratch [E + 1].
-__device__ __forceinline__ void block_losses(const int32_t *counts, const float *partials,
-                                             int rows, int T, int k, int E, float *aux,
-                                             float *zloss, double *term)
+// The loss terms from the phase sums ps[g * C + col] (ps in shared memory,
+// complete): the G phase sums of a column added in phase order, then one
+// thread adds the E terms in expert order.  term: shared scratch of kMaxE + 1
+// doubles.  Every thread of the block calls it.
+__device__ __forceinline__ void losses_from_phase_sums(const int32_t *counts, const double *ps,
+                                                       int T, int k, int E, float *aux,
+                                                       float *zloss, double *term)
 {
-    const int C = E + 1;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = blockDim.x >> 5;
-    for (int col = warp; col < C; col += warps) {
-        const double s = loss_column_sum(partials, rows, C, col, lane);
-        if (lane == 0)
-            term[col] = col < E ? ((double)counts[col] / ((double)T * (double)k)) * (s / (double)T)
-                                : s / (double)T;
+    const int C = E + 1, G = loss_phases(C);
+    for (int col = threadIdx.x; col < C; col += blockDim.x) {
+        double s = 0.0;
+        for (int g = 0; g < G; ++g)
+            s += ps[g * C + col];
+        term[col] = col < E ? ((double)counts[col] / ((double)T * (double)k)) * (s / (double)T)
+                            : s / (double)T;
     }
     __syncthreads();
     if (threadIdx.x == 0) {

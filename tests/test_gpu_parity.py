@@ -262,6 +262,44 @@ def test_full_size_config(name):
                               storage(inp.W3), storage(inp.W2), shape.act, storage(inp.Ws1),
                               storage(inp.Ws3), storage(inp.Ws2), tokens)
     check_y(shape, fwd.y[torch.as_tensor(tokens, device="cuda").long()], y_ref)
+    # the per-stage losses call (its partials staged through shared memory in
+    # several row tiles at these sizes) gives the forward's bits
+    cfg = moe.moe_config(shape)
+    topk, _, part, _, _ = moe.moe_route(cfg, inp.x, inp.W_r, inp.logit_bias, inp.select_bias)
+    aux_s, z_s = moe.moe_losses(cfg, moe.moe_capacity(cfg, topk).counts, part)
+    assert torch.equal(aux_s, fwd.aux) and torch.equal(z_s, fwd.zloss)
+    del inp, fwd
+    torch.cuda.empty_cache()
+
+
+LONG = {
+    # 2048 rows of loss partials with 65 columns (3 row phases, 17 shared tiles)
+    "deepseekmoe_long": shrink(CONFIGS["deepseekmoe"], T=65536, d=128, d_ff=128,
+                               d_ff_shared=128),
+    # 625 rows with 257 columns (one phase, ragged last tile and token block)
+    "deepseek_v3_long": shrink(CONFIGS["deepseek_v3"], T=20000, d=128, d_ff=128,
+                               d_ff_shared=128),
+}
+
+
+@pytest.mark.parametrize("name", list(LONG))
+def test_losses_over_many_token_blocks(name):
+    """Both losses over many token blocks: the forward (losses in its capacity
+    launch) and the per-stage call against the oracle, and bit for bit against
+    each other."""
+    shape = LONG[name]
+    inp = remove_near_ties(generate(shape, device="cuda"))
+    fwd = run_forward(inp)
+    r = oracle_route(inp)
+    cap = oracle.capacity_walk(r.topk, shape.E, shape.cf, shape.priority)
+    aux, zl = oracle.losses(r.scores, cap.counts, r.lse, shape.k, shape.score)
+    np.testing.assert_array_equal(fwd.counts.cpu().numpy(), cap.counts)
+    assert float(fwd.aux.item()) == pytest.approx(aux, rel=LOSS_RTOL)
+    assert float(fwd.zloss.item()) == pytest.approx(zl, rel=LOSS_RTOL)
+    cfg = moe.moe_config(shape)
+    topk, _, part, _, _ = moe.moe_route(cfg, inp.x, inp.W_r, inp.logit_bias, inp.select_bias)
+    aux_s, z_s = moe.moe_losses(cfg, moe.moe_capacity(cfg, topk).counts, part)
+    assert torch.equal(aux_s, fwd.aux) and torch.equal(z_s, fwd.zloss)
     del inp, fwd
     torch.cuda.empty_cache()
 
