@@ -56,7 +56,8 @@ def route_kernels(shape) -> int:
 
 def kernels_per_step(shape) -> int:
     """Kernels of ours one moe_forward launches: the router (route_kernels),
-    capacity 2 (histograms; placement with the totals and the losses),
+    capacity 2 (histograms and the loss phase sums; placement with the
+    totals and the losses),
     dispatch 1, expert FFN (bf16: the two grouped GEMMs; fp32: two, plus two
     for shared experts), combine 1 (0 for a top-1 layer without shared
     experts: GEMM2 writes y); the score-ordered capacity adds three launches
