@@ -136,6 +136,14 @@ SMALL = {
     # Mixtral-shaped K (d = 4096, d_ff = 14336), many tiles per SM pair, odd
     # trailing 128-row halves; every token compared
     "mixtral_full_k_pair": shrink(CONFIGS["mixtral"], T=2048),
+    # SM-pair tiles with GELU, and (top-1, no shared expert) the forward's
+    # gate fused into GEMM2; 5 of the 8 segments end in an odd 128-row half
+    # tile (the pair's second CTA computes rows it does not store)
+    "switch_pair": shrink(CONFIGS["switch"], T=4096, d=512, d_ff=1024),
+    # SM-pair SwiGLU tiles with two shared experts over T = 1900 rows: the
+    # shared set ends in an odd, ragged 128-row half tile
+    "deepseekmoe_pair": shrink(CONFIGS["deepseekmoe"], T=1900, d=256, d_ff=256,
+                               d_ff_shared=256, E=16),
 }
 
 
