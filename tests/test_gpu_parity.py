@@ -140,6 +140,9 @@ SMALL = {
     # gate fused into GEMM2; 5 of the 8 segments end in an odd 128-row half
     # tile (the pair's second CTA computes rows it does not store)
     "switch_pair": shrink(CONFIGS["switch"], T=4096, d=512, d_ff=1024),
+    # SM-pair SwiGLU tiles, fewer than the clusters in GEMM2 (36 tiles for 74
+    # SM pairs) and about one per cluster in GEMM1, short K
+    "mixtral_pair_few_tiles": shrink(CONFIGS["mixtral"], T=2048, d=512, d_ff=1024),
     # SM-pair SwiGLU tiles with two shared experts over T = 1900 rows: the
     # shared set ends in an odd, ragged 128-row half tile
     "deepseekmoe_pair": shrink(CONFIGS["deepseekmoe"], T=1900, d=256, d_ff=256,
