@@ -9,7 +9,9 @@
 // The sequential definition is a walk over the T*k assignments in priority
 // order with one counter per expert.  It is computed here in two launches:
 //   count  - each block of 256 tokens histograms its assignments per (rank j,
-//            expert e) in shared memory (integer atomics, order-free);
+//            expert e) in shared memory (integer atomics, order-free) and
+//            writes it per (j, e), or in token order per expert (the k ranks
+//            summed: a later block's base needs no more);
 //   place  - each block sums the histograms of the blocks before it (and,
 //            rank-major, all blocks' lower ranks): the number of assignments
 //            to each expert that come before the block in priority order;
@@ -42,7 +44,7 @@ namespace {
 constexpr int CT = kCapTokens;   // tokens per block (also the thread count)
 
 __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int T, int k, int E,
-                                                       int32_t *hist, int nblk,
+                                                       int hcols, int32_t *hist, int nblk,
                                                        const float *partials, int prows,
                                                        double *loss_ps)
 {
@@ -71,8 +73,18 @@ __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int 
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < k * E; i += CT)
-        hist[(int64_t)blockIdx.x * k * E + i] = h[i];
+    if (hcols == E) {
+        // token order: one column per expert, the k slots summed
+        for (int e = threadIdx.x; e < E; e += CT) {
+            int v = 0;
+            for (int j = 0; j < k; ++j)
+                v += h[j * E + e];
+            hist[(int64_t)blockIdx.x * E + e] = v;
+        }
+    } else {
+        for (int i = threadIdx.x; i < k * E; i += CT)
+            hist[(int64_t)blockIdx.x * k * E + i] = h[i];
+    }
 }
 
 // Column sums of the per-block histograms [nblk][cols]: before[col] = blocks
@@ -107,7 +119,8 @@ __device__ __forceinline__ void hist_sums(const int32_t *__restrict__ hist, int 
 // partials, also the two balancing losses (the forward's losses stage, in the
 // same fixed order as moe_losses).
 __device__ void capacity_totals(const int32_t *__restrict__ hist, int nblk, int k, int E,
-                                long long C, const int32_t *__restrict__ count_base, int T,
+                                int hcols, long long C, const int32_t *__restrict__ count_base,
+                                int T,
                                 int32_t *__restrict__ counts, int32_t *__restrict__ kept,
                                 int32_t *__restrict__ offsets, int32_t *__restrict__ n_dropped,
                                 const double *loss_ps, float *aux, float *zloss,
@@ -117,11 +130,12 @@ __device__ void capacity_totals(const int32_t *__restrict__ hist, int nblk, int 
     __shared__ int32_t kept_s[kMaxE];
     __shared__ double term[kMaxE + 1];
     __shared__ double ps[kLossUnits];
-    hist_sums(hist, nblk, k * E, nblk, colsum, nullptr);
+    hist_sums(hist, nblk, hcols, nblk, colsum, nullptr);
     __syncthreads();
+    const int ranks = hcols == E ? 1 : k;   // histogram rows per expert column
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int s = 0;
-        for (int j = 0; j < k; ++j)
+        for (int j = 0; j < ranks; ++j)
             s += colsum[j * E + e];
         // slots left for this batch: C, less what earlier shards of the same
         // global batch already took (count_base, sharded capacity only)
@@ -202,22 +216,17 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
     pdl_wait();   // topk from the router, the histograms from cap_count
     pdl_trigger();
     const int cols = k * E;
+    const bool token_order = priority == MOE_PRIORITY_TOKEN;
+    const int hcols = token_order ? E : cols;   // cap_count's histogram columns
     if (blockIdx.x == nblk) {
-        capacity_totals(hist, nblk, k, E, C, count_base, T, counts, kept, offsets, n_dropped,
-                        loss_ps, aux, zloss, before);
+        capacity_totals(hist, nblk, k, E, hcols, C, count_base, T, counts, kept, offsets,
+                        n_dropped, loss_ps, aux, zloss, before);
         return;
     }
-    const bool token_order = priority == MOE_PRIORITY_TOKEN;
-    hist_sums(hist, nblk, cols, blockIdx.x, before, token_order ? nullptr : total);
+    // token order: before[e] = the base of expert e (any rank)
+    hist_sums(hist, nblk, hcols, blockIdx.x, before, token_order ? nullptr : total);
     __syncthreads();
-    if (token_order) {
-        for (int e = threadIdx.x; e < E; e += CT) {
-            int s = 0;
-            for (int j = 0; j < k; ++j)
-                s += before[j * E + e];
-            total[e] = s;   // base of expert e (any rank)
-        }
-    } else {
+    if (!token_order) {
         for (int col = threadIdx.x; col < cols; col += CT) {
             const int j = col / E, e = col % E;
             int s = 0;
@@ -227,7 +236,7 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
         }
     }
     __syncthreads();
-    const int32_t *bb = token_order ? total : before;
+    const int32_t *bb = before;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int tw = blockIdx.x * CT + warp * 32;   // this warp's first token
@@ -462,9 +471,11 @@ cudaError_t launch_capacity(const moe_config &c, int64_t C, const int32_t *topk,
     // with the losses: extra count blocks for the phase sums of the partials
     const int lblk = partials ? (loss_phases(c.E + 1) * (c.E + 1) + CT - 1) / CT : 0;
     if (nblk + lblk > 0) {
+        // token order: histogram rows of one column per expert
+        const int hcols = c.priority == MOE_PRIORITY_TOKEN ? c.E : c.k * c.E;
         cudaError_t err = launch_pdl(cap_count_kernel, dim3(nblk + lblk), dim3(CT),
-                                     sizeof(int32_t) * c.k * c.E, s, topk, c.T, c.k, c.E, hist,
-                                     nblk, partials, partial_rows(c), loss_ps);
+                                     sizeof(int32_t) * c.k * c.E, s, topk, c.T, c.k, c.E, hcols,
+                                     hist, nblk, partials, partial_rows(c), loss_ps);
         if (err != cudaSuccess)
             return err;
     }

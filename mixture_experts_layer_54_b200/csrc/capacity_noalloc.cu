@@ -19,8 +19,8 @@
 
 namespace {
 
-// one int32 table: the per-block histograms, one entry per (block of 256
-// tokens, rank, expert)
+// one int32 table: the per-block histograms, room for one entry per (block
+// of 256 tokens, rank, expert) (token order uses one per (block, expert))
 constexpr int64_t kTableInts = 65536;
 static __device__ __align__(256) int32_t g_capacity_scratch[kTableInts];
 
