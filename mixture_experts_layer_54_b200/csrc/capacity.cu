@@ -89,29 +89,69 @@ __global__ void __launch_bounds__(CT) cap_count_kernel(const int32_t *topk, int 
 
 // Column sums of the per-block histograms [nblk][cols]: before[col] = blocks
 // [0, upto), and (total != nullptr) total[col] = all blocks; BATCH loads of a
-// column in flight per thread.
+// column in flight per thread.  With fewer columns than threads the blocks
+// are split into P parts (thread t: column t mod cols, blocks t / cols,
+// + P, ...) whose sums meet in shared memory (integers: exact in any order).
+// Every thread of the block calls it; it ends with the block synchronised.
 __device__ __forceinline__ void hist_sums(const int32_t *__restrict__ hist, int nblk, int cols,
                                           int upto, int32_t *before, int32_t *total)
 {
     constexpr int BATCH = 16;
+    __shared__ int32_t pb[kCapTokens], pt[kCapTokens];
     const int end = total ? nblk : upto;
-    for (int col = threadIdx.x; col < cols; col += blockDim.x) {
+    const int P = cols >= (int)blockDim.x ? 1 : (int)blockDim.x / cols;
+    if (P == 1) {
+        for (int col = threadIdx.x; col < cols; col += blockDim.x) {
+            int bsum = 0, tsum = 0;
+            for (int b0 = 0; b0 < end; b0 += BATCH) {
+                int v[BATCH];
+#pragma unroll
+                for (int i = 0; i < BATCH; ++i)
+                    v[i] = b0 + i < end ? hist[(int64_t)(b0 + i) * cols + col] : 0;
+#pragma unroll
+                for (int i = 0; i < BATCH; ++i) {
+                    bsum += b0 + i < upto ? v[i] : 0;
+                    tsum += v[i];
+                }
+            }
+            before[col] = bsum;
+            if (total)
+                total[col] = tsum;
+        }
+        __syncthreads();
+        return;
+    }
+    const int t = threadIdx.x, col = t % cols, part = t / cols;
+    if (part < P) {
         int bsum = 0, tsum = 0;
-        for (int b0 = 0; b0 < end; b0 += BATCH) {
+        for (int b0 = part; b0 < end; b0 += BATCH * P) {
             int v[BATCH];
 #pragma unroll
-            for (int i = 0; i < BATCH; ++i)
-                v[i] = b0 + i < end ? hist[(int64_t)(b0 + i) * cols + col] : 0;
+            for (int i = 0; i < BATCH; ++i) {
+                const int b = b0 + i * P;
+                v[i] = b < end ? hist[(int64_t)b * cols + col] : 0;
+            }
 #pragma unroll
             for (int i = 0; i < BATCH; ++i) {
-                bsum += b0 + i < upto ? v[i] : 0;
+                bsum += b0 + i * P < upto ? v[i] : 0;
                 tsum += v[i];
             }
         }
-        before[col] = bsum;
-        if (total)
-            total[col] = tsum;
+        pb[t] = bsum;
+        pt[t] = tsum;
     }
+    __syncthreads();
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+        int sb = 0, st = 0;
+        for (int q = 0; q < P; ++q) {
+            sb += pb[q * cols + c];
+            st += pt[q * cols + c];
+        }
+        before[c] = sb;
+        if (total)
+            total[c] = st;
+    }
+    __syncthreads();
 }
 
 // The block after the placement blocks: counts, kept, the padded segment
@@ -131,7 +171,6 @@ __device__ void capacity_totals(const int32_t *__restrict__ hist, int nblk, int 
     __shared__ double term[kMaxE + 1];
     __shared__ double ps[kLossUnits];
     hist_sums(hist, nblk, hcols, nblk, colsum, nullptr);
-    __syncthreads();
     const int ranks = hcols == E ? 1 : k;   // histogram rows per expert column
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int s = 0;
@@ -225,7 +264,6 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
     }
     // token order: before[e] = the base of expert e (any rank)
     hist_sums(hist, nblk, hcols, blockIdx.x, before, token_order ? nullptr : total);
-    __syncthreads();
     if (!token_order) {
         for (int col = threadIdx.x; col < cols; col += CT) {
             const int j = col / E, e = col % E;
