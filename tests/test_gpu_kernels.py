@@ -178,20 +178,36 @@ def test_expert_ffn_fp32_simt_against_torch():
 
 @pytest.mark.parametrize("priority", [0, 1])
 @pytest.mark.parametrize("T,E,k,cf", [(1000, 8, 2, 1.0), (777, 64, 6, 1.25), (300, 256, 8, 1.0),
-                                      (5, 4, 4, 1.0), (1, 3, 1, 1.0)])
+                                      (5, 4, 4, 1.0), (1, 3, 1, 1.0),
+                                      # many capacity blocks (64 to 256 of 256 tokens),
+                                      # a ragged last one
+                                      (65536, 8, 2, 1.0), (16384, 64, 6, 1.5),
+                                      (20000, 256, 8, 1.0)])
 def test_capacity_bit_exact_with_sequential_walk(priority, T, E, k, cf):
     """Skewed random top-k lists (distinct experts per token) against the pages'
-    one-hot cumulative-sum formulation, in integers."""
+    one-hot cumulative-sum formulation, in integers (for long lists, the same
+    positions from a stable sort by expert)."""
     rng = np.random.default_rng(T + E + priority)
     w = 1.0 / np.arange(1, E + 1) ** 1.1
-    topk = np.stack([rng.choice(E, size=k, replace=False, p=w / w.sum()) for _ in range(T)])
+    w = w / w.sum()
+    if T <= 1000:
+        topk = np.stack([rng.choice(E, size=k, replace=False, p=w) for _ in range(T)])
+    else:   # k distinct experts per token: the k smallest of exponential keys scaled by w
+        keys = rng.exponential(size=(T, E)) / w
+        topk = np.argsort(keys, axis=1)[:, :k]
     topk = topk.astype(np.int32)
     cfg = moe.moe_config(T=T, d=64, E=E, k=k, d_ff=64, dtype=1, cf=cf, priority=priority)
     C = moe.moe_capacity_value(cfg)
     out = moe.moe_capacity(cfg, torch.tensor(topk, device=DEV))
     flat = topk.reshape(-1) if priority == 0 else topk.T.reshape(-1)
-    onehot = np.eye(E, dtype=np.int64)[flat]
-    pf = np.take_along_axis(np.cumsum(onehot, axis=0), flat[:, None], axis=1)[:, 0] - 1
+    if T <= 1000:
+        onehot = np.eye(E, dtype=np.int64)[flat]
+        pf = np.take_along_axis(np.cumsum(onehot, axis=0), flat[:, None], axis=1)[:, 0] - 1
+    else:   # place within the expert's list, the list in priority order (stable sort)
+        order = np.argsort(flat, kind="stable")
+        first = np.searchsorted(flat[order], np.arange(E))
+        pf = np.empty(flat.size, dtype=np.int64)
+        pf[order] = np.arange(flat.size) - first[flat[order]]
     pos = pf.reshape(T, k) if priority == 0 else pf.reshape(k, T).T
     counts = np.bincount(flat, minlength=E)
     kept = np.minimum(counts, C)
