@@ -974,7 +974,8 @@ __global__ void __launch_bounds__(LOGIT_THREADS, 1) logits_kernel(const __grid_c
 // to 64 experts (four blocks per SM fit, so one wave; 5% faster on the
 // DeepSeekMoE shape) and NT = 1 above (eight experts per lane: two tokens per
 // warp in 16-warp blocks measured 18% slower on the DeepSeek-V3 shape).
-template <int PL, int NT>
+// ONE: a single K part (its logits read straight, no loop over parts).
+template <int PL, int NT, bool ONE>
 __global__ void __launch_bounds__(32 * kPartialTokens / NT)
     select_kernel(const __grid_constant__ RouteParams a, const float *__restrict__ partial,
                   int parts, int E_pad)
@@ -1006,8 +1007,11 @@ __global__ void __launch_bounds__(32 * kPartialTokens / NT)
             const int e = lane + 32 * i;
             float s = 0.f;
             if (e < E && tv[n]) {
-                for (int q = 0; q < parts; ++q)
-                    s += partial[((int64_t)q * a.T + tt[n]) * E_pad + e];
+                if (ONE)
+                    s = partial[(int64_t)tt[n] * E_pad + e];
+                else
+                    for (int q = 0; q < parts; ++q)
+                        s += partial[((int64_t)q * a.T + tt[n]) * E_pad + e];
                 if (a.logit_bias)
                     s += a.logit_bias[e];
             }
@@ -1253,18 +1257,28 @@ cudaError_t launch_route_tc(const moe_config &c, const void *x, const float *W_r
     if (err != cudaSuccess)
         return err;
     const unsigned rows = (unsigned)ceil_div(c.T, kPartialTokens);
+    const float *pl = plog;
+    const bool one = r.k_parts == 1;
     if (c.E <= 32)
-        err = launch_pdl(select_kernel<1, 4>, dim3(rows), dim3(32 * kPartialTokens / 4), 0, s, p,
-                         (const float *)plog, r.k_parts, r.E_pad);
+        err = one ? launch_pdl(select_kernel<1, 4, true>, dim3(rows), dim3(32 * kPartialTokens / 4),
+                               0, s, p, pl, r.k_parts, r.E_pad)
+                  : launch_pdl(select_kernel<1, 4, false>, dim3(rows),
+                               dim3(32 * kPartialTokens / 4), 0, s, p, pl, r.k_parts, r.E_pad);
     else if (c.E <= 64)
-        err = launch_pdl(select_kernel<2, 4>, dim3(rows), dim3(32 * kPartialTokens / 4), 0, s, p,
-                         (const float *)plog, r.k_parts, r.E_pad);
+        err = one ? launch_pdl(select_kernel<2, 4, true>, dim3(rows), dim3(32 * kPartialTokens / 4),
+                               0, s, p, pl, r.k_parts, r.E_pad)
+                  : launch_pdl(select_kernel<2, 4, false>, dim3(rows),
+                               dim3(32 * kPartialTokens / 4), 0, s, p, pl, r.k_parts, r.E_pad);
     else if (c.E <= 128)
-        err = launch_pdl(select_kernel<4, 1>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
-                         (const float *)plog, r.k_parts, r.E_pad);
+        err = one ? launch_pdl(select_kernel<4, 1, true>, dim3(rows), dim3(32 * kPartialTokens), 0,
+                               s, p, pl, r.k_parts, r.E_pad)
+                  : launch_pdl(select_kernel<4, 1, false>, dim3(rows), dim3(32 * kPartialTokens),
+                               0, s, p, pl, r.k_parts, r.E_pad);
     else
-        err = launch_pdl(select_kernel<8, 1>, dim3(rows), dim3(32 * kPartialTokens), 0, s, p,
-                         (const float *)plog, r.k_parts, r.E_pad);
+        err = one ? launch_pdl(select_kernel<8, 1, true>, dim3(rows), dim3(32 * kPartialTokens), 0,
+                               s, p, pl, r.k_parts, r.E_pad)
+                  : launch_pdl(select_kernel<8, 1, false>, dim3(rows), dim3(32 * kPartialTokens),
+                               0, s, p, pl, r.k_parts, r.E_pad);
     return err;
 }
 
