@@ -281,13 +281,12 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
     const int nw = max(0, min(32, T - tw));       // its tokens
     const int passes = token_order ? 1 : k;
     for (int p = 0; p < passes; ++p) {
-        const int len = token_order ? nw * k : nw;
-        // (A) this warp's assignments per expert
-        for (int i = lane; i < E; i += 32)
-            wrun[warp][i] = 0;
-        __syncwarp();
-        for (int c0 = 0; c0 < len; c0 += 32) {
-            const int n = c0 + lane;
+        const int len = token_order ? nw * k : nw;   // <= 32 kMaxK
+        // this pass's experts, entry i * 32 + lane in ev[i], all loads in flight
+        int ev[kMaxK];
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i) {
+            const int n = i * 32 + lane;
             int e = E;   // sentinel for idle lanes and invalid experts
             if (n < len) {
                 const int tl = token_order ? n / k : n, j = token_order ? n % k : p;
@@ -295,6 +294,17 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
                 if (e < 0 || e >= E)
                     e = E;
             }
+            ev[i] = e;
+        }
+        // (A) this warp's assignments per expert
+        for (int i = lane; i < E; i += 32)
+            wrun[warp][i] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i) {
+            if (i * 32 >= len)
+                break;
+            const int e = ev[i];
             const unsigned peers = __match_any_sync(0xffffffffu, e);
             if ((peers & lt_mask) == 0 && e < E)
                 wrun[warp][e] += __popc(peers);
@@ -313,16 +323,13 @@ cap_place_kernel(const int32_t *__restrict__ topk, int T, int k, int E, int prio
         }
         __syncthreads();
         // (C) positions, in priority order
-        for (int c0 = 0; c0 < len; c0 += 32) {
-            const int n = c0 + lane;
-            int e = E, tl = 0, j = 0;
-            if (n < len) {
-                tl = token_order ? n / k : n;
-                j = token_order ? n % k : p;
-                e = topk[(int64_t)(tw + tl) * k + j];
-                if (e < 0 || e >= E)
-                    e = E;
-            }
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i) {
+            if (i * 32 >= len)
+                break;
+            const int n = i * 32 + lane;
+            const int e = ev[i];
+            const int tl = token_order ? n / k : n, j = token_order ? n % k : p;
             const unsigned peers = __match_any_sync(0xffffffffu, e);
             if (n < len) {
                 const int64_t a = (int64_t)(tw + tl) * k + j;
