@@ -10,8 +10,10 @@
 // destinations, so it moves T*d + N_kept*d elements.  Combine reads the k
 // expert rows of a token, its shared-expert row (and residual) and writes y,
 // summing in fp32 in slot order.  A warp owns one token at a time (grid-stride
-// over tokens): lanes 0..k-1 look up the slots, then the row moves as 16-byte
-// vectors, four per lane in flight.
+// over tokens).  It looks up the slots of its next 32 / k tokens at once (lane
+// l: slot l mod k of the (l / k)-th of them; two dependent loads, so they are
+// paid once per 32 / k tokens) and hands each token its rows by shuffle; then
+// the rows move as 16-byte vectors, several per lane in flight.
 #include "internal.cuh"
 
 namespace moe {
@@ -20,24 +22,6 @@ namespace {
 constexpr int THREADS = 256;   // 8 warps, one token per warp at a time
 constexpr int WARPS = THREADS / 32;
 constexpr int UNROLL = 4;      // 16-byte vectors in flight per lane
-
-// The kept destinations of token t: lane j < k looks up slot j, then every lane
-// gets the k rows (or -1) by shuffle.
-__device__ __forceinline__ void slot_rows(int t, int k, int E, const int32_t *topk,
-                                          const int32_t *pos, const uint8_t *keep,
-                                          const int32_t *offsets, int lane, int64_t *rows)
-{
-    int64_t mine = -1;
-    if (lane < k) {
-        const int64_t a = (int64_t)t * k + lane;
-        const int e = topk[a];
-        if (keep[a] && e >= 0 && e < E)
-            mine = (int64_t)offsets[e] + pos[a];
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-        rows[j] = __shfl_sync(0xffffffffu, mine, j);
-}
 
 // x_perm nullable: only the slot table.  src_slot nullable: row r of a kept
 // slot gets its assignment t k + j.  zero_rows nullable: the row of a token
@@ -53,46 +37,67 @@ dispatch_vec_kernel(const uint4 *__restrict__ x, int T, int k, int E, int nvec,
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
-    for (int t = gw; t < T; t += gridDim.x * WARPS) {
-        int64_t rows[kMaxK];
-        slot_rows(t, k, E, topk, pos, keep, offsets, lane, rows);
-        bool any = false;
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            any |= j < k && rows[j] >= 0;
-        if (src_slot) {   // lane j records slot j's row
+    const int stride = gridDim.x * WARPS;
+    const int tpb = 32 / k;   // tokens whose slots one lookup round covers
+    for (int tb = gw; tb < T; tb += stride * tpb) {
+        // the slots of this warp's next tpb tokens at once: lane l takes slot
+        // l mod k of token tb + (l / k) stride
+        int64_t mine = -1;
+        {
+            const int i = lane / k, j = lane % k, t = tb + i * stride;
+            if (i < tpb && t < T) {
+                const int64_t a = (int64_t)t * k + j;
+                const int e = topk[a];
+                if (keep[a] && e >= 0 && e < E)
+                    mine = (int64_t)offsets[e] + pos[a];
+            }
+        }
+        for (int ti = 0; ti < tpb; ++ti) {
+            const int t = tb + ti * stride;
+            if (t >= T)
+                break;
+            int64_t rows[kMaxK];   // rows[j], j < k: slot j's row or -1
 #pragma unroll
             for (int j = 0; j < kMaxK; ++j)
-                if (j == lane && j < k && rows[j] >= 0)
-                    src_slot[rows[j]] = t * k + j;
-        }
-        if (!any) {
-            if (zero_rows)
-                for (int v = lane; v < nvec; v += 32)
-                    zero_rows[(int64_t)t * nvec + v] = make_uint4(0u, 0u, 0u, 0u);
-            continue;
-        }
-        if (!x_perm)
-            continue;
-        const uint4 *src = x + (int64_t)t * nvec;
-        for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
-            uint4 val[UNROLL];
+                rows[j] = __shfl_sync(0xffffffffu, mine, (ti * k + j) & 31);
+            bool any = false;
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int v = v0 + u * 32 + lane;
-                if (v < nvec)
-                    val[u] = __ldcs(src + v);
+            for (int j = 0; j < kMaxK; ++j)
+                any |= j < k && rows[j] >= 0;
+            if (src_slot) {   // lane j records slot j's row
+#pragma unroll
+                for (int j = 0; j < kMaxK; ++j)
+                    if (j == lane && j < k && rows[j] >= 0)
+                        src_slot[rows[j]] = t * k + j;
             }
-#pragma unroll
-            for (int j = 0; j < kMaxK; ++j) {
-                if (j >= k || rows[j] < 0)
-                    continue;
-                uint4 *dst = x_perm + rows[j] * nvec;
+            if (!any) {
+                if (zero_rows)
+                    for (int v = lane; v < nvec; v += 32)
+                        zero_rows[(int64_t)t * nvec + v] = make_uint4(0u, 0u, 0u, 0u);
+                continue;
+            }
+            if (!x_perm)
+                continue;
+            const uint4 *src = x + (int64_t)t * nvec;
+            for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
+                uint4 val[UNROLL];
 #pragma unroll
                 for (int u = 0; u < UNROLL; ++u) {
                     const int v = v0 + u * 32 + lane;
                     if (v < nvec)
-                        __stcs(dst + v, val[u]);
+                        val[u] = __ldcs(src + v);
+                }
+#pragma unroll
+                for (int j = 0; j < kMaxK; ++j) {
+                    if (j >= k || rows[j] < 0)
+                        continue;
+                    uint4 *dst = x_perm + rows[j] * nvec;
+#pragma unroll
+                    for (int u = 0; u < UNROLL; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        if (v < nvec)
+                            __stcs(dst + v, val[u]);
+                    }
                 }
             }
         }
@@ -163,7 +168,7 @@ template <> struct Vec<float> {
 // at least two per slot), then summed in fp32 in slot order, then the shared
 // experts and the residual.
 template <typename Elem, int KS>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 2)
 combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y_sh,
                    const float *__restrict__ gates, const int32_t *__restrict__ topk,
                    const int32_t *__restrict__ pos, const uint8_t *__restrict__ keep,
@@ -174,69 +179,99 @@ combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y
     pdl_trigger();
     constexpr int N = Vec<Elem>::N;
     constexpr int U = KS >= 4 ? 2 : 8 / KS;
+    constexpr int TPB = 32 / KS;   // tokens whose slots one lookup round covers
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
-    for (int t = gw; t < T; t += gridDim.x * WARPS) {
-        int64_t rows[kMaxK];
-        slot_rows(t, KS, E, topk, pos, keep, offsets, lane, rows);
-        const float mg = lane < KS ? gates[(int64_t)t * KS + lane] : 0.f;
-        float g[KS];
-#pragma unroll
-        for (int j = 0; j < KS; ++j)
-            g[j] = __shfl_sync(0xffffffffu, mg, j);
-        for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
-            uint4 raw[KS][U];
-#pragma unroll
-            for (int j = 0; j < KS; ++j)
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int v = v0 + u * 32 + lane;
-                    raw[j][u] = (rows[j] >= 0 && v < nvec) ? __ldcs(Y_perm + rows[j] * nvec + v)
-                                                           : make_uint4(0u, 0u, 0u, 0u);
-                }
-            float acc[U][N];
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-#pragma unroll
-                for (int i = 0; i < N; ++i)
-                    acc[u][i] = 0.f;
-            // slots in order, then the shared experts, then the residual
+    const int stride = gridDim.x * WARPS;
+    for (int tb = gw; tb < T; tb += stride * TPB) {
+        // the slots of this warp's next TPB tokens at once: lane l takes slot
+        // l mod KS of token tb + (l / KS) stride (the row or -1, and the gate)
+        int64_t mine = -1;
+        float gmine = 0.f;
+        {
+            const int i = lane / KS, j = lane % KS, t = tb + i * stride;
+            if (i < TPB && t < T) {
+                const int64_t a = (int64_t)t * KS + j;
+                const int e = topk[a];
+                if (keep[a] && e >= 0 && e < E)
+                    mine = (int64_t)offsets[e] + pos[a];
+                gmine = gates[a];
+            }
+        }
+        for (int ti = 0; ti < TPB; ++ti) {
+            const int t = tb + ti * stride;
+            if (t >= T)
+                break;
+            int64_t rows[KS];
+            float g[KS];
 #pragma unroll
             for (int j = 0; j < KS; ++j) {
-                if (rows[j] < 0)
-                    continue;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    float f[N];
-                    Vec<Elem>::load(raw[j][u], f);
-#pragma unroll
-                    for (int i = 0; i < N; ++i)
-                        acc[u][i] = fmaf(g[j], f[i], acc[u][i]);
-                }
+                rows[j] = __shfl_sync(0xffffffffu, mine, ti * KS + j);
+                g[j] = __shfl_sync(0xffffffffu, gmine, ti * KS + j);
             }
             const uint4 *extra[2] = {Y_sh ? Y_sh + (int64_t)t * nvec : nullptr,
                                      residual ? residual + (int64_t)t * nvec : nullptr};
+            for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
+                // the slot rows and the shared-expert / residual rows in flight together
+                uint4 raw[KS][U], ex[2][U];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                if (!extra[q])
-                    continue;
+                for (int j = 0; j < KS; ++j)
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        raw[j][u] = (rows[j] >= 0 && v < nvec) ? __ldcs(Y_perm + rows[j] * nvec + v)
+                                                               : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        ex[q][u] = (extra[q] && v < nvec) ? __ldcs(extra[q] + v)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
+                    }
+                float acc[U][N];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int i = 0; i < N; ++i)
+                        acc[u][i] = 0.f;
+                // slots in order, then the shared experts, then the residual
+#pragma unroll
+                for (int j = 0; j < KS; ++j) {
+                    if (rows[j] < 0)
+                        continue;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        float f[N];
+                        Vec<Elem>::load(raw[j][u], f);
+#pragma unroll
+                        for (int i = 0; i < N; ++i)
+                            acc[u][i] = fmaf(g[j], f[i], acc[u][i]);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    if (!extra[q])
+                        continue;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        if (v < nvec) {
+                            float f[N];
+                            Vec<Elem>::load(ex[q][u], f);
+#pragma unroll
+                            for (int i = 0; i < N; ++i)
+                                acc[u][i] += f[i];
+                        }
+                    }
+                }
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int v = v0 + u * 32 + lane;
-                    if (v < nvec) {
-                        float f[N];
-                        Vec<Elem>::load(__ldcs(extra[q] + v), f);
-#pragma unroll
-                        for (int i = 0; i < N; ++i)
-                            acc[u][i] += f[i];
-                    }
+                    if (v < nvec)
+                        y[(int64_t)t * nvec + v] = Vec<Elem>::store(acc[u]);
                 }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int v = v0 + u * 32 + lane;
-                if (v < nvec)
-                    y[(int64_t)t * nvec + v] = Vec<Elem>::store(acc[u]);
             }
         }
     }
