@@ -178,7 +178,9 @@ combine_vec_kernel(const uint4 *__restrict__ Y_perm, const uint4 *__restrict__ Y
     pdl_wait();   // the expert rows come from the expert GEMMs
     pdl_trigger();
     constexpr int N = Vec<Elem>::N;
-    constexpr int U = KS >= 4 ? 2 : 8 / KS;
+    // 16-byte vectors per slot row and lane in flight (k = 1: 4, so that the
+    // shared-expert and residual rows fit beside them in 128 registers)
+    constexpr int U = KS >= 4 ? 2 : (KS == 1 ? 4 : 8 / KS);
     constexpr int TPB = 32 / KS;   // tokens whose slots one lookup round covers
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * WARPS + (threadIdx.x >> 5);
